@@ -1,0 +1,403 @@
+"""Pins of the CPU oracle against facts fixed by the pages and by mathematics (no GPU needed).
+
+Each test checks the oracle against something other than itself: exact rational arithmetic, brute force
+over all 16 levels, closed forms, an independent multiprecision library (mpmath), hand-worked examples
+and invariants the AWQ pages state (the scaling identity of section 一 of the gsyq.cn AWQ page, ratio 0
+reducing to plain round-to-nearest, the noise rule of section 2.1 of the hncyxsy.com outlier page).
+"""
+from decimal import Decimal, localcontext
+from fractions import Fraction
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+
+from oracle import awq_oracle as orc
+from weight_only_quantization_act_b200 import inputs
+
+F32 = np.float32
+
+
+def nearest_f32_of_fraction(v: Fraction) -> np.float32:
+    """The float32 nearest to an exact rational (ties to even), found by exact comparison."""
+    f = F32(float(v))
+    cands = [np.nextafter(f, F32(-np.inf)), f, np.nextafter(f, F32(np.inf))]
+    best = None
+    for c in cands:
+        d = abs(Fraction(float(c)) - v)
+        if best is None or d < best[0] or (d == best[0] and int(c.view(np.uint32)) % 2 == 0):
+            best = (d, c)
+    return F32(best[1])
+
+
+def midpoints(y: np.float32):
+    lo = np.nextafter(y, F32(-np.inf))
+    hi = np.nextafter(y, F32(np.inf))
+    return (Fraction(float(lo)) + Fraction(float(y))) / 2, (Fraction(float(y)) + Fraction(float(hi))) / 2
+
+
+# ------------------------------------------------------------------------------------------------ a1
+def test_act_mean_matches_exact_rational_mean_tiny_workload():
+    X, _, _ = inputs.make_inputs(inputs.workload(1))
+    got = orc.act_mean(X)
+    xf = inputs.bf16_bits_to_f32(X)
+    N, K = X.shape
+    bad = []
+    for k in range(K):
+        exact = sum(Fraction(float(abs(v))) for v in xf[:, k]) / N
+        if nearest_f32_of_fraction(exact) != got[k]:
+            bad.append(k)
+    assert not bad, f"columns whose fp64 ordered mean does not round like the exact mean: {bad}"
+
+
+def test_act_mean_single_row_and_constant_column():
+    rng = np.random.default_rng(3)
+    row = inputs.f32_to_bf16_bits(rng.standard_normal((1, 384)).astype(F32))
+    assert np.array_equal(orc.act_mean(row), np.abs(inputs.bf16_bits_to_f32(row[0])))
+    col = np.full((1000, 128), inputs.f32_to_bf16_bits(np.array([-0.375], F32))[0], np.uint16)
+    assert np.all(orc.act_mean(col) == F32(0.375))
+
+
+def test_act_mean_takes_absolute_values_per_column():
+    x = np.zeros((3, 128), F32)
+    x[:, 5] = [-1.0, 2.0, -3.0]
+    x[:, 7] = [4.0, -4.0, 4.0]
+    got = orc.act_mean(inputs.f32_to_bf16_bits(x))
+    assert got[5] == F32(2.0) and got[7] == F32(4.0)
+    assert np.count_nonzero(got) == 2
+
+
+# ------------------------------------------------------------------------------------------------ a2
+def test_ratio_grid_is_nearest_fp32_of_j_over_n():
+    for n in (20, 7, 11):
+        for j in range(n):
+            assert orc.ratio(j, n) == nearest_f32_of_fraction(Fraction(j, n))
+    assert orc.ratio(0, 20) == 0 and orc.ratio(19, 20) < 1
+
+
+def test_pow_special_cases():
+    for a in (F32(0), F32(1e-30), F32(0.5), F32(1), F32(37.25)):
+        assert orc.cr_pow(a, F32(0)) == F32(1)
+    for j in range(1, 20):
+        r = orc.ratio(j, 20)
+        assert orc.cr_pow(F32(1), r) == F32(1)
+        assert orc.cr_pow(F32(0), r) == F32(0)
+    assert orc.cr_pow(F32(256), F32(0.25)) == F32(4)
+    assert orc.cr_pow(F32(256), F32(0.75)) == F32(64)
+    assert orc.cr_pow(F32(2.0 ** -20), F32(0.5)) == F32(2.0 ** -10)
+    assert orc.cr_pow(F32(2.0 ** 40), F32(0.75)) == F32(2.0 ** 30)
+
+
+@pytest.mark.parametrize("p", [1, 2, 3])
+def test_pow_quarter_exponents_by_exact_integer_powers(p):
+    """r = p/4 is exact in fp32: y is the correctly rounded a^(p/4) iff lo^4 < a^p < hi^4 for the
+    midpoints lo, hi around y (exact rational arithmetic, no transcendental function)."""
+    rng = np.random.default_rng(10 + p)
+    a_vals = np.concatenate([rng.random(150) * 50, rng.random(50) * 1e-3]).astype(F32)
+    r = F32(p / 4)
+    for a in a_vals:
+        if a == 0:
+            continue
+        y = orc.cr_pow(a, r)
+        lo, hi = midpoints(y)
+        ap = Fraction(float(a)) ** p
+        assert lo ** 4 < ap < hi ** 4, (a, p, y)
+
+
+def _mp_round_to_f32(y) -> np.float32:
+    f = F32(float(y))
+    best = None
+    for c in (np.nextafter(f, F32(-np.inf)), f, np.nextafter(f, F32(np.inf))):
+        d = abs(mpmath.mpf(float(c)) - y)
+        if best is None or d < best[0]:
+            best = (d, c)
+    return F32(best[1])
+
+
+def test_pow_matches_mpmath_200_bits_random():
+    rng = np.random.default_rng(21)
+    a_vals = np.concatenate([rng.random(60) * 40, 10.0 ** rng.uniform(-8, 3, 60)]).astype(F32)
+    with mpmath.workprec(200):
+        for i, a in enumerate(a_vals):
+            j = 1 + i % 19
+            r = orc.ratio(j, 20)
+            ref = _mp_round_to_f32(mpmath.power(mpmath.mpf(float(a)), mpmath.mpf(float(r))))
+            assert orc.cr_pow(a, r) == ref, (a, r)
+
+
+def near_midpoint_cases(count=12, seed=5, rel=2.0 ** -34):
+    """(a, j) pairs whose real power a^(j/20) lies within ``rel`` (relative) of a float32 midpoint,
+    screened with fp64 pow and confirmed with mpmath at 200 bits."""
+    rng = np.random.default_rng(seed)
+    found = []
+    with mpmath.workprec(200):
+        while len(found) < count:
+            a = (rng.random(200000) * 30 + 1e-3).astype(F32)
+            j = rng.integers(1, 20, a.shape[0])
+            r = (j.astype(F32) / F32(20)).astype(F32)
+            y = np.power(a.astype(np.float64), r.astype(np.float64))
+            bits = y.view(np.uint64) & np.uint64((1 << 29) - 1)
+            cand = np.nonzero(np.abs(bits.astype(np.int64) - (1 << 28)) < (1 << 14))[0]
+            for i in cand:
+                ym = mpmath.power(mpmath.mpf(float(a[i])), mpmath.mpf(float(r[i])))
+                f = F32(float(ym))
+                lo, hi = midpoints(f)
+                dist = min(abs(mpmath.mpf(lo.numerator) / lo.denominator - ym),
+                           abs(mpmath.mpf(hi.numerator) / hi.denominator - ym)) / ym
+                if dist < rel:
+                    found.append((F32(a[i]), int(j[i])))
+                if len(found) >= count:
+                    break
+    return found
+
+
+def test_pow_near_fp32_midpoints_matches_mpmath():
+    cases = near_midpoint_cases()
+    assert len(cases) >= 12
+    with mpmath.workprec(200):
+        for a, j in cases:
+            r = orc.ratio(j, 20)
+            ref = _mp_round_to_f32(mpmath.power(mpmath.mpf(float(a)), mpmath.mpf(float(r))))
+            assert orc.cr_pow(a, r) == ref, (a, j)
+
+
+def test_scale_table_closed_form_two_channels():
+    """act = [1, 4] at ratio 1/2: t = [1, 2], d = nearest fp32 of sqrt(2), s = nearest fp32 of t / d."""
+    s = orc.scale_candidates(np.array([1.0, 4.0], F32), F32(0.5))
+    with localcontext() as ctx:
+        ctx.prec = 80
+        d = nearest_f32_of_fraction(Fraction(Decimal(2).sqrt()))
+    assert s[0] == nearest_f32_of_fraction(Fraction(1) / Fraction(float(d)))
+    assert s[1] == nearest_f32_of_fraction(Fraction(2) / Fraction(float(d)))
+
+
+def test_scale_table_invariants():
+    rng = np.random.default_rng(7)
+    act = np.concatenate([rng.random(250).astype(F32) * 2, np.array([0.0, 1e-9, 35.0], F32)])
+    act = act.astype(F32)
+    T = orc.scale_table(act, 20)
+    assert T.shape == (20, act.shape[0]) and T.dtype == F32
+    assert np.all(T[0] == F32(1.0)), "ratio 0 must give scales of exactly one"
+    order = np.argsort(act, kind="stable")
+    for j in range(1, 20):
+        s = T[j]
+        prod = float(s.max()) * float(s.min())
+        assert abs(prod - 1.0) <= 4 * 2.0 ** -23, (j, prod)
+        assert np.all(np.diff(s[order]) >= 0), "scales must follow the order of the statistic"
+        # a zero statistic hits the 1e-4 floor; 1e-9 ** r does too once r > 4/9
+        assert s[-3] == s.min()
+        if j >= 9:
+            assert s[-2] == s[-3]
+        else:
+            assert s[-2] > s[-3]
+        assert s[-1] == s.max()
+
+
+# ------------------------------------------------------------------------------------------------ a3
+def test_quantizer_codes_and_error_bound_random_groups():
+    rng = np.random.default_rng(11)
+    wp = (rng.standard_normal((64, 512)) * rng.uniform(0.001, 3, (64, 1))).astype(F32)
+    wp[:8] += F32(5)              # all-positive groups: negative zero points
+    wp[8:12] -= F32(7)            # all-negative groups: zero points above 15
+    q, step, z, deq = orc.quantize_groups(wp)
+    assert np.all(q == np.rint(q)) and q.min() >= 0 and q.max() <= 15
+    assert np.all(z == np.rint(z))
+    assert (z[:8] < 0).any() and (z[8:12] > 15).any()
+    raw = np.rint(wp.reshape(64, 4, 128) / step[..., None]) + z[..., None]
+    unclipped = ((raw >= 0) & (raw <= 15)).reshape(64, 512)
+    err = np.abs(wp.astype(np.float64) - deq.astype(np.float64))
+    bound = np.repeat(step.astype(np.float64), 128, axis=1) / 2 * (1 + 2.0 ** -22)
+    assert np.all(err[unclipped] <= bound[unclipped])
+
+
+def test_quantizer_brute_force_over_all_16_levels():
+    """Given (step, z), each code is the level nearest to w' among all 16, by exact arithmetic;
+    a near-tie (exact quotient within 2 ulp of a half-integer) may go either way."""
+    rng = np.random.default_rng(12)
+    wp = (rng.standard_normal((24, 256)) * rng.uniform(0.01, 2, (24, 1))).astype(F32)
+    q, step, z, _ = orc.quantize_groups(wp)
+    for o in range(wp.shape[0]):
+        for g in range(2):
+            st = Fraction(float(step[o, g]))
+            zz = Fraction(float(z[o, g]))
+            for kk in range(128):
+                w = Fraction(float(wp[o, g * 128 + kk]))
+                dists = [abs(w - (lvl - zz) * st) for lvl in range(16)]
+                best = min(dists)
+                chosen = int(q[o, g * 128 + kk])
+                if dists[chosen] != best:
+                    quo = w / st
+                    half = Fraction(int(np.floor(float(quo)))) + Fraction(1, 2)
+                    assert abs(quo - half) <= 2 * abs(quo) * Fraction(1, 2 ** 23), (o, g, kk)
+
+
+def test_quantizer_step_and_zero_rounding_is_exact_division():
+    rng = np.random.default_rng(13)
+    wp = (rng.standard_normal((16, 384)) * 0.05).astype(F32)
+    q, step, z, _ = orc.quantize_groups(wp)
+    g = wp.reshape(16, 3, 128)
+    for o in range(16):
+        for gi in range(3):
+            mx, mn = g[o, gi].max(), g[o, gi].min()
+            rng_f = nearest_f32_of_fraction(Fraction(float(mx)) - Fraction(float(mn)))
+            st = nearest_f32_of_fraction(Fraction(float(rng_f)) / 15)
+            st = max(st, F32(1e-5))
+            assert step[o, gi] == st
+            zq = nearest_f32_of_fraction(-Fraction(float(mn)) / Fraction(float(st)))
+            assert z[o, gi] == F32(np.rint(zq)) + F32(0)
+
+
+def test_quantizer_constant_groups_use_step_floor():
+    wp = np.zeros((3, 256), F32)
+    wp[0, :128] = F32(0.3)
+    wp[1, :] = F32(-2.5)
+    q, step, z, deq = orc.quantize_groups(wp)
+    assert np.all(step == F32(1e-5))
+    assert np.all(q == 0)
+    assert np.all(np.abs(deq.astype(np.float64) - wp) <= 0.5e-5 * (1 + 1e-6))
+    assert not np.signbit(z).any() or np.all(z[np.signbit(z)] != 0), "zero points must not be -0"
+    assert np.all(np.signbit(z[2]) == False)  # noqa: E712
+
+
+def test_quantizer_noise_rms_is_step_over_sqrt12():
+    """Uniform rounding noise has standard deviation step/sqrt(12) (section 2.1 of the hncyxsy.com outlier
+    page); checked within 5% on groups whose values are spread over many levels."""
+    rng = np.random.default_rng(14)
+    wp = rng.uniform(-1, 1, (512, 1024)).astype(F32)
+    q, step, z, deq = orc.quantize_groups(wp)
+    err = (wp.astype(np.float64) - deq).reshape(512, 8, 128) / step[..., None].astype(np.float64)
+    rms = np.sqrt(np.mean(err ** 2))
+    assert abs(rms - 1 / np.sqrt(12)) < 0.05 / np.sqrt(12)
+
+
+def on_grid_weight(O, K, seed):
+    """W = (q - z) * 2^-7 with levels 0 and 15 present in every group and z in [0, 15] per group."""
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, 16, (O, K))
+    q[:, 0::128] = 0
+    q[:, 1::128] = 15
+    z = np.repeat(rng.integers(0, 16, (O, K // 128)), 128, axis=1)
+    return inputs.f32_to_bf16_bits(((q - z) * 2.0 ** -7).astype(F32))
+
+
+def test_on_grid_weight_gives_zero_loss_at_ratio_zero():
+    W = on_grid_weight(96, 256, 15)
+    X = inputs.random_bf16((200, 256), 16, outliers=3, factor=40)
+    res = orc.search(X, W, n_grid=20)
+    assert res["losses"][0] == 0.0
+    assert res["best_j"] == 0
+    w_hat, _, _, _ = orc.pseudo_quantize(W, np.ones(256, F32))
+    assert np.array_equal(w_hat, inputs.bf16_bits_to_f32(W))
+
+
+def torch_plain_rtn(w_f32: np.ndarray) -> np.ndarray:
+    """Independent plain round-to-nearest INT4 (no scaling), written with torch float32 ops."""
+    w = torch.from_numpy(w_f32.copy()).reshape(-1, 128)
+    hi = w.amax(dim=1, keepdim=True)
+    lo = w.amin(dim=1, keepdim=True)
+    st = torch.clamp((hi - lo) / 15.0, min=float(np.float32(1e-5)))
+    zp = torch.round(-lo / st)
+    q = torch.clamp(torch.round(w / st) + zp, 0, 15)
+    return ((q - zp) * st).reshape(w_f32.shape).numpy()
+
+
+def test_ratio_zero_equals_plain_rtn():
+    wl = inputs.workload(1)
+    X, W, _ = inputs.make_inputs(wl)
+    res = orc.search(X, W, n_grid=20)
+    rtn = torch_plain_rtn(inputs.bf16_bits_to_f32(W))
+    assert res["losses"][0] == orc.loss_of(X, W, rtn)
+    w_hat, _, _, _ = orc.pseudo_quantize(W, res["table"][0])
+    assert np.array_equal(w_hat, rtn)
+
+
+def test_awq_beats_rtn_with_outlier_channels():
+    """The pages' claim (gsyq.cn AWQ page, section 三): scaling protects outlier channels, so some
+    ratio beats plain RTN on activations with outliers."""
+    X, W, _ = inputs.make_inputs(inputs.workload(1))
+    res = orc.search(X, W, n_grid=20)
+    assert res["best_j"] > 0
+    assert res["losses"][res["best_j"]] < 0.9 * res["losses"][0]
+
+
+# ------------------------------------------------------------------------------------------------ a4
+def test_scaling_identity_without_quantization():
+    """X W^T == (X diag(s)^-1)(diag(s) W)^T (section 一 of the gsyq.cn AWQ page), in fp64."""
+    X = inputs.random_bf16((96, 256), 31, outliers=2, factor=30)
+    W = inputs.random_bf16((80, 256), 32, scale=0.02)
+    act = orc.act_mean(X)
+    s = orc.scale_candidates(act, orc.ratio(13, 20)).astype(np.float64)
+    x = inputs.bf16_bits_to_f32(X).astype(np.float64)
+    w = inputs.bf16_bits_to_f32(W).astype(np.float64)
+    ref = x @ w.T
+    alt = (x / s[None, :]) @ (w * s[None, :]).T
+    assert np.max(np.abs(ref - alt)) <= 1e-12 * np.max(np.abs(ref))
+    # with an identity quantizer the oracle's scale/unscale round trip leaves only fp32 rounding
+    w_hat = ((inputs.bf16_bits_to_f32(W) * s.astype(F32)[None, :]).astype(F32) / s.astype(F32)[None, :])
+    assert np.max(np.abs(w_hat - inputs.bf16_bits_to_f32(W))) <= 2.0 ** -23 * np.abs(w).max()
+    assert orc.loss_of(X, W, w_hat) < 1e-10 * orc.loss_of(X, W, np.zeros_like(w_hat))
+
+
+def test_loss_delta_form_equals_two_gemm_form():
+    X = inputs.random_bf16((384, 256), 41, outliers=3, factor=50)
+    W = inputs.random_bf16((192, 256), 42, scale=0.02)
+    s = orc.scale_candidates(orc.act_mean(X), orc.ratio(9, 20))
+    w_hat, _, _, _ = orc.pseudo_quantize(W, s)
+    x = inputs.bf16_bits_to_f32(X).astype(np.float64)
+    w = inputs.bf16_bits_to_f32(W).astype(np.float64)
+    two = np.mean((x @ w.T - x @ w_hat.astype(np.float64).T) ** 2)
+    assert abs(orc.loss_of(X, W, w_hat) - two) <= 1e-12 * two
+
+
+def test_loss_hand_example_mean_normalisation():
+    """One off-grid weight, a unit activation on its channel: the loss is err^2 / (N * O)."""
+    W = on_grid_weight(2, 128, 51).astype(np.uint16)
+    wf = inputs.bf16_bits_to_f32(W).copy()
+    k = 5
+    wf[1, k] = wf[1, k] + F32(2.0 ** -9)         # a quarter step off the grid, min/max unchanged
+    assert wf[1, k] < wf[1].max() and wf[1, k] > wf[1].min()
+    W2 = inputs.f32_to_bf16_bits(wf)
+    x = np.zeros((3, 128), F32)
+    x[0, k] = 1.0
+    X = inputs.f32_to_bf16_bits(x)
+    w_hat, _, _, _ = orc.pseudo_quantize(W2, np.ones(128, F32))
+    assert orc.loss_of(X, W2, w_hat) == (2.0 ** -9) ** 2 / (3 * 2)
+
+
+# ------------------------------------------------------------------------------------------------ a5
+def test_argmin_first_minimum_wins():
+    assert orc.argmin_first([3.0, 1.0, 1.0, 2.0]) == 1
+    assert orc.argmin_first([1.0, 1.0]) == 0
+    assert orc.argmin_first([5.0, 4.0, 3.0, 3.0, 3.0]) == 2
+    assert orc.argmin_first([0.5]) == 0
+    assert orc.argmin_first([2.0, 1.0, 0.25, 0.25 + 1e-18, 0.25]) == 2
+
+
+# ------------------------------------------------------------------------------------------------ a6
+def test_pack_layout_and_round_trip():
+    q = np.zeros((2, 16), np.uint8)
+    q[0, :8] = np.arange(8)
+    q[1, 8] = 15
+    words = orc.pack_codes(q)
+    assert words[0, 0] == 0x76543210 and words[0, 1] == 0
+    assert words[1, 0] == 0 and words[1, 1] == 0x0000000F
+    rng = np.random.default_rng(61)
+    q = rng.integers(0, 16, (33, 256)).astype(np.uint8)
+    assert np.array_equal(orc.unpack_codes(orc.pack_codes(q), 256), q)
+
+
+def test_shared_input_concatenation_is_one_search():
+    """Several linears on one input share one scale (NormLinearSubgraph on the msModelSlim AWQ page):
+    the loss of the stacked weight is the row-weighted mean of the per-linear losses."""
+    X = inputs.random_bf16((160, 256), 71, outliers=2, factor=60)
+    Wq = inputs.random_bf16((128, 256), 72, scale=0.02)
+    Wk = inputs.random_bf16((64, 256), 73, scale=0.02)
+    W = np.concatenate([Wq, Wk])
+    act = orc.act_mean(X)
+    T = orc.scale_table(act, 20)
+    res = orc.search(X, W, n_grid=20, act=act, table=T)
+    for j in (0, 7, 19):
+        lq = orc.loss_of(X, Wq, orc.pseudo_quantize(Wq, T[j])[0])
+        lk = orc.loss_of(X, Wk, orc.pseudo_quantize(Wk, T[j])[0])
+        assert abs(res["losses"][j] - (128 * lq + 64 * lk) / 192) <= 1e-12 * res["losses"][j]
