@@ -1,0 +1,424 @@
+"""Benchmark of the AWQ scale search on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
+
+A step is one pass of the whole path over one layer: the activation statistic, the search (scale table,
+weight-error producer, tensor-core loss GEMM, argmin) and the packed INT4 artefact at the best scales.
+Inputs are resident in HBM when a step starts; L2 is flushed between steps (a 512 MiB write). The
+metric is candidates/s (n_grid candidates per step); the loss GEMM is also timed alone (events recorded
+around its launch inside the library) for the roofline. ``e2e`` repeats the measurement through the
+public Python API with pinned host buffers: H2D of X and W, the path, D2H of codes/steps/zeros/scales/
+losses/best_j, all inside the timed region.
+
+With N > 1 (torchrun) every rank quantizes its own layer (independent replicas, no data exchange); the
+time is the max over ranks and ``value`` counts every rank's candidates. ``--impl reference`` times the
+CPU oracle on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "AWQ search candidates/sec per layer and effective TFLOP/s vs BF16 peak"
+UNIT = "candidates/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_SOURCES = ["kernel_loss_gemm.cuh", "ptx.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "weight_only_quantization_act_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: int):
+    """Per-launch DRAM bytes of the loss GEMM from the committed ncu summary, if it was taken on the
+    current kernel source (same hash); otherwise None."""
+    path = os.path.join(ROOT, "profiles", f"loss_gemm_workload{workload}.md")
+    if not os.path.exists(path):
+        return None
+    src_hash, traffic = None, None
+    with open(path) as f:
+        for line in f:
+            if line.startswith("kernel_source_sha256_16:"):
+                src_hash = line.split(":", 1)[1].strip()
+            if line.startswith("dram_bytes_per_launch:"):
+                traffic = float(line.split(":", 1)[1].strip())
+    if src_hash != gemm_source_hash():
+        return None
+    return traffic
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------ oracle arm
+def oracle_sample(wl, X, W, j_list=(0, 10), tokens=512):
+    """Time the oracle on a bounded sample of the workload and extrapolate to candidates/s.
+
+    Sample: the statistic over all N tokens; for each sampled ratio j one scale-table row (correctly
+    rounded powers over K), the quantizer over the full W, and the fp64 loss GEMM on the first `tokens`
+    tokens, whose time is scaled by N / tokens (the loss GEMM is linear in N)."""
+    from oracle import awq_oracle as orc
+
+    t0 = time.perf_counter()
+    act = orc.act_mean(X)
+    t_act = time.perf_counter() - t0
+    t_scale = t_quant = t_loss = 0.0
+    for j in j_list:
+        t0 = time.perf_counter()
+        s = orc.scale_candidates(act, orc.ratio(j, wl.n_grid))
+        t1 = time.perf_counter()
+        w_hat, _, _, _ = orc.pseudo_quantize(W, s)
+        t2 = time.perf_counter()
+        orc.loss_of(X[:tokens], W, w_hat)
+        t3 = time.perf_counter()
+        t_scale += t1 - t0
+        t_quant += t2 - t1
+        t_loss += t3 - t2
+    n = len(j_list)
+    per_cand = (t_scale + t_quant + t_loss * (wl.N / tokens)) / n
+    per_layer = t_act + wl.n_grid * per_cand
+    wall = t_act + t_scale + t_quant + t_loss
+    return {
+        "value": wl.n_grid / per_layer,
+        "unit": UNIT,
+        "cores": int(os.cpu_count() or 1),
+        "kind": "oracle",
+        "sample": (f"workload {wl.number}: statistic over all {wl.N} tokens; {n} of {wl.n_grid} ratios "
+                   f"(scale row + quantizer over full W + fp64 loss GEMM on the first {tokens} tokens, "
+                   f"loss time scaled by {wl.N}/{tokens}); extrapolated to one layer of {wl.n_grid} candidates; "
+                   f"sample wall {wall:.1f} s"),
+        "threads": _blas_threads(),
+    }
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return sum(int(i.get("num_threads", 0)) for i in threadpool_info() if i.get("user_api") == "blas") or None
+    except Exception:
+        return None
+
+
+def run_reference(args, rank, world):
+    from weight_only_quantization_act_b200 import inputs
+
+    if rank != 0:
+        return
+    wl = inputs.workload(args.workload)
+    X, W, _ = inputs.make_inputs(wl)
+    for _ in range(args.warmup):
+        oracle_sample(wl, X, W, j_list=(0,), tokens=256)
+    vals, t_total = [], 0.0
+    res = None
+    for k in range(args.steps):
+        t0 = time.perf_counter()
+        res = oracle_sample(wl, X, W, j_list=((5 * k) % wl.n_grid,), tokens=256)
+        t_total += time.perf_counter() - t0
+        vals.append(res["value"])
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.n_grid / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(wl, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": res["cores"], "kind": "oracle",
+                         "sample": res["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, gpus):
+    return {"workload": f"AWQ search, workload {wl.number}: {wl.name}", "N": wl.N, "K": wl.K, "O": wl.O,
+            "out_rows": list(wl.out_rows), "group": wl.group, "n_grid": wl.n_grid,
+            "parallelism": f"replicas x{gpus}" if gpus > 1 else "single GPU",
+            "l2": "flushed between steps (512 MiB write)"}
+
+
+# ------------------------------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from weight_only_quantization_act_b200 import awq, inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    awq.load_library()
+    wl = inputs.workload(args.workload)
+    # each rank quantizes its own layer: same shapes, its own draw
+    seed_wl = wl if rank == 0 else dataclasses.replace(wl, number=wl.number + 1000 * rank)
+    X, W, _ = inputs.make_inputs(seed_wl)
+    Xh = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16)
+    Wh = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16)
+    Xd, Wd = Xh.to(dev), Wh.to(dev)
+    N, K, O, J = wl.N, wl.K, wl.O, wl.n_grid
+    stream = torch.cuda.current_stream()
+
+    act = torch.empty(K, dtype=torch.float32, device=dev)
+    act_ws = torch.empty(awq.act_stats_workspace_size(N, K), dtype=torch.uint8, device=dev)
+    res = awq.search(Xd, Wd, awq.act_stats(Xd, out=act, workspace=act_ws), n_grid=J)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        awq.act_stats(Xd, out=act, workspace=act_ws)
+        awq.search(Xd, Wd, act, n_grid=J, workspace=res.workspace, out=res)
+        return awq.quantize_pack(Wd, res.scales)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for e in ev:
+        for x in e:
+            x.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(args.steps):
+        flush.zero_()
+        e = ev[k]
+        e[0].record(stream)
+        awq.act_stats(Xd, out=act, workspace=act_ws)
+        e[1].record(stream)
+        awq.set_profile_events(e[2], e[3])
+        awq.search(Xd, Wd, act, n_grid=J, workspace=res.workspace, out=res)
+        awq.set_profile_events(None, None)
+        e[4].record(stream)
+        awq.quantize_pack(Wd, res.scales)
+        e[5].record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+
+    step_ms = [e[0].elapsed_time(e[5]) for e in ev]
+    act_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    search_ms = [e[1].elapsed_time(e[4]) for e in ev]
+    gemm_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    pack_ms = [e[4].elapsed_time(e[5]) for e in ev]
+    total_ms = float(np.sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # correctness guard on the timed result (cheap): a valid ratio and finite losses
+    best = int(res.best_j.item())
+    assert 0 <= best < J and torch.isfinite(res.losses).all()
+
+    e2e = None if args.no_e2e else measure_e2e(args, Xh, Wh, dev, J)
+    if world > 1:
+        e2e_t = torch.tensor([e2e["ms"] if e2e else 0.0], dtype=torch.float64, device=dev)
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+        if e2e:
+            e2e["ms"] = float(e2e_t.item())
+
+    if rank != 0:
+        return
+    peaks, peaks_src = load_peaks()
+    ms_per_step = total_ms / args.steps
+    value = J * world * args.steps / (total_ms / 1e3)
+    flops = J * 2.0 * N * O * K
+    gemm_avg_s = float(np.mean(gemm_ms)) / 1e3
+    achieved_tflops = flops / gemm_avg_s / 1e12
+    traffic = profiled_traffic(wl.number)
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = oracle_sample(wl, X, W)
+        cpu.pop("threads", None)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(wl, world),
+        "effective_tflops": flops / (ms_per_step / 1e3) / 1e12,
+        "breakdown_ms": {"act_stats": float(np.mean(act_ms)), "search": float(np.mean(search_ms)),
+                         "loss_gemm": float(np.mean(gemm_ms)), "quantize_pack": float(np.mean(pack_ms))},
+        "roofline": {"bound": "tensor", "kernel": "loss_gemm_kernel", "achieved": achieved_tflops,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved_tflops / peaks["bf16_tflops"],
+                     "frac_of_sustained": achieved_tflops / peaks["bf16_tflops_sustained"],
+                     "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)" if peaks_src == "measured"
+                     else "fallback 1.59 PFLOP/s",
+                     "traffic": traffic, "algorithmic_flops_per_launch": flops},
+        "hbm": {"act_stats_gbs": (2.0 * N * K + 4.0 * K) / (np.mean(act_ms) / 1e3) / 1e9,
+                "quantize_pack_gbs": (2.0 * O * K + 4.0 * K + O * K / 2.0 + 8.0 * O * K / 128)
+                / (np.mean(pack_ms) / 1e3) / 1e9,
+                "peak_gbs": peaks.get("hbm_gbs")},
+        "gpu_launches": 8 * args.steps,
+        "clocks": clocks,
+        "best_j": best,
+        "wall_s": wall,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if e2e is not None:
+        line["e2e"] = {"value": J * world / (e2e["ms"] / 1e3), "unit": UNIT,
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": e2e["ms"]}
+    print(json.dumps(line), flush=True)
+
+
+def measure_e2e(args, Xh, Wh, dev, J):
+    """Same path through the public API with pinned host buffers; H2D and D2H inside the timed region."""
+    import torch
+
+    from weight_only_quantization_act_b200 import awq
+
+    Xp, Wp = Xh.pin_memory(), Wh.pin_memory()
+    stream = torch.cuda.current_stream()
+
+    def one():
+        Xd = Xp.to(dev, non_blocking=True)
+        Wd = Wp.to(dev, non_blocking=True)
+        out = awq.quantize_layer(Xd, Wd, n_grid=J)
+        host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()
+                if k in ("codes", "steps", "zeros", "scales", "losses", "best_j")}
+        for k, h in host.items():
+            h.copy_(out[k], non_blocking=True)
+        return host
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    steps = max(2, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        host = one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = Xh.numel() * 2 + Wh.numel() * 2
+    d2h = sum(h.numel() * h.element_size() for h in host.values())
+    return {"ms": ms, "h2d": int(h2d), "d2h": int(d2h)}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group(backend="nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

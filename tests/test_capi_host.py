@@ -1,0 +1,121 @@
+"""Host-side checks of libawq that need no GPU: the library loads, exports every entry point that
+include/awq.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from weight_only_quantization_act_b200 import awq, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "awq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return awq.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(awq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("awq_act_stats", "awq_search", "awq_quantize_pack", "awq_search_workspace_size",
+                     "awq_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", awq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\w+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(lib, n)
+    assert set(awq.SIGNATURES) == set(declared_functions())
+    # nothing else leaks out of the library (hidden visibility)
+    assert all(e.startswith("awq_") for e in exported if not e.startswith("_")), sorted(exported)[:20]
+
+
+def test_version_and_sizes(lib):
+    assert lib.awq_version() == 100
+    assert lib.awq_search_workspace_size(512, 256, 256, 128, 20) > 20 * 256 * 256 * 2
+    assert lib.awq_search_workspace_size(512, 256, 256, 64, 20) == 0
+    assert lib.awq_act_stats_workspace_size(512, 256) >= 2 * 256 * 8
+    assert lib.awq_scale_table_workspace_size(256, 65) == 0
+
+
+def test_layout_geometry(lib):
+    lay = awq.search_layout(300, 384, 600, 20)
+    assert (lay.tile_n, lay.tile_o) == (128, 256)
+    assert (lay.tiles_n, lay.tiles_o) == (3, 3)
+    assert lay.partials_offset % 8 == 0
+    assert lay.workspace_bytes == awq.search_workspace_size(300, 384, 600, 20)
+
+
+FAKE = ctypes.c_void_p(1 << 20)        # never dereferenced: every call below fails validation first
+MISALIGNED = ctypes.c_void_p((1 << 20) + 4)
+
+
+def status_and_message(lib, rc):
+    return rc, lib.awq_last_error().decode()
+
+
+def test_search_rejects_bad_arguments(lib):
+    ws = 1 << 30
+    common = dict(N=512, K=256, ldx=256, O=256, ldw=256)
+
+    def call(X=FAKE, N=512, K=256, ldx=256, W=FAKE, O=256, ldw=256, act=FAKE, group=128, n_grid=20, flags=0,
+             wsp=FAKE, wsb=ws, losses=FAKE, best=FAKE, scales=FAKE):
+        return lib.awq_search_ex(X, N, K, ldx, W, O, ldw, act, group, n_grid, flags, wsp, wsb, losses, best,
+                                 scales, None)
+
+    assert call(group=64) == 2
+    assert call(n_grid=0) == 1 and call(n_grid=65) == 1
+    assert call(X=None) == 1
+    assert call(X=MISALIGNED) == 1
+    assert call(K=200, ldx=200, ldw=200) == 1            # not a multiple of 128
+    assert call(ldx=100) == 1                            # stride below K
+    assert call(ldx=260) == 1                            # stride not a multiple of 8
+    assert call(N=0) == 1 and call(O=0) == 1
+    assert call(act=None) == 1 and call(scales=None) == 1
+    assert call(flags=0x8) == 1
+    assert call(wsp=None) == 3
+    assert call(wsb=1000) == 3
+    rc, msg = status_and_message(lib, call(wsb=1000))
+    assert rc == 3 and "workspace" in msg
+    assert common
+
+
+def test_other_entry_points_reject_bad_arguments(lib):
+    assert lib.awq_act_stats(None, 10, 256, 256, FAKE, 1 << 20, FAKE, None) == 1
+    assert lib.awq_act_stats(FAKE, 10, 255, 256, FAKE, 1 << 20, FAKE, None) == 1
+    assert lib.awq_act_stats(FAKE, 10, 256, 256, FAKE, 8, FAKE, None) == 3
+    assert lib.awq_act_stats(FAKE, 0, 256, 256, FAKE, 1 << 20, FAKE, None) == 1
+    assert lib.awq_quantize_pack(FAKE, 4, 256, 256, FAKE, 32, FAKE, FAKE, FAKE, None) == 2
+    assert lib.awq_quantize_pack(FAKE, 4, 192, 192, FAKE, 128, FAKE, FAKE, FAKE, None) == 1
+    assert lib.awq_quantize_pack(FAKE, 4, 256, 256, None, 128, FAKE, FAKE, FAKE, None) == 1
+    assert lib.awq_quantize_pack_ex(FAKE, 4, 256, 256, FAKE, 128, 0x2, FAKE, FAKE, FAKE, None) == 1
+    assert lib.awq_scale_table(FAKE, 256, 0, 0, FAKE, 1 << 20, FAKE, None) == 1
+    assert lib.awq_scale_table(FAKE, 256, 20, 0x1, FAKE, 1 << 20, FAKE, None) == 1
+    assert lib.awq_scale_table(FAKE, 256, 20, 0, FAKE, 4, FAKE, None) == 3
+    assert lib.awq_search_status(None, 0, None) == 3
+    assert lib.awq_search_get_layout(10, 256, 10, 128, 20, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = awq._lib
+    try:
+        awq._lib = None
+        with pytest.raises(RuntimeError, match="libawq.so not found"):
+            awq.load_library(str(tmp_path / "missing.so"))
+    finally:
+        awq._lib = saved

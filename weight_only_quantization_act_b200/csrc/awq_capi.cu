@@ -1,0 +1,401 @@
+// awq_capi.cu - host side of libawq: argument validation, workspace layout, TMA descriptors and the
+// launch sequence of every entry point declared in include/awq.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "awq.h"
+#include "kernel_loss_gemm.cuh"
+#include "kernels_simple.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+thread_local cudaEvent_t g_prof_before = nullptr;
+thread_local cudaEvent_t g_prof_after = nullptr;
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+
+awq_status fail(awq_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+awq_status ok() {
+  g_err[0] = '\0';
+  return AWQ_OK;
+}
+
+#define AWQ_CUDA(call)                                                                        \
+  do {                                                                                        \
+    cudaError_t e_ = (call);                                                                  \
+    if (e_ != cudaSuccess) return fail(AWQ_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+struct DeviceInfo {
+  int sms = 0;
+  int cc_major = 0;
+  bool gemm_attr_set = false;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+awq_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  AWQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(AWQ_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.sms == 0) {
+    AWQ_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    AWQ_CUDA(cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev));
+  }
+  if (d.cc_major != 10)
+    return fail(AWQ_ERR_UNSUPPORTED, "compute capability %d.x: this library is built for sm_100a", d.cc_major);
+  if (!d.gemm_attr_set) {
+    AWQ_CUDA(cudaFuncSetAttribute(awq::lg::loss_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::lg::SMEM_BYTES));
+    d.gemm_attr_set = true;
+  }
+  *out = &d;
+  return AWQ_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 [rows, cols] with row stride ld (elements), tiles of box_rows x 64 columns, 128 B swizzle.
+awq_status make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(awq::lg::BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return AWQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ----------------------------------------------------------------------------- workspace layouts
+struct ActLayout {
+  int n_chunks;
+  size_t bytes;
+};
+ActLayout act_layout(int64_t N, int64_t K) {
+  ActLayout l;
+  l.n_chunks = static_cast<int>((N + awq::kActChunk - 1) / awq::kActChunk);
+  l.bytes = align_up(static_cast<size_t>(l.n_chunks) * static_cast<size_t>(K) * sizeof(double), 256);
+  return l;
+}
+
+struct ScaleLayout {
+  int nblk;
+  size_t part_off, bytes;
+};
+ScaleLayout scale_layout(int64_t K, int n_grid) {
+  ScaleLayout l;
+  l.nblk = static_cast<int>((K + awq::kScaleThreads - 1) / awq::kScaleThreads);
+  l.part_off = 0;
+  l.bytes = align_up(static_cast<size_t>(n_grid) * l.nblk * sizeof(float2), 256);
+  return l;
+}
+
+struct SearchLayout {
+  int64_t O_pad, tiles_n, tiles_o;
+  size_t status_off, table_off, rtable_off, spart_off, partials_off, dw_off, bytes;
+  ScaleLayout sl;
+};
+SearchLayout search_layout(int64_t N, int64_t K, int64_t O, int n_grid) {
+  SearchLayout l;
+  l.O_pad = (O + awq::lg::BN - 1) / awq::lg::BN * awq::lg::BN;
+  l.tiles_n = (N + awq::lg::BM - 1) / awq::lg::BM;
+  l.tiles_o = l.O_pad / awq::lg::BN;
+  l.sl = scale_layout(K, n_grid);
+  size_t off = 0;
+  l.status_off = off;
+  off += 256;
+  l.table_off = off;
+  off = align_up(off + static_cast<size_t>(n_grid) * K * sizeof(float), 256);
+  l.rtable_off = off;
+  off = align_up(off + static_cast<size_t>(n_grid) * K * sizeof(float), 256);
+  l.spart_off = off;
+  off = align_up(off + l.sl.bytes, 256);
+  l.partials_off = off;
+  off = align_up(off + static_cast<size_t>(n_grid) * l.tiles_o * l.tiles_n * 4 * sizeof(double), 1024);
+  l.dw_off = off;
+  off = align_up(off + static_cast<size_t>(n_grid) * l.O_pad * K * 2, 1024);
+  l.bytes = off;
+  return l;
+}
+
+awq_status check_group(int group) {
+  if (group != 128) return fail(AWQ_ERR_UNSUPPORTED, "group size %d: only 128 is supported", group);
+  return AWQ_OK;
+}
+
+awq_status check_grid(int n_grid) {
+  if (n_grid < 1 || n_grid > AWQ_MAX_N_GRID)
+    return fail(AWQ_ERR_INVALID_ARG, "n_grid %d outside [1, %d]", n_grid, AWQ_MAX_N_GRID);
+  return AWQ_OK;
+}
+
+awq_status check_matrix(const char* name, const void* p, int64_t rows, int64_t K, int64_t ld) {
+  if (p == nullptr) return fail(AWQ_ERR_INVALID_ARG, "%s is null", name);
+  if (!aligned16(p)) return fail(AWQ_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  if (rows < 1 || K < 1) return fail(AWQ_ERR_INVALID_ARG, "%s has an empty shape (%lld x %lld)", name,
+                                     static_cast<long long>(rows), static_cast<long long>(K));
+  if (rows >= (1ll << 31) || K >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "%s is too large", name);
+  if (ld < K || ld % 8 != 0)
+    return fail(AWQ_ERR_INVALID_ARG, "%s row stride %lld must be >= K (%lld) and a multiple of 8", name,
+                static_cast<long long>(ld), static_cast<long long>(K));
+  return AWQ_OK;
+}
+
+awq_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(AWQ_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return AWQ_OK;
+}
+
+#define AWQ_TRY(x)                      \
+  do {                                  \
+    awq_status s_ = (x);                \
+    if (s_ != AWQ_OK) return s_;        \
+  } while (0)
+
+awq_status launch_scale_table(const float* act, int64_t K, int n_grid, bool exact_pow, float* table, float* rtable,
+                              float2* part, cudaStream_t st) {
+  const int nblk = static_cast<int>((K + awq::kScaleThreads - 1) / awq::kScaleThreads);
+  dim3 grid(nblk, n_grid);
+  awq::scale_pow_kernel<<<grid, awq::kScaleThreads, 0, st>>>(act, K, n_grid, exact_pow ? 1 : 0, table, part);
+  AWQ_TRY(check_launch("scale_pow_kernel"));
+  awq::scale_normalize_kernel<<<grid, awq::kScaleThreads, 0, st>>>(table, rtable, part, K, nblk);
+  return check_launch("scale_normalize_kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* awq_last_error(void) { return g_err; }
+
+int awq_version(void) { return 100; }
+
+void awq_set_profile_events(void* before_loss_gemm, void* after_loss_gemm) {
+  g_prof_before = static_cast<cudaEvent_t>(before_loss_gemm);
+  g_prof_after = static_cast<cudaEvent_t>(after_loss_gemm);
+}
+
+void awq_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns < 1000000ull ? 1000000ull : ns); }
+
+size_t awq_act_stats_workspace_size(int64_t N, int64_t K) {
+  if (N < 1 || K < 1) return 0;
+  return act_layout(N, K).bytes;
+}
+
+awq_status awq_act_stats(const void* X, int64_t N, int64_t K, int64_t ldx, void* workspace, size_t ws_bytes,
+                         float* act_mean, awq_stream_t stream) {
+  AWQ_TRY(check_matrix("X", X, N, K, ldx));
+  if (K % 2 != 0) return fail(AWQ_ERR_INVALID_ARG, "K must be even");
+  if (act_mean == nullptr) return fail(AWQ_ERR_INVALID_ARG, "act_mean is null");
+  const ActLayout l = act_layout(N, K);
+  if (workspace == nullptr || ws_bytes < l.bytes)
+    return fail(AWQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", l.bytes, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(AWQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  DeviceInfo* d = nullptr;
+  AWQ_TRY(device_info(&d));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  double* part = static_cast<double*>(workspace);
+  dim3 grid(static_cast<unsigned>((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock), l.n_chunks);
+  awq::act_chunk_sums_kernel<<<grid, awq::kActThreads, 0, st>>>(static_cast<const uint16_t*>(X), N, K, ldx, part);
+  AWQ_TRY(check_launch("act_chunk_sums_kernel"));
+  awq::act_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(part, N, K, l.n_chunks, act_mean);
+  AWQ_TRY(check_launch("act_finalize_kernel"));
+  return ok();
+}
+
+size_t awq_scale_table_workspace_size(int64_t K, int n_grid) {
+  if (K < 1 || n_grid < 1 || n_grid > AWQ_MAX_N_GRID) return 0;
+  return scale_layout(K, n_grid).bytes;
+}
+
+awq_status awq_scale_table(const float* act_mean, int64_t K, int n_grid, unsigned flags, void* workspace,
+                           size_t ws_bytes, float* table, awq_stream_t stream) {
+  if (act_mean == nullptr || table == nullptr) return fail(AWQ_ERR_INVALID_ARG, "null pointer");
+  if (K < 1 || K >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "bad K");
+  AWQ_TRY(check_grid(n_grid));
+  if (flags & ~AWQ_FLAG_EXACT_POW) return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const ScaleLayout l = scale_layout(K, n_grid);
+  if (workspace == nullptr || ws_bytes < l.bytes)
+    return fail(AWQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", l.bytes, workspace ? ws_bytes : 0);
+  DeviceInfo* d = nullptr;
+  AWQ_TRY(device_info(&d));
+  AWQ_TRY(launch_scale_table(act_mean, K, n_grid, (flags & AWQ_FLAG_EXACT_POW) != 0, table, nullptr,
+                             reinterpret_cast<float2*>(static_cast<char*>(workspace) + l.part_off),
+                             reinterpret_cast<cudaStream_t>(stream)));
+  return ok();
+}
+
+size_t awq_search_workspace_size(int64_t N, int64_t K, int64_t O, int group, int n_grid) {
+  if (N < 1 || K < 1 || O < 1 || group != 128 || n_grid < 1 || n_grid > AWQ_MAX_N_GRID) return 0;
+  return search_layout(N, K, O, n_grid).bytes;
+}
+
+awq_status awq_search_get_layout(int64_t N, int64_t K, int64_t O, int group, int n_grid, awq_search_layout* out) {
+  if (out == nullptr) return fail(AWQ_ERR_INVALID_ARG, "out is null");
+  AWQ_TRY(check_group(group));
+  AWQ_TRY(check_grid(n_grid));
+  if (N < 1 || K < 1 || O < 1) return fail(AWQ_ERR_INVALID_ARG, "empty shape");
+  const SearchLayout l = search_layout(N, K, O, n_grid);
+  out->tile_n = awq::lg::BM;
+  out->tile_o = awq::lg::BN;
+  out->tiles_n = l.tiles_n;
+  out->tiles_o = l.tiles_o;
+  out->partials_offset = l.partials_off;
+  out->workspace_bytes = l.bytes;
+  return ok();
+}
+
+awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const void* W, int64_t O, int64_t ldw,
+                         const float* act_mean, int group, int n_grid, unsigned flags, void* workspace,
+                         size_t ws_bytes, double* losses, int* best_j, float* scales, awq_stream_t stream) {
+  AWQ_TRY(check_group(group));
+  AWQ_TRY(check_grid(n_grid));
+  AWQ_TRY(check_matrix("X", X, N, K, ldx));
+  AWQ_TRY(check_matrix("W", W, O, K, ldw));
+  if (K % 128 != 0) return fail(AWQ_ERR_INVALID_ARG, "K (%lld) must be a multiple of 128", static_cast<long long>(K));
+  if (act_mean == nullptr || losses == nullptr || best_j == nullptr || scales == nullptr)
+    return fail(AWQ_ERR_INVALID_ARG, "null output or act_mean pointer");
+  if (flags & ~(AWQ_FLAG_EXACT_DIVISION | AWQ_FLAG_EXACT_POW | AWQ_FLAG_INJECT_STALL))
+    return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const SearchLayout l = search_layout(N, K, O, n_grid);
+  if (static_cast<int64_t>(n_grid) * l.O_pad >= (1ll << 31))
+    return fail(AWQ_ERR_INVALID_ARG, "n_grid * O is too large");
+  if (static_cast<int64_t>(n_grid) * l.tiles_o * l.tiles_n >= (1ll << 31))
+    return fail(AWQ_ERR_INVALID_ARG, "too many tiles");
+  if (workspace == nullptr || ws_bytes < l.bytes)
+    return fail(AWQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", l.bytes, workspace ? ws_bytes : 0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 1023u) != 0)
+    return fail(AWQ_ERR_INVALID_ARG, "workspace must be 1024-byte aligned");
+  DeviceInfo* d = nullptr;
+  AWQ_TRY(device_info(&d));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  auto* status = reinterpret_cast<awq::DeviceStatus*>(ws + l.status_off);
+  float* table = reinterpret_cast<float*>(ws + l.table_off);
+  float* rtable = reinterpret_cast<float*>(ws + l.rtable_off);
+  auto* spart = reinterpret_cast<float2*>(ws + l.spart_off);
+  auto* partials = reinterpret_cast<double*>(ws + l.partials_off);
+  auto* dw = reinterpret_cast<__nv_bfloat16*>(ws + l.dw_off);
+
+  CUtensorMap tmX, tmD;
+  AWQ_TRY(make_tmap(&tmX, X, N, K, ldx, awq::lg::BM));
+  AWQ_TRY(make_tmap(&tmD, dw, static_cast<int64_t>(n_grid) * l.O_pad, K, K, awq::lg::BN));
+
+  AWQ_CUDA(cudaMemsetAsync(status, 0, sizeof(awq::DeviceStatus), st));
+  AWQ_TRY(launch_scale_table(act_mean, K, n_grid, (flags & AWQ_FLAG_EXACT_POW) != 0, table, rtable, spart, st));
+
+  const int64_t segs = (K + awq::kProdWarpCols - 1) / awq::kProdWarpCols;
+  const int64_t warps = l.O_pad * segs;
+  const int64_t blocks = (warps * 32 + awq::kProdThreads - 1) / awq::kProdThreads;
+  awq::produce_dw_kernel<<<static_cast<unsigned>(blocks), awq::kProdThreads, 0, st>>>(
+      static_cast<const uint16_t*>(W), O, l.O_pad, K, ldw, n_grid, table, rtable,
+      (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0, dw, status);
+  AWQ_TRY(check_launch("produce_dw_kernel"));
+
+  awq::lg::Params p;
+  p.n_tiles_n = static_cast<int>(l.tiles_n);
+  p.n_bands = static_cast<int>(static_cast<int64_t>(n_grid) * l.tiles_o);
+  p.num_kb = static_cast<int>(K / awq::lg::BK);
+  p.num_tiles = p.n_tiles_n * p.n_bands;
+  p.partials = partials;
+  p.status = status;
+  p.limit_ns = g_wait_limit_ns.load();
+  p.flags = flags;
+  const int grid = p.num_tiles < d->sms ? p.num_tiles : d->sms;
+  if (g_prof_before != nullptr) AWQ_CUDA(cudaEventRecord(g_prof_before, st));
+  awq::lg::loss_gemm_kernel<<<grid, awq::lg::THREADS, awq::lg::SMEM_BYTES, st>>>(tmX, tmD, p);
+  AWQ_TRY(check_launch("loss_gemm_kernel"));
+  if (g_prof_after != nullptr) AWQ_CUDA(cudaEventRecord(g_prof_after, st));
+
+  awq::finalize_kernel<<<1, 1024, 0, st>>>(partials, l.tiles_o * l.tiles_n * 4, n_grid,
+                                           static_cast<double>(N) * static_cast<double>(O), table, K, losses,
+                                           best_j, scales, status);
+  AWQ_TRY(check_launch("finalize_kernel"));
+  return ok();
+}
+
+awq_status awq_search(const void* X, int64_t N, int64_t K, int64_t ldx, const void* W, int64_t O, int64_t ldw,
+                      const float* act_mean, int group, int n_grid, void* workspace, size_t ws_bytes,
+                      double* losses, int* best_j, float* scales, awq_stream_t stream) {
+  return awq_search_ex(X, N, K, ldx, W, O, ldw, act_mean, group, n_grid, 0u, workspace, ws_bytes, losses, best_j,
+                       scales, stream);
+}
+
+awq_status awq_search_status(const void* workspace, size_t ws_bytes, awq_stream_t stream) {
+  if (workspace == nullptr || ws_bytes < sizeof(awq::DeviceStatus))
+    return fail(AWQ_ERR_WORKSPACE, "workspace is null or too small");
+  AWQ_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  awq::DeviceStatus h;
+  AWQ_CUDA(cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost));
+  if (h.code == 5u)
+    return fail(AWQ_ERR_TIMEOUT, "device wait gave up (site %u, block %u)", h.where, h.block);
+  if (h.code != 0u) return fail(AWQ_ERR_CUDA, "unknown device status %u", h.code);
+  return ok();
+}
+
+awq_status awq_quantize_pack_ex(const void* W, int64_t O, int64_t K, int64_t ldw, const float* scales, int group,
+                                unsigned flags, uint32_t* codes, float* steps, float* zeros, awq_stream_t stream) {
+  AWQ_TRY(check_group(group));
+  AWQ_TRY(check_matrix("W", W, O, K, ldw));
+  if (K % 128 != 0) return fail(AWQ_ERR_INVALID_ARG, "K (%lld) must be a multiple of 128", static_cast<long long>(K));
+  if (scales == nullptr || codes == nullptr || steps == nullptr || zeros == nullptr)
+    return fail(AWQ_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(scales)) return fail(AWQ_ERR_INVALID_ARG, "scales is not 16-byte aligned");
+  if (flags & ~AWQ_FLAG_EXACT_DIVISION) return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  DeviceInfo* d = nullptr;
+  AWQ_TRY(device_info(&d));
+  const int64_t segs = (K + 255) / 256;
+  const int64_t blocks = (O * segs * 32 + awq::kPackThreads - 1) / awq::kPackThreads;
+  awq::quantize_pack_kernel<<<static_cast<unsigned>(blocks), awq::kPackThreads, 0,
+                              reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(W), O, K, ldw, scales, (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0, codes, steps,
+      zeros);
+  AWQ_TRY(check_launch("quantize_pack_kernel"));
+  return ok();
+}
+
+awq_status awq_quantize_pack(const void* W, int64_t O, int64_t K, int64_t ldw, const float* scales, int group,
+                             uint32_t* codes, float* steps, float* zeros, awq_stream_t stream) {
+  return awq_quantize_pack_ex(W, O, K, ldw, scales, group, 0u, codes, steps, zeros, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,254 @@
+// kernel_loss_gemm.cuh - the reconstruction loss on the 5th-generation tensor cores.
+//
+// For every candidate j and every tile of 128 tokens x 256 output rows, E = X_tile * dW_tile^T is
+// accumulated over K in tensor memory (tcgen05.mma kind::f16, bf16 x bf16 -> fp32, M = 128, N = 256,
+// K = 16 per instruction); the epilogue reads E from tensor memory, squares and sums it per row in fp32,
+// and adds the 32 rows of each warp in fp64. E is never written to global memory.
+//
+// Persistent kernel, one CTA per SM, 6 warps:
+//   warp 0      TMA producer: X tile [128 x 64] and dW tile [256 x 64] per stage, 128-byte swizzle
+//   warp 1      owns tensor memory (512 columns = two 128x256 fp32 accumulators) and issues the MMAs
+//   warps 2-5   epilogue: one TMEM lane quarter each (warp w reads lanes 32*(w%4) .. +31)
+// Barriers: full/empty per smem stage, full/empty per accumulator. Every wait is bounded.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+
+#include "ptx.cuh"
+
+namespace awq {
+namespace lg {
+
+constexpr int BM = 128;                          // tokens per tile (MMA M, TMEM lanes)
+constexpr int BN = 256;                          // output rows per tile (MMA N, TMEM columns)
+constexpr int BK = 64;                           // in-features per stage (one 128-byte swizzle row)
+constexpr int UK = 16;                           // K of one tcgen05.mma kind::f16
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;             // 16 KB
+constexpr int B_BYTES = BN * BK * 2;             // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 48 KB
+constexpr int NUM_ACC = 2;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int THREADS = 192;
+constexpr int BANDS_PER_GROUP = 8;               // tile raster: 8 dW bands advance together over X
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+struct Params {
+  int n_tiles_n;      // ceil(N / BM)
+  int n_bands;        // n_grid * O_pad / BN
+  int num_kb;         // K / BK
+  int num_tiles;      // n_tiles_n * n_bands
+  double* partials;   // [n_bands][n_tiles_n][4]
+  DeviceStatus* status;
+  uint64_t limit_ns;
+  unsigned flags;
+};
+
+__device__ __forceinline__ void tile_coords(int t, const Params& p, int& band, int& nt) {
+  const int per_group = BANDS_PER_GROUP * p.n_tiles_n;
+  const int g = t / per_group;
+  const int local = t - g * per_group;
+  const int bands_in_g = min(BANDS_PER_GROUP, p.n_bands - g * BANDS_PER_GROUP);
+  band = g * BANDS_PER_GROUP + local % bands_in_g;
+  nt = local / bands_in_g;
+}
+
+// All 32 lanes wait; the outcome is uniform across the warp.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, DeviceStatus* st, uint64_t limit,
+                                          unsigned where) {
+  uint64_t t0 = 0;
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) t0 = global_timer_ns();
+#pragma unroll 1
+  for (uint32_t it = 0;; ++it) {
+    const bool done = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    int give_up = 0;
+    if (lane == 0 && (it & 63u) == 63u) {
+      if (status_code(st) != 0u) give_up = 1;
+      else if (global_timer_ns() - t0 > limit) {
+        raise_timeout(st, where);
+        give_up = 1;
+      }
+    }
+    if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    loss_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmD,
+                     Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bars[2 * STAGES + 2 * NUM_ACC + 2];
+  __shared__ uint32_t tmem_slot;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t bar0 = smem_u32(&bars[0]);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + NUM_ACC + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * NUM_ACC);
+  const uint32_t never_bar = drain_bar + 8u;
+  const uint32_t smem_base = smem_u32(smem);
+  auto a_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s) * STAGE_BYTES; };
+  auto b_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s) * STAGE_BYTES + A_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < NUM_ACC; ++a) {
+      mbar_init(accf_bar(a), 1);
+      mbar_init(acce_bar(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    mbar_init(never_bar, 1);
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), TMEM_COLS);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmD);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  DeviceStatus* st = p.status;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t pending = 0, pend_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+        int band, nt;
+        tile_coords(t, p, band, nt);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, st, p.limit_ns, kSiteTmaEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
+          tma_load_2d(a_tile(stage), &tmX, kb * BK, nt * BM, full_bar(stage));
+          tma_load_2d(b_tile(stage), &tmD, kb * BK, band * BN, full_bar(stage));
+          pending |= 1u << stage;
+          pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (status_code(st) != 0u) {
+        // Wait (bounded) for this thread's copies still in flight before the CTA may exit.
+        for (int s = 0; s < STAGES; ++s)
+          if (pending & (1u << s)) {
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(full_bar(s), (pend_phase >> s) & 1u))
+              if (global_timer_ns() - t0 > p.limit_ns) {
+                raise_timeout(st, kSiteDrainTma);
+                break;
+              }
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      if (p.flags & AWQ_FLAG_INJECT_STALL) ok = mbar_wait(never_bar, 0u, st, p.limit_ns, kSiteMmaInjected);
+      int local = 0;
+      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
+        if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, st, p.limit_ns, kSiteMmaAccEmpty)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, st, p.limit_ns, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = a_tile(stage), b0 = b_tile(stage);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk)
+            umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * UK * 2), smem_desc_sw128(b0 + kk * UK * 2), IDESC,
+                      (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(accf_bar(acc));
+      }
+      // Every MMA this thread issued must be complete before tensor memory is released.
+      umma_commit(drain_bar);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain_bar, 0u))
+        if (global_timer_ns() - t0 > p.limit_ns) {
+          raise_timeout(st, kSiteDrainMma);
+          break;
+        }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    int local = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
+      if (!warp_wait(accf_bar(acc), acc_phase, st, p.limit_ns, kSiteEpiAccFull)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+      float sum = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sum = fmaf(v[i], v[i], sum);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar(acc));
+      double ds = static_cast<double>(sum);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ds = __dadd_rn(ds, __shfl_xor_sync(0xffffffffu, ds, off));
+      if (lane == 0) {
+        int band, nt;
+        tile_coords(t, p, band, nt);
+        p.partials[(static_cast<int64_t>(band) * p.n_tiles_n + nt) * 4 + quarter] = ds;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace lg
+}  // namespace awq

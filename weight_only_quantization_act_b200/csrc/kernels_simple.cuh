@@ -1,0 +1,339 @@
+// kernels_simple.cuh - the HBM- and ALU-bound kernels of the AWQ search: activation statistic, scale
+// table, weight-error producer, loss/argmin finalisation and the INT4 pack.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "numerics.cuh"
+#include "ptx.cuh"
+
+namespace awq {
+
+// ===================================================================================================
+// (1) activation statistic: act_mean[k] = RN32(RN64(S_k / N)), S_k = sum_i |X[i,k]| in fp64 in a fixed
+// order (256-row chunks; rows in increasing order inside a chunk; chunk totals in chunk order).
+// ===================================================================================================
+constexpr int kMaxGrid = 64;  // largest n_grid (AWQ_MAX_N_GRID)
+constexpr int kActChunk = 256;
+constexpr int kActThreads = 256;
+constexpr int kActColsPerThread = 2;
+constexpr int kActColsPerBlock = kActThreads * kActColsPerThread;
+constexpr int kActUnroll = 32;
+
+// grid (ceil(K / 512), n_chunks): thread owns 2 adjacent columns of one chunk and walks its rows.
+__global__ void __launch_bounds__(kActThreads) act_chunk_sums_kernel(const uint16_t* __restrict__ X,
+                                                                     int64_t N, int64_t K, int64_t ldx,
+                                                                     double* __restrict__ part) {
+  const int64_t c = (static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x) * kActColsPerThread;
+  if (c >= K) return;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kActChunk;
+  const int64_t r1 = min(N, r0 + kActChunk);
+  const int64_t stride = ldx / 2;  // in 32-bit words
+  const uint32_t* p = reinterpret_cast<const uint32_t*>(X + r0 * ldx + c);
+  double s0 = 0.0, s1 = 0.0;
+  int64_t i = r0;
+  for (; i + kActUnroll <= r1; i += kActUnroll) {
+    uint32_t v[kActUnroll];
+#pragma unroll
+    for (int u = 0; u < kActUnroll; ++u) v[u] = __ldcs(p + (i - r0 + u) * stride);
+#pragma unroll
+    for (int u = 0; u < kActUnroll; ++u) {
+      s0 = __dadd_rn(s0, fabs(static_cast<double>(bf16_lo(v[u]))));
+      s1 = __dadd_rn(s1, fabs(static_cast<double>(bf16_hi(v[u]))));
+    }
+  }
+  for (; i < r1; ++i) {
+    const uint32_t v = __ldcs(p + (i - r0) * stride);
+    s0 = __dadd_rn(s0, fabs(static_cast<double>(bf16_lo(v))));
+    s1 = __dadd_rn(s1, fabs(static_cast<double>(bf16_hi(v))));
+  }
+  double* out = part + static_cast<int64_t>(blockIdx.y) * K + c;
+  out[0] = s0;
+  out[1] = s1;
+}
+
+// grid ceil(K / 256): chunk totals in chunk order, then the mean.
+__global__ void __launch_bounds__(256) act_finalize_kernel(const double* __restrict__ part, int64_t N,
+                                                           int64_t K, int n_chunks,
+                                                           float* __restrict__ act_mean) {
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (k >= K) return;
+  double S = 0.0;
+  for (int c = 0; c < n_chunks; ++c) S = __dadd_rn(S, part[static_cast<int64_t>(c) * K + k]);
+  act_mean[k] = __double2float_rn(__ddiv_rn(S, static_cast<double>(N)));
+}
+
+// ===================================================================================================
+// (2) scale table: t = CR32(act^r) clamped at 1e-4, then t / sqrt(max t * min t) per row j.
+// ===================================================================================================
+constexpr int kScaleThreads = 256;
+
+__device__ __forceinline__ void block_max_min(float& mx, float& mn, float* red /* [2 * 32] */) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+  }
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) {
+    red[w] = mx;
+    red[32 + w] = mn;
+  }
+  __syncthreads();
+  if (w == 0) {
+    const int nw = blockDim.x >> 5;
+    mx = l < nw ? red[l] : 0.0f;
+    mn = l < nw ? red[32 + l] : __int_as_float(0x7f800000);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    }
+  }
+}
+
+// grid (ceil(K / 256), n_grid)
+__global__ void __launch_bounds__(kScaleThreads) scale_pow_kernel(const float* __restrict__ act, int64_t K,
+                                                                  int n_grid, int force_slow,
+                                                                  float* __restrict__ table,
+                                                                  float2* __restrict__ part) {
+  __shared__ float red[64];
+  const int j = blockIdx.y;
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * kScaleThreads + threadIdx.x;
+  const float r = __fdiv_rn(static_cast<float>(j), static_cast<float>(n_grid));
+  float mx = 0.0f, mn = __int_as_float(0x7f800000);
+  if (k < K) {
+    const float t = fmaxf(pow_f32_cr(act[k], r, force_slow != 0), AWQ_SCALE_FLOOR);
+    table[static_cast<int64_t>(j) * K + k] = t;
+    mx = t;
+    mn = t;
+  }
+  block_max_min(mx, mn, red);
+  if (threadIdx.x == 0) part[static_cast<int64_t>(j) * gridDim.x + blockIdx.x] = make_float2(mx, mn);
+}
+
+// grid (ceil(K / 256), n_grid): every block reduces the row's partial max/min (cheap, <= a few hundred
+// entries) and normalises its 256 columns in place. Optionally also writes RN32(1/s) for the producer.
+__global__ void __launch_bounds__(kScaleThreads) scale_normalize_kernel(float* __restrict__ table,
+                                                                        float* __restrict__ rtable,
+                                                                        const float2* __restrict__ part,
+                                                                        int64_t K, int nblk) {
+  __shared__ float red[64];
+  const int j = blockIdx.y;
+  float mx = 0.0f, mn = __int_as_float(0x7f800000);
+  for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+    const float2 v = part[static_cast<int64_t>(j) * nblk + b];
+    mx = fmaxf(mx, v.x);
+    mn = fminf(mn, v.y);
+  }
+  block_max_min(mx, mn, red);
+  __shared__ float d_sh;
+  if (threadIdx.x == 0) d_sh = __fsqrt_rn(__fmul_rn(mx, mn));
+  __syncthreads();
+  const float d = d_sh;
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * kScaleThreads + threadIdx.x;
+  if (k < K) {
+    const int64_t idx = static_cast<int64_t>(j) * K + k;
+    const float s = __fdiv_rn(table[idx], d);
+    table[idx] = s;
+    if (rtable != nullptr) rtable[idx] = __frcp_rn(s);
+  }
+}
+
+// ===================================================================================================
+// (3) weight-error producer: dW_j[o, k] = bf16(RN32(w - w_hat_j)) for every candidate j, written as the
+// B operand of the loss GEMM (row j * O_pad + o, K contiguous). Rows o >= O are written as zeros.
+// One thread owns 16 consecutive in-features of one row (8 lanes per group of 128); one warp owns 512
+// in-features of one row; the thread keeps its 16 weights in registers across all candidates.
+// w_hat = deq * RN32(1/s) here (within one fp32 rounding of deq / s; it only feeds the loss).
+// ===================================================================================================
+constexpr int kProdThreads = 256;
+constexpr int kProdCols = 16;
+constexpr int kProdWarpCols = 32 * kProdCols;  // 512
+
+__global__ void __launch_bounds__(kProdThreads) produce_dw_kernel(
+    const uint16_t* __restrict__ W, int64_t O, int64_t O_pad, int64_t K, int64_t ldw, int n_grid,
+    const float* __restrict__ table, const float* __restrict__ rtable, int exact,
+    __nv_bfloat16* __restrict__ dW, const DeviceStatus* st) {
+  const int64_t segs = (K + kProdWarpCols - 1) / kProdWarpCols;
+  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * kProdThreads + threadIdx.x) >> 5;
+  if (gw >= O_pad * segs) return;  // whole warps exit together
+  if (status_code(st) != 0u) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t o = gw / segs;
+  const int64_t k0 = (gw - o * segs) * kProdWarpCols + static_cast<int64_t>(lane) * kProdCols;
+  const bool active = k0 < K;  // K % 128 == 0: 8-lane groups are all active or all idle
+  const bool pad_row = o >= O;
+
+  float w[kProdCols];
+  if (active && !pad_row) {
+    const uint4* src = reinterpret_cast<const uint4*>(W + o * ldw + k0);
+    const uint4 a = __ldg(src), b = __ldg(src + 1);
+    const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w[2 * i] = bf16_lo(u[i]);
+      w[2 * i + 1] = bf16_hi(u[i]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kProdCols; ++i) w[i] = 0.0f;
+  }
+
+  for (int j = 0; j < n_grid; ++j) {
+    uint32_t outw[8];
+    if (!pad_row) {
+      float s[kProdCols], rs[kProdCols];
+      if (active) {
+        const float4* ps = reinterpret_cast<const float4*>(table + static_cast<int64_t>(j) * K + k0);
+        const float4* pr = reinterpret_cast<const float4*>(rtable + static_cast<int64_t>(j) * K + k0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 a = __ldg(ps + i), b = __ldg(pr + i);
+          s[4 * i] = a.x; s[4 * i + 1] = a.y; s[4 * i + 2] = a.z; s[4 * i + 3] = a.w;
+          rs[4 * i] = b.x; rs[4 * i + 1] = b.y; rs[4 * i + 2] = b.z; rs[4 * i + 3] = b.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kProdCols; ++i) { s[i] = 1.0f; rs[i] = 1.0f; }
+      }
+      float wp[kProdCols];
+      float mx = -__int_as_float(0x7f800000), mn = __int_as_float(0x7f800000);
+#pragma unroll
+      for (int i = 0; i < kProdCols; ++i) {
+        wp[i] = __fmul_rn(w[i], s[i]);
+        mx = fmaxf(mx, wp[i]);
+        mn = fminf(mn, wp[i]);
+      }
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      }
+      const GroupParams g = group_params(mx, mn);
+#pragma unroll
+      for (int i = 0; i < kProdCols; i += 2) {
+        const float q0 = code_of(wp[i], g, exact != 0), q1 = code_of(wp[i + 1], g, exact != 0);
+        const float h0 = __fmul_rn(dequant(q0, g), rs[i]);
+        const float h1 = __fmul_rn(dequant(q1, g), rs[i + 1]);
+        const __nv_bfloat162 pr = __floats2bfloat162_rn(__fsub_rn(w[i], h0), __fsub_rn(w[i + 1], h1));
+        outw[i / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) outw[i] = 0u;
+    }
+    if (active) {
+      uint4* dst = reinterpret_cast<uint4*>(dW + (static_cast<int64_t>(j) * O_pad + o) * K + k0);
+      __stcs(dst, make_uint4(outw[0], outw[1], outw[2], outw[3]));
+      __stcs(dst + 1, make_uint4(outw[4], outw[5], outw[6], outw[7]));
+    }
+  }
+}
+
+// ===================================================================================================
+// (4)-(5) finalisation: loss_j = (sum of the tile partials in a fixed order) / (N * O); best_j is the
+// first index of the minimum; scales = row best_j of the table. Single block of 1024 threads.
+// ===================================================================================================
+__global__ void __launch_bounds__(1024) finalize_kernel(const double* __restrict__ partials,
+                                                        int64_t per_cand, int n_grid, double denom,
+                                                        const float* __restrict__ table, int64_t K,
+                                                        double* __restrict__ losses, int* __restrict__ best_j,
+                                                        float* __restrict__ scales,
+                                                        const DeviceStatus* st) {
+  __shared__ double loss_sh[kMaxGrid];
+  __shared__ int best_sh;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool failed = status_code(st) != 0u;
+  for (int j = warp; j < n_grid; j += 32) {
+    double acc = 0.0;
+    const double* p = partials + static_cast<int64_t>(j) * per_cand;
+    for (int64_t i = lane; i < per_cand; i += 32) acc = __dadd_rn(acc, p[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc = __dadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+    if (lane == 0) loss_sh[j] = failed ? __longlong_as_double(0x7ff8000000000000ll) : __ddiv_rn(acc, denom);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    double v = __longlong_as_double(0x7ff0000000000000ll);
+    int idx = 0x7fffffff;
+    for (int j = lane; j < n_grid; j += 32) {
+      const double l = loss_sh[j];
+      if (l < v) { v = l; idx = j; }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, v, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
+      if (ov < v || (ov == v && oi < idx)) { v = ov; idx = oi; }
+    }
+    if (lane == 0) {
+      if (failed || idx == 0x7fffffff) idx = -1;
+      best_sh = idx;
+      *best_j = idx;
+    }
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < n_grid; j += blockDim.x) losses[j] = loss_sh[j];
+  const int b = best_sh;
+  if (b >= 0)
+    for (int64_t k = threadIdx.x; k < K; k += blockDim.x) scales[k] = table[static_cast<int64_t>(b) * K + k];
+}
+
+// ===================================================================================================
+// (5) pack: codes, steps and zeros of W at scales s. One thread owns 8 in-features (one code word);
+// 16 lanes per group; one warp covers 256 in-features of one row.
+// ===================================================================================================
+constexpr int kPackThreads = 256;
+
+__global__ void __launch_bounds__(kPackThreads) quantize_pack_kernel(
+    const uint16_t* __restrict__ W, int64_t O, int64_t K, int64_t ldw, const float* __restrict__ scales,
+    int exact, uint32_t* __restrict__ codes, float* __restrict__ steps, float* __restrict__ zeros) {
+  const int64_t segs = (K + 255) / 256;
+  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
+  if (gw >= O * segs) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t o = gw / segs;
+  const int64_t k0 = (gw - o * segs) * 256 + static_cast<int64_t>(lane) * 8;
+  const bool active = k0 < K;
+  float wp[8];
+  float mx = -__int_as_float(0x7f800000), mn = __int_as_float(0x7f800000);
+  if (active) {
+    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(W + o * ldw + k0));
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(scales + k0));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(scales + k0) + 1);
+    const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    const uint32_t u[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      wp[2 * i] = __fmul_rn(bf16_lo(u[i]), s[2 * i]);
+      wp[2 * i + 1] = __fmul_rn(bf16_hi(u[i]), s[2 * i + 1]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      mx = fmaxf(mx, wp[i]);
+      mn = fminf(mn, wp[i]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wp[i] = 0.0f;
+  }
+#pragma unroll
+  for (int off = 1; off < 16; off <<= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+  }
+  if (!active) return;
+  const GroupParams g = group_params(mx, mn);
+  uint32_t word = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) word |= static_cast<uint32_t>(code_of(wp[i], g, exact != 0)) << (4 * i);
+  __stcs(codes + o * (K / 8) + k0 / 8, word);
+  if ((lane & 15) == 0) {
+    const int64_t gi = o * (K / 128) + k0 / 128;
+    steps[gi] = g.step;
+    zeros[gi] = g.zero;
+  }
+}
+
+}  // namespace awq
