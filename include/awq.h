@@ -98,6 +98,27 @@ AWQ_API awq_status awq_act_stats(const void *X, int64_t N, int64_t K, int64_t ld
                          size_t ws_bytes, float *act_mean, awq_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------------
+ * Activation statistic that allocates nothing. The pages have no counterpart: this is a deployment
+ * convenience. Some callers cannot call cudaMalloc when they invoke the statistic: a plugin running
+ * inside an inference engine that owns all device memory and forbids allocation on its execution path,
+ * or a process that reserved nearly all HBM up front (KV caches, weight pools) where cudaMalloc would
+ * fail or implicitly synchronise the device. For them this variant takes no workspace: its fp64 chunk
+ * sums live in a fixed 16 MiB device array inside the library (AWQ_NOALLOC_SCRATCH_DOUBLES doubles),
+ * which every GPU that loads the library holds until the process exits.
+ *   Same inputs, output and result as awq_act_stats (bit-identical act_mean).
+ *   Limit: ceil(N / 256) * K <= AWQ_NOALLOC_SCRATCH_DOUBLES, else AWQ_ERR_INVALID_ARG and no launch
+ *   (e.g. N = 16384 with K <= 32768, or N = 4096 with K <= 131072).
+ *   The first call on each device looks up the array's device address (cudaGetSymbolAddress, which may
+ *   load the library's device code on that device); make that first call before any stream capture.
+ *   All calls share the one array, which keeps the last call's contents (every value a call reads is
+ *   first written by that call, so nothing needs clearing): calls that overlap on the GPU, e.g. on two
+ *   streams, race and give wrong results. Serialise them.
+ * ------------------------------------------------------------------------------------------------- */
+#define AWQ_NOALLOC_SCRATCH_DOUBLES (1ull << 21)
+AWQ_API awq_status awq_act_stats_noalloc(const void *X, int64_t N, int64_t K, int64_t ldx, float *act_mean,
+                                         awq_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------------
  * (2) Scale table alone (the first stage of awq_search, exposed for testing and for callers that want
  * the candidates). Row j of table (device, float [n_grid, K]) receives, with r = RN32(j / n_grid):
  *   t = correctly rounded fp32 of act_mean[k]^r (0^0 = 1), t = max(t, RN32(1e-4)),

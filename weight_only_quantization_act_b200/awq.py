@@ -38,6 +38,7 @@ SIGNATURES = {
     "awq_set_profile_events": (None, [_P, _P]),
     "awq_act_stats_workspace_size": (_SZ, [_I64, _I64]),
     "awq_act_stats": (_I, [_P, _I64, _I64, _I64, _P, _SZ, _P, _P]),
+    "awq_act_stats_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P]),
     "awq_scale_table_workspace_size": (_SZ, [_I64, _I]),
     "awq_scale_table": (_I, [_P, _I64, _I, _U, _P, _SZ, _P, _P]),
     "awq_search_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I]),
@@ -153,6 +154,18 @@ def act_stats(X: torch.Tensor, out: torch.Tensor | None = None, workspace: torch
     ws = _workspace(lib.awq_act_stats_workspace_size(N, K), X.device, workspace)
     _check("awq_act_stats", lib.awq_act_stats(_ptr(X), N, K, X.stride(0), _ptr(ws), ws.numel(), _ptr(out),
                                               _stream(stream)))
+    return out
+
+
+def act_stats_noalloc(X: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+    """Same statistic with no workspace, for callers that cannot allocate device memory at call time
+    (the scratch is a fixed 16 MiB array inside the library; ceil(N/256)*K <= 2**21). ``out`` must be
+    preallocated; calls that overlap on the GPU race on the shared scratch."""
+    lib = load_library()
+    X = _bf16_matrix("X", X)
+    N, K = X.shape
+    _check("awq_act_stats_noalloc", lib.awq_act_stats_noalloc(_ptr(X), N, K, X.stride(0), _ptr(out),
+                                                              _stream(stream)))
     return out
 
 

@@ -399,3 +399,69 @@ awq_status awq_quantize_pack(const void* W, int64_t O, int64_t K, int64_t ldw, c
 }
 
 }  // extern "C"
+
+// ===================================================================================================
+// Activation statistic without any allocation, for callers that cannot allocate device memory when
+// they call (see awq_act_stats_noalloc in awq.h). The fp64 chunk sums live in this file-scope device
+// array instead of a caller workspace. Every GPU that loads the library holds it until the process
+// exits. Host code must not use the array's name as a pointer: it only names the symbol; the device
+// address comes from cudaGetSymbolAddress, once per device, with that device current.
+// ===================================================================================================
+static __device__ __align__(256) double awq_act_scratch[AWQ_NOALLOC_SCRATCH_DOUBLES];
+
+namespace {
+
+struct ScratchSlot {
+  bool ready = false;
+  double* ptr = nullptr;
+};
+ScratchSlot g_scratch[kMaxDevices];
+std::mutex g_scratch_mu;
+
+awq_status act_scratch_address(double** out) {
+  int dev = 0;
+  AWQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(AWQ_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  ScratchSlot& slot = g_scratch[dev];
+  if (!slot.ready) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, awq_act_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(AWQ_ERR_CUDA, "cudaGetSymbolAddress of the no-alloc scratch failed on device %d: %s", dev,
+                  cudaGetErrorString(e));
+    slot.ptr = static_cast<double*>(p);
+    slot.ready = true;
+  }
+  *out = slot.ptr;
+  return AWQ_OK;
+}
+
+}  // namespace
+
+extern "C" awq_status awq_act_stats_noalloc(const void* X, int64_t N, int64_t K, int64_t ldx, float* act_mean,
+                                            awq_stream_t stream) {
+  AWQ_TRY(check_matrix("X", X, N, K, ldx));
+  if (K % 2 != 0) return fail(AWQ_ERR_INVALID_ARG, "K must be even");
+  if (act_mean == nullptr) return fail(AWQ_ERR_INVALID_ARG, "act_mean is null");
+  const ActLayout l = act_layout(N, K);
+  const uint64_t need = static_cast<uint64_t>(l.n_chunks) * static_cast<uint64_t>(K);
+  if (need > AWQ_NOALLOC_SCRATCH_DOUBLES)
+    return fail(AWQ_ERR_INVALID_ARG,
+                "awq_act_stats_noalloc: ceil(N/256)*K = %llu fp64 partial sums exceed the fixed scratch of %llu "
+                "(16 MiB); use awq_act_stats with a workspace",
+                static_cast<unsigned long long>(need), static_cast<unsigned long long>(AWQ_NOALLOC_SCRATCH_DOUBLES));
+  DeviceInfo* d = nullptr;
+  AWQ_TRY(device_info(&d));
+  double* part = nullptr;
+  AWQ_TRY(act_scratch_address(&part));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Each (chunk, column) entry the finaliser reads is written first by this call, so the scratch needs
+  // no clearing; what the previous call left there is simply overwritten.
+  dim3 grid(static_cast<unsigned>((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock), l.n_chunks);
+  awq::act_chunk_sums_kernel<<<grid, awq::kActThreads, 0, st>>>(static_cast<const uint16_t*>(X), N, K, ldx, part);
+  AWQ_TRY(check_launch("act_chunk_sums_kernel"));
+  awq::act_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(part, N, K, l.n_chunks, act_mean);
+  AWQ_TRY(check_launch("act_finalize_kernel"));
+  return ok();
+}
