@@ -130,7 +130,7 @@ ScaleLayout scale_layout(int64_t K, int n_grid) {
 
 struct SearchLayout {
   int64_t O_pad, tiles_n, tiles_o;
-  size_t status_off, table_off, rtable_off, spart_off, partials_off, dw_off, bytes;
+  size_t status_off, produced_off, table_off, rtable_off, spart_off, partials_off, dw_off, bytes;
   ScaleLayout sl;
 };
 SearchLayout search_layout(int64_t N, int64_t K, int64_t O, int n_grid) {
@@ -140,8 +140,9 @@ SearchLayout search_layout(int64_t N, int64_t K, int64_t O, int n_grid) {
   l.tiles_o = l.O_pad / awq::lg::BN;
   l.sl = scale_layout(K, n_grid);
   size_t off = 0;
-  l.status_off = off;
-  off += 256;
+  l.status_off = off;              // DeviceStatus (16 B)
+  l.produced_off = off + 256;      // unsigned produced[AWQ_MAX_N_GRID]
+  off += 512;
   l.table_off = off;
   off = align_up(off + static_cast<size_t>(n_grid) * K * sizeof(float), 256);
   l.rtable_off = off;
@@ -319,20 +320,14 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   CUtensorMap tmX, tmD;
   AWQ_TRY(make_tmap(&tmX, X, N, K, ldx, awq::lg::BM));
   AWQ_TRY(make_tmap(&tmD, dw, static_cast<int64_t>(n_grid) * l.O_pad, K, K, awq::lg::BN));
+  auto* produced = reinterpret_cast<unsigned int*>(ws + l.produced_off);
 
-  AWQ_CUDA(cudaMemsetAsync(status, 0, sizeof(awq::DeviceStatus), st));
+  AWQ_CUDA(cudaMemsetAsync(ws + l.status_off, 0, 512, st));  // status word and production counters
   AWQ_TRY(launch_scale_table(act_mean, K, n_grid, (flags & AWQ_FLAG_EXACT_POW) != 0, table, rtable, spart, st));
-
-  const int64_t segs = (K + awq::kProdWarpCols - 1) / awq::kProdWarpCols;
-  const int64_t warps = l.O_pad * segs;
-  const int64_t blocks = (warps * 32 + awq::kProdThreads - 1) / awq::kProdThreads;
-  awq::produce_dw_kernel<<<static_cast<unsigned>(blocks), awq::kProdThreads, 0, st>>>(
-      static_cast<const uint16_t*>(W), O, l.O_pad, K, ldw, n_grid, table, rtable,
-      (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0, dw, status);
-  AWQ_TRY(check_launch("produce_dw_kernel"));
 
   awq::lg::Params p;
   p.n_tiles_n = static_cast<int>(l.tiles_n);
+  p.band_begin = 0;
   p.n_bands = static_cast<int>(static_cast<int64_t>(n_grid) * l.tiles_o);
   p.num_kb = static_cast<int>(K / awq::lg::BK);
   p.num_tiles = p.n_tiles_n * p.n_bands;
@@ -340,9 +335,35 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
   p.flags = flags;
-  const int grid = p.num_tiles < d->sms ? p.num_tiles : d->sms;
+  p.tiles_o = static_cast<int>(l.tiles_o);
+  p.n_grid = n_grid;
+  p.prod.W = static_cast<const uint16_t*>(W);
+  p.prod.O = O;
+  p.prod.O_pad = l.O_pad;
+  p.prod.K = K;
+  p.prod.ldw = ldw;
+  p.prod.segs = (K + awq::kProdWarpCols - 1) / awq::kProdWarpCols;
+  p.prod.table = table;
+  p.prod.rtable = rtable;
+  p.prod.dW = dw;
+  p.prod.exact = (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0;
+  p.items_per_cand = l.O_pad * p.prod.segs;
+  p.produced = produced;
+
+  // One CTA per SM, launched cooperatively: the TMA warps wait for rows that the producer warps of
+  // every other CTA write, which is only safe when all CTAs are resident at once.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(d->sms));
+  cfg.blockDim = dim3(awq::lg::THREADS);
+  cfg.dynamicSmemBytes = awq::lg::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (g_prof_before != nullptr) AWQ_CUDA(cudaEventRecord(g_prof_before, st));
-  awq::lg::loss_gemm_kernel<<<grid, awq::lg::THREADS, awq::lg::SMEM_BYTES, st>>>(tmX, tmD, p);
+  AWQ_CUDA(cudaLaunchKernelEx(&cfg, awq::lg::loss_gemm_kernel, tmX, tmD, p));
   AWQ_TRY(check_launch("loss_gemm_kernel"));
   if (g_prof_after != nullptr) AWQ_CUDA(cudaEventRecord(g_prof_after, st));
 

@@ -5,15 +5,20 @@
 // K = 16 per instruction); the epilogue reads E from tensor memory, squares and sums it per row in fp32,
 // and adds the 32 rows of each warp in fp64. E is never written to global memory.
 //
-// Persistent kernel, one CTA per SM, 6 warps:
-//   warp 0      TMA producer: X tile [128 x 64] and dW tile [256 x 64] per stage, 128-byte swizzle
+// Persistent cooperative kernel, one CTA per SM, 14 warps:
+//   warp 0      TMA: X tile [128 x 64] and dW tile [256 x 64] per stage, 128-byte swizzle
 //   warp 1      owns tensor memory (512 columns = two 128x256 fp32 accumulators) and issues the MMAs
 //   warps 2-5   epilogue: one TMEM lane quarter each (warp w reads lanes 32*(w%4) .. +31)
+//   warps 6-13  weight-error producers: they write dW_j (bf16, global memory) candidate by candidate,
+//               all CTAs sharing each candidate's rows, and count finished rows per candidate. The
+//               ALU work of the quantizer thus runs on the same SMs while the tensor cores evaluate
+//               earlier candidates; the TMA warp starts on candidate j once its count is complete.
 // Barriers: full/empty per smem stage, full/empty per accumulator. Every wait is bounded.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
 
+#include "kernels_simple.cuh"
 #include "ptx.cuh"
 
 namespace awq {
@@ -29,20 +34,27 @@ constexpr int B_BYTES = BN * BK * 2;             // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 48 KB
 constexpr int NUM_ACC = 2;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int THREADS = 192;
+constexpr int PROD_WARPS = 8;
+constexpr int THREADS = 192 + 32 * PROD_WARPS;
 constexpr int BANDS_PER_GROUP = 8;               // tile raster: 8 dW bands advance together over X
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 
 struct Params {
   int n_tiles_n;      // ceil(N / BM)
-  int n_bands;        // n_grid * O_pad / BN
+  int band_begin;     // first dW band (of BN rows) this launch covers
+  int n_bands;        // bands this launch covers
   int num_kb;         // K / BK
   int num_tiles;      // n_tiles_n * n_bands
-  double* partials;   // [n_bands][n_tiles_n][4]
+  double* partials;   // [all bands][n_tiles_n][4]
   DeviceStatus* status;
   uint64_t limit_ns;
   unsigned flags;
+  int tiles_o;               // bands per candidate
+  int n_grid;
+  ProducerArgs prod;         // weight-error production for every candidate
+  int64_t items_per_cand;    // producer work items (warp x 512 in-features) per candidate
+  unsigned int* produced;    // [n_grid] finished items per candidate (zeroed before launch)
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& band, int& nt) {
@@ -50,7 +62,7 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& band, i
   const int g = t / per_group;
   const int local = t - g * per_group;
   const int bands_in_g = min(BANDS_PER_GROUP, p.n_bands - g * BANDS_PER_GROUP);
-  band = g * BANDS_PER_GROUP + local % bands_in_g;
+  band = p.band_begin + g * BANDS_PER_GROUP + local % bands_in_g;
   nt = local / bands_in_g;
 }
 
@@ -129,9 +141,29 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       uint32_t pending = 0, pend_phase = 0;
       bool ok = true;
+      int ready = -1;  // candidates < ready + 1 are known to be fully produced
       for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
         int band, nt;
         tile_coords(t, p, band, nt);
+        const int cand = band / p.tiles_o;
+        if (cand > ready) {
+          const uint64_t t0 = global_timer_ns();
+          while (ld_acquire_u32(p.produced + cand) < static_cast<unsigned int>(p.items_per_cand)) {
+            if (status_code(st) != 0u) {
+              ok = false;
+              break;
+            }
+            if (global_timer_ns() - t0 > p.limit_ns) {
+              raise_timeout(st, kSiteTmaProduced);
+              ok = false;
+              break;
+            }
+            __nanosleep(256);
+          }
+          if (!ok) break;
+          fence_proxy_async_global();
+          ready = cand;
+        }
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, st, p.limit_ns, kSiteTmaEmpty)) {
             ok = false;
@@ -209,6 +241,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
     __syncwarp();
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------------------------ producers
+    // Warp v owns one segment (seg = v % segs) and every wps-th row of it, so the segment's scales are
+    // loaded once per candidate; with fewer warps than segments a warp walks several whole segments.
+    const int64_t v = static_cast<int64_t>(blockIdx.x) * PROD_WARPS + (warp - 6);
+    const int64_t total = static_cast<int64_t>(gridDim.x) * PROD_WARPS;
+    const int64_t segs = p.prod.segs;
+    for (int j = 0; j < p.n_grid; ++j) {
+      unsigned int done = 0;
+      if (total >= segs) {
+        const int64_t wps = total / segs;
+        if (v < wps * segs) done = produce_rows(p.prod, v % segs, v / segs, wps, j, lane);
+      } else {
+        for (int64_t seg = v; seg < segs; seg += total) done += produce_rows(p.prod, seg, 0, 1, j, lane);
+      }
+      fence_proxy_async_global();
+      __threadfence();
+      __syncwarp();
+      if (lane == 0 && done != 0u) atomicAdd(p.produced + j, done);
+    }
   } else {
     // ------------------------------------------------------------------------------ epilogue
     const int quarter = warp & 3;

@@ -141,94 +141,108 @@ __global__ void __launch_bounds__(kScaleThreads) scale_normalize_kernel(float* _
 }
 
 // ===================================================================================================
-// (3) weight-error producer: dW_j[o, k] = bf16(RN32(w - w_hat_j)) for every candidate j, written as the
-// B operand of the loss GEMM (row j * O_pad + o, K contiguous). Rows o >= O are written as zeros.
-// One thread owns 16 consecutive in-features of one row (8 lanes per group of 128); one warp owns 512
-// in-features of one row; the thread keeps its 16 weights in registers across all candidates.
+// (3) weight-error producer: dW_j[o, k] = bf16(RN32(w - w_hat_j)), written as the B operand of the loss
+// GEMM (row j * O_pad + o, K contiguous); rows o >= O are written as zeros. A work item is 512
+// consecutive in-features (a segment) of one row, done by one warp: each lane owns 16 in-features
+// (8 lanes per group of 128). The producer warps of the loss-GEMM kernel call produce_rows.
 // w_hat = deq * RN32(1/s) here (within one fp32 rounding of deq / s; it only feeds the loss).
 // ===================================================================================================
-constexpr int kProdThreads = 256;
 constexpr int kProdCols = 16;
 constexpr int kProdWarpCols = 32 * kProdCols;  // 512
 
-__global__ void __launch_bounds__(kProdThreads) produce_dw_kernel(
-    const uint16_t* __restrict__ W, int64_t O, int64_t O_pad, int64_t K, int64_t ldw, int n_grid,
-    const float* __restrict__ table, const float* __restrict__ rtable, int exact,
-    __nv_bfloat16* __restrict__ dW, const DeviceStatus* st) {
-  const int64_t segs = (K + kProdWarpCols - 1) / kProdWarpCols;
-  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * kProdThreads + threadIdx.x) >> 5;
-  if (gw >= O_pad * segs) return;  // whole warps exit together
-  if (status_code(st) != 0u) return;
-  const int lane = threadIdx.x & 31;
-  const int64_t o = gw / segs;
-  const int64_t k0 = (gw - o * segs) * kProdWarpCols + static_cast<int64_t>(lane) * kProdCols;
-  const bool active = k0 < K;  // K % 128 == 0: 8-lane groups are all active or all idle
-  const bool pad_row = o >= O;
+struct ProducerArgs {
+  const uint16_t* W;
+  int64_t O, O_pad, K, ldw, segs;  // segs = ceil(K / 512) items per row
+  const float* table;              // [n_grid][K] scales
+  const float* rtable;             // [n_grid][K] RN32(1 / scale)
+  __nv_bfloat16* dW;               // [n_grid * O_pad][K]
+  int exact;                       // AWQ_FLAG_EXACT_DIVISION
+};
 
-  float w[kProdCols];
-  if (active && !pad_row) {
-    const uint4* src = reinterpret_cast<const uint4*>(W + o * ldw + k0);
-    const uint4 a = __ldg(src), b = __ldg(src + 1);
-    const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+// Weight errors of one row of one 512-in-feature segment for candidate j, from the row's raw bf16 words.
+__device__ __forceinline__ void produce_row(const ProducerArgs& a, const uint4 (&u)[2], const float (&s)[kProdCols],
+                                            const float (&rs)[kProdCols], bool real_row, uint32_t (&outw)[8]) {
+  if (!real_row) {  // padding rows (o >= O) are zeros; warp-uniform
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      w[2 * i] = bf16_lo(u[i]);
-      w[2 * i + 1] = bf16_hi(u[i]);
+    for (int i = 0; i < 8; ++i) outw[i] = 0u;
+    return;
+  }
+  const uint32_t raw[8] = {u[0].x, u[0].y, u[0].z, u[0].w, u[1].x, u[1].y, u[1].z, u[1].w};
+  float w[kProdCols], wp[kProdCols];
+  float mx = -__int_as_float(0x7f800000), mn = __int_as_float(0x7f800000);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    w[2 * i] = bf16_lo(raw[i]);
+    w[2 * i + 1] = bf16_hi(raw[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < kProdCols; ++i) {
+    wp[i] = __fmul_rn(w[i], s[i]);
+    mx = fmaxf(mx, wp[i]);
+    mn = fminf(mn, wp[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+  }
+  const GroupParams g = group_params(mx, mn);
+#pragma unroll
+  for (int i = 0; i < kProdCols; i += 2) {
+    const float q0 = code_of(wp[i], g, a.exact != 0), q1 = code_of(wp[i + 1], g, a.exact != 0);
+    const float h0 = __fmul_rn(dequant(q0, g), rs[i]);
+    const float h1 = __fmul_rn(dequant(q1, g), rs[i + 1]);
+    const __nv_bfloat162 pr = __floats2bfloat162_rn(__fsub_rn(w[i], h0), __fsub_rn(w[i + 1], h1));
+    outw[i / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+  }
+}
+
+// Rows o_first, o_first + o_step, ... < O_pad of segment `seg` for candidate j. The segment's scales
+// stay in registers; the next row's weights are loaded while the current row is computed. Returns the
+// number of (row, segment) items written.
+__device__ __forceinline__ unsigned int produce_rows(const ProducerArgs& a, int64_t seg, int64_t o_first,
+                                                     int64_t o_step, int j, int lane) {
+  const int64_t k0 = seg * kProdWarpCols + static_cast<int64_t>(lane) * kProdCols;
+  const bool active = k0 < a.K;  // K % 128 == 0: 8-lane groups are all active or all idle
+  float s[kProdCols], rs[kProdCols];
+  if (active) {
+    const float4* ps = reinterpret_cast<const float4*>(a.table + static_cast<int64_t>(j) * a.K + k0);
+    const float4* pr = reinterpret_cast<const float4*>(a.rtable + static_cast<int64_t>(j) * a.K + k0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 x = __ldg(ps + i), y = __ldg(pr + i);
+      s[4 * i] = x.x; s[4 * i + 1] = x.y; s[4 * i + 2] = x.z; s[4 * i + 3] = x.w;
+      rs[4 * i] = y.x; rs[4 * i + 1] = y.y; rs[4 * i + 2] = y.z; rs[4 * i + 3] = y.w;
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < kProdCols; ++i) w[i] = 0.0f;
+    for (int i = 0; i < kProdCols; ++i) { s[i] = 1.0f; rs[i] = 1.0f; }
   }
-
-  for (int j = 0; j < n_grid; ++j) {
+  unsigned int count = 0;
+  uint4 nxt[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+  if (o_first < a.O && active) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.W + o_first * a.ldw + k0);
+    nxt[0] = __ldg(src);
+    nxt[1] = __ldg(src + 1);
+  }
+  for (int64_t o = o_first; o < a.O_pad; o += o_step) {
+    const uint4 cur[2] = {nxt[0], nxt[1]};
+    const int64_t on = o + o_step;
+    if (on < a.O && active) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.W + on * a.ldw + k0);
+      nxt[0] = __ldg(src);
+      nxt[1] = __ldg(src + 1);
+    }
     uint32_t outw[8];
-    if (!pad_row) {
-      float s[kProdCols], rs[kProdCols];
-      if (active) {
-        const float4* ps = reinterpret_cast<const float4*>(table + static_cast<int64_t>(j) * K + k0);
-        const float4* pr = reinterpret_cast<const float4*>(rtable + static_cast<int64_t>(j) * K + k0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 a = __ldg(ps + i), b = __ldg(pr + i);
-          s[4 * i] = a.x; s[4 * i + 1] = a.y; s[4 * i + 2] = a.z; s[4 * i + 3] = a.w;
-          rs[4 * i] = b.x; rs[4 * i + 1] = b.y; rs[4 * i + 2] = b.z; rs[4 * i + 3] = b.w;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < kProdCols; ++i) { s[i] = 1.0f; rs[i] = 1.0f; }
-      }
-      float wp[kProdCols];
-      float mx = -__int_as_float(0x7f800000), mn = __int_as_float(0x7f800000);
-#pragma unroll
-      for (int i = 0; i < kProdCols; ++i) {
-        wp[i] = __fmul_rn(w[i], s[i]);
-        mx = fmaxf(mx, wp[i]);
-        mn = fminf(mn, wp[i]);
-      }
-#pragma unroll
-      for (int off = 1; off < 8; off <<= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-      }
-      const GroupParams g = group_params(mx, mn);
-#pragma unroll
-      for (int i = 0; i < kProdCols; i += 2) {
-        const float q0 = code_of(wp[i], g, exact != 0), q1 = code_of(wp[i + 1], g, exact != 0);
-        const float h0 = __fmul_rn(dequant(q0, g), rs[i]);
-        const float h1 = __fmul_rn(dequant(q1, g), rs[i + 1]);
-        const __nv_bfloat162 pr = __floats2bfloat162_rn(__fsub_rn(w[i], h0), __fsub_rn(w[i + 1], h1));
-        outw[i / 2] = *reinterpret_cast<const uint32_t*>(&pr);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) outw[i] = 0u;
-    }
+    produce_row(a, cur, s, rs, o < a.O, outw);
     if (active) {
-      uint4* dst = reinterpret_cast<uint4*>(dW + (static_cast<int64_t>(j) * O_pad + o) * K + k0);
-      __stcs(dst, make_uint4(outw[0], outw[1], outw[2], outw[3]));
-      __stcs(dst + 1, make_uint4(outw[4], outw[5], outw[6], outw[7]));
+      uint4* dst = reinterpret_cast<uint4*>(a.dW + (static_cast<int64_t>(j) * a.O_pad + o) * a.K + k0);
+      dst[0] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+      dst[1] = make_uint4(outw[4], outw[5], outw[6], outw[7]);
     }
+    ++count;
   }
+  return count;
 }
 
 // ===================================================================================================

@@ -23,6 +23,7 @@ enum WaitSite : unsigned int {
   kSiteMmaInjected = 5,
   kSiteDrainTma = 6,
   kSiteDrainMma = 7,
+  kSiteTmaProduced = 8,
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -106,6 +107,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, DeviceS
       return false;
     }
   }
+}
+
+// Global-memory flag helpers for the producer -> TMA hand-off inside one kernel.
+__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Orders this thread's generic-proxy global accesses with later async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------------------------- TMA
