@@ -159,12 +159,14 @@ AWQ_API awq_status awq_search_ex(const void *X, int64_t N, int64_t K, int64_t ld
 AWQ_API awq_status awq_search_status(const void *workspace, size_t ws_bytes, awq_stream_t stream);
 
 /* Where awq_search leaves its per-tile partial sums inside the workspace (valid after the call):
- * double partial[n_grid][tiles_o][tiles_n] at byte offset partials_offset; partial[j][a][b] is the sum
- * of squares of the outputs of rows [b*tile_n, (b+1)*tile_n) of X and output rows [a*tile_o,
- * (a+1)*tile_o) of W for candidate j (rows past N or O contribute zero). */
+ * double partial[n_grid][tiles_o][tiles_n][partials_per_tile] at byte offset partials_offset;
+ * partial[j][a][b][e] is the sum of squares of the outputs of token rows
+ * [b*tile_n + e*r, b*tile_n + (e+1)*r), r = tile_n / partials_per_tile, and output rows
+ * [a*tile_o, (a+1)*tile_o) for candidate j (rows past N or O contribute zero). */
 typedef struct awq_search_layout {
   int64_t tile_n, tile_o;   /* tile extent along tokens and along output rows */
   int64_t tiles_n, tiles_o; /* tiles per candidate along tokens and along output rows */
+  int64_t partials_per_tile;
   size_t partials_offset;   /* bytes from the workspace start */
   size_t workspace_bytes;   /* same as awq_search_workspace_size() */
 } awq_search_layout;

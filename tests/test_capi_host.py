@@ -55,8 +55,9 @@ def test_version_and_sizes(lib):
 
 def test_layout_geometry(lib):
     lay = awq.search_layout(300, 384, 600, 20)
-    assert (lay.tile_n, lay.tile_o) == (128, 256)
-    assert (lay.tiles_n, lay.tiles_o) == (3, 3)
+    assert (lay.tile_n, lay.tile_o) == (256, 256)
+    assert (lay.tiles_n, lay.tiles_o) == (2, 3)
+    assert lay.partials_per_tile == 8
     assert lay.partials_offset % 8 == 0
     assert lay.workspace_bytes == awq.search_workspace_size(300, 384, 600, 20)
 

@@ -53,7 +53,7 @@ SIGNATURES = {
 
 class SearchLayout(ctypes.Structure):
     _fields_ = [("tile_n", ctypes.c_int64), ("tile_o", ctypes.c_int64), ("tiles_n", ctypes.c_int64),
-                ("tiles_o", ctypes.c_int64), ("partials_offset", ctypes.c_size_t),
+                ("tiles_o", ctypes.c_int64), ("partials_per_tile", ctypes.c_int64), ("partials_offset", ctypes.c_size_t),
                 ("workspace_bytes", ctypes.c_size_t)]
 
 
@@ -241,11 +241,12 @@ def search_status(result: SearchResult, stream=None) -> int:
 
 
 def tile_partials(result: SearchResult, N: int, K: int, O: int, n_grid: int = 20) -> torch.Tensor:
-    """View of the per-tile partial sums: float64 [n_grid, tiles_o, tiles_n, 4] (4 = TMEM lane quarters)."""
+    """View of the per-tile partial sums: float64 [n_grid, tiles_o, tiles_n, partials_per_tile]; entry e of
+    a tile covers tile_n / partials_per_tile consecutive token rows."""
     lay = search_layout(N, K, O, n_grid)
-    count = n_grid * lay.tiles_o * lay.tiles_n * 4
+    count = n_grid * lay.tiles_o * lay.tiles_n * lay.partials_per_tile
     raw = result.workspace[lay.partials_offset: lay.partials_offset + 8 * count]
-    return raw.view(torch.float64).view(n_grid, lay.tiles_o, lay.tiles_n, 4)
+    return raw.view(torch.float64).view(n_grid, lay.tiles_o, lay.tiles_n, lay.partials_per_tile)
 
 
 # --------------------------------------------------------------------------------------------- (5)

@@ -44,6 +44,7 @@ struct DeviceInfo {
   int sms = 0;
   int cc_major = 0;
   bool gemm_attr_set = false;
+  int gemm_clusters = 0;  // CTA pairs of the loss GEMM that fit on the device at once
 };
 
 constexpr int kMaxDevices = 64;
@@ -65,6 +66,19 @@ awq_status device_info(DeviceInfo** out) {
   if (!d.gemm_attr_set) {
     AWQ_CUDA(cudaFuncSetAttribute(awq::lg::loss_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   awq::lg::SMEM_BYTES));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(d.sms & ~1));
+    cfg.blockDim = dim3(awq::lg::THREADS);
+    cfg.dynamicSmemBytes = awq::lg::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    AWQ_CUDA(cudaOccupancyMaxActiveClusters(&d.gemm_clusters, awq::lg::loss_gemm_kernel, &cfg));
+    if (d.gemm_clusters < 1) return fail(AWQ_ERR_UNSUPPORTED, "the loss GEMM does not fit on this device");
     d.gemm_attr_set = true;
   }
   *out = &d;
@@ -150,7 +164,8 @@ SearchLayout search_layout(int64_t N, int64_t K, int64_t O, int n_grid) {
   l.spart_off = off;
   off = align_up(off + l.sl.bytes, 256);
   l.partials_off = off;
-  off = align_up(off + static_cast<size_t>(n_grid) * l.tiles_o * l.tiles_n * 4 * sizeof(double), 1024);
+  off = align_up(off + static_cast<size_t>(n_grid) * l.tiles_o * l.tiles_n * awq::lg::PARTIALS_PER_TILE *
+                           sizeof(double), 1024);
   l.dw_off = off;
   off = align_up(off + static_cast<size_t>(n_grid) * l.O_pad * K * 2, 1024);
   l.bytes = off;
@@ -280,6 +295,7 @@ awq_status awq_search_get_layout(int64_t N, int64_t K, int64_t O, int group, int
   out->tile_o = awq::lg::BN;
   out->tiles_n = l.tiles_n;
   out->tiles_o = l.tiles_o;
+  out->partials_per_tile = awq::lg::PARTIALS_PER_TILE;
   out->partials_offset = l.partials_off;
   out->workspace_bytes = l.bytes;
   return ok();
@@ -318,8 +334,8 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   auto* dw = reinterpret_cast<__nv_bfloat16*>(ws + l.dw_off);
 
   CUtensorMap tmX, tmD;
-  AWQ_TRY(make_tmap(&tmX, X, N, K, ldx, awq::lg::BM));
-  AWQ_TRY(make_tmap(&tmD, dw, static_cast<int64_t>(n_grid) * l.O_pad, K, K, awq::lg::BN));
+  AWQ_TRY(make_tmap(&tmX, X, N, K, ldx, awq::lg::HALF));
+  AWQ_TRY(make_tmap(&tmD, dw, static_cast<int64_t>(n_grid) * l.O_pad, K, K, awq::lg::HALF));
   auto* produced = reinterpret_cast<unsigned int*>(ws + l.produced_off);
 
   AWQ_CUDA(cudaMemsetAsync(ws + l.status_off, 0, 512, st));  // status word and production counters
@@ -350,10 +366,10 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   p.items_per_cand = l.O_pad * p.prod.segs;
   p.produced = produced;
 
-  // One CTA per SM, launched cooperatively: the TMA warps wait for rows that the producer warps of
-  // every other CTA write, which is only safe when all CTAs are resident at once.
+  // As many CTA pairs as fit at once, launched cooperatively: the TMA warps wait for rows that the
+  // producer warps of every other CTA write, which is only safe when all CTAs are resident together.
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(d->sms));
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * d->gemm_clusters));
   cfg.blockDim = dim3(awq::lg::THREADS);
   cfg.dynamicSmemBytes = awq::lg::SMEM_BYTES;
   cfg.stream = st;
@@ -367,7 +383,7 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   AWQ_TRY(check_launch("loss_gemm_kernel"));
   if (g_prof_after != nullptr) AWQ_CUDA(cudaEventRecord(g_prof_after, st));
 
-  awq::finalize_kernel<<<1, 1024, 0, st>>>(partials, l.tiles_o * l.tiles_n * 4, n_grid,
+  awq::finalize_kernel<<<1, 1024, 0, st>>>(partials, l.tiles_o * l.tiles_n * awq::lg::PARTIALS_PER_TILE, n_grid,
                                            static_cast<double>(N) * static_cast<double>(O), table, K, losses,
                                            best_j, scales, status);
   AWQ_TRY(check_launch("finalize_kernel"));

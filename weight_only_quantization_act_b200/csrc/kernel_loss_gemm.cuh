@@ -1,19 +1,23 @@
 // kernel_loss_gemm.cuh - the reconstruction loss on the 5th-generation tensor cores.
 //
-// For every candidate j and every tile of 128 tokens x 256 output rows, E = X_tile * dW_tile^T is
-// accumulated over K in tensor memory (tcgen05.mma kind::f16, bf16 x bf16 -> fp32, M = 128, N = 256,
-// K = 16 per instruction); the epilogue reads E from tensor memory, squares and sums it per row in fp32,
-// and adds the 32 rows of each warp in fp64. E is never written to global memory.
+// For every candidate j and every tile of 256 tokens x 256 output rows, E = X_tile * dW_tile^T is
+// accumulated over K in tensor memory by a CTA pair (tcgen05.mma.cta_group::2 kind::f16, bf16 x bf16 ->
+// fp32, M = 256, N = 256, K = 16 per instruction). Each CTA of the pair stages half of the X rows and
+// half of the dW rows, and receives its 128 token rows of E in its own tensor memory. The epilogue
+// squares and sums each row in fp32 and adds the 32 rows of each warp in fp64. E is never written to
+// global memory.
 //
-// Persistent cooperative kernel, one CTA per SM, 14 warps:
-//   warp 0      TMA: X tile [128 x 64] and dW tile [256 x 64] per stage, 128-byte swizzle
-//   warp 1      owns tensor memory (512 columns = two 128x256 fp32 accumulators) and issues the MMAs
+// Persistent cooperative kernel, clusters of 2 CTAs, one CTA per SM, 14 warps per CTA:
+//   warp 0      TMA: X tile [128 x 64] and dW tile [128 x 64] per stage for this CTA, 128-byte
+//               swizzle; the bytes of both CTAs are counted on the even CTA's barrier
+//   warp 1      pair-wide tensor memory (512 columns = two 256-column fp32 accumulators); in the even
+//               CTA one thread issues the pair MMAs and commits to barriers in both CTAs
 //   warps 2-5   epilogue: one TMEM lane quarter each (warp w reads lanes 32*(w%4) .. +31)
 //   warps 6-13  weight-error producers: they write dW_j (bf16, global memory) candidate by candidate,
 //               all CTAs sharing each candidate's rows, and count finished rows per candidate. The
 //               ALU work of the quantizer thus runs on the same SMs while the tensor cores evaluate
-//               earlier candidates; the TMA warp starts on candidate j once its count is complete.
-// Barriers: full/empty per smem stage, full/empty per accumulator. Every wait is bounded.
+//               earlier candidates; the TMA warps start on candidate j once its count is complete.
+// Every wait is bounded (see ptx.cuh).
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -24,20 +28,22 @@
 namespace awq {
 namespace lg {
 
-constexpr int BM = 128;                          // tokens per tile (MMA M, TMEM lanes)
-constexpr int BN = 256;                          // output rows per tile (MMA N, TMEM columns)
+constexpr int BM = 256;                          // tokens per pair tile (MMA M; 128 per CTA)
+constexpr int BN = 256;                          // output rows per pair tile (MMA N; 128 staged per CTA)
+constexpr int HALF = 128;                        // rows of each operand staged by one CTA
 constexpr int BK = 64;                           // in-features per stage (one 128-byte swizzle row)
 constexpr int UK = 16;                           // K of one tcgen05.mma kind::f16
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;             // 16 KB
-constexpr int B_BYTES = BN * BK * 2;             // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 48 KB
+constexpr int STAGES = 6;
+constexpr int A_BYTES = HALF * BK * 2;           // 16 KB
+constexpr int B_BYTES = HALF * BK * 2;           // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 32 KB per CTA
 constexpr int NUM_ACC = 2;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int PROD_WARPS = 8;
 constexpr int THREADS = 192 + 32 * PROD_WARPS;
 constexpr int BANDS_PER_GROUP = 8;               // tile raster: 8 dW bands advance together over X
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+constexpr int PARTIALS_PER_TILE = 8;             // 2 CTAs x 4 lane quarters, 32 token rows each
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 
 struct Params {
@@ -46,7 +52,7 @@ struct Params {
   int n_bands;        // bands this launch covers
   int num_kb;         // K / BK
   int num_tiles;      // n_tiles_n * n_bands
-  double* partials;   // [all bands][n_tiles_n][4]
+  double* partials;   // [all bands][n_tiles_n][PARTIALS_PER_TILE]
   DeviceStatus* status;
   uint64_t limit_ns;
   unsigned flags;
@@ -88,7 +94,22 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, DeviceS
   }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+// Bounded wait until every producer warp has published candidate `cand`.
+__device__ __forceinline__ bool wait_produced(const Params& p, int cand, DeviceStatus* st) {
+  const uint64_t t0 = global_timer_ns();
+  while (ld_acquire_u32(p.produced + cand) < static_cast<unsigned int>(p.items_per_cand)) {
+    if (status_code(st) != 0u) return false;
+    if (global_timer_ns() - t0 > p.limit_ns) {
+      raise_timeout(st, kSiteTmaProduced);
+      return false;
+    }
+    __nanosleep(256);
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     loss_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmD,
                      Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -98,6 +119,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();  // 0 = even CTA (issues the MMAs), 1 = odd CTA
   const uint32_t bar0 = smem_u32(&bars[0]);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -111,98 +133,77 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(full_bar(s), 1);   // the even CTA's TMA thread arms it for both CTAs' bytes
+      mbar_init(empty_bar(s), 1);  // one multicast commit per consumed stage
     }
     for (int a = 0; a < NUM_ACC; ++a) {
       mbar_init(accf_bar(a), 1);
-      mbar_init(acce_bar(a), 4);
+      mbar_init(acce_bar(a), 8);   // 4 epilogue warps in each CTA of the pair
     }
     mbar_init(drain_bar, 1);
     mbar_init(never_bar, 1);
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), TMEM_COLS);
+  if (warp == 1) tmem_alloc_pair(smem_u32(&tmem_slot), TMEM_COLS);
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmD);
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any remote arrive or transaction
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   DeviceStatus* st = p.status;
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int n_pairs = static_cast<int>(gridDim.x >> 1);
 
   if (warp == 0) {
-    // ------------------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------------------ TMA
     if (elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t pending = 0, pend_phase = 0;
       bool ok = true;
-      int ready = -1;  // candidates < ready + 1 are known to be fully produced
-      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+      int ready = -1;  // candidates <= ready are known to be fully produced
+      for (int t = pair; ok && t < p.num_tiles; t += n_pairs) {
         int band, nt;
         tile_coords(t, p, band, nt);
         const int cand = band / p.tiles_o;
         if (cand > ready) {
-          const uint64_t t0 = global_timer_ns();
-          while (ld_acquire_u32(p.produced + cand) < static_cast<unsigned int>(p.items_per_cand)) {
-            if (status_code(st) != 0u) {
-              ok = false;
-              break;
-            }
-            if (global_timer_ns() - t0 > p.limit_ns) {
-              raise_timeout(st, kSiteTmaProduced);
-              ok = false;
-              break;
-            }
-            __nanosleep(256);
+          if (!wait_produced(p, cand, st)) {
+            ok = false;
+            break;
           }
-          if (!ok) break;
-          fence_proxy_async_global();
           ready = cand;
         }
+        const int32_t a_row = nt * BM + static_cast<int32_t>(rank) * HALF;
+        const int32_t b_row = band * BN + static_cast<int32_t>(rank) * HALF;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, st, p.limit_ns, kSiteTmaEmpty)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
-          tma_load_2d(a_tile(stage), &tmX, kb * BK, nt * BM, full_bar(stage));
-          tma_load_2d(b_tile(stage), &tmD, kb * BK, band * BN, full_bar(stage));
-          pending |= 1u << stage;
-          pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
+          const uint32_t fb = map_to_rank(full_bar(stage), 0);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          tma_load_2d_pair(a_tile(stage), &tmX, kb * BK, a_row, fb);
+          tma_load_2d_pair(b_tile(stage), &tmD, kb * BK, b_row, fb);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-      if (status_code(st) != 0u) {
-        // Wait (bounded) for this thread's copies still in flight before the CTA may exit.
-        for (int s = 0; s < STAGES; ++s)
-          if (pending & (1u << s)) {
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(full_bar(s), (pend_phase >> s) & 1u))
-              if (global_timer_ns() - t0 > p.limit_ns) {
-                raise_timeout(st, kSiteDrainTma);
-                break;
-              }
-          }
-      }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
+    // ------------------------------------------------------------------------------ MMA (even CTA)
+    if (rank == 0 && elect_one()) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       if (p.flags & AWQ_FLAG_INJECT_STALL) ok = mbar_wait(never_bar, 0u, st, p.limit_ns, kSiteMmaInjected);
       int local = 0;
-      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++local) {
+      for (int t = pair; ok && t < p.num_tiles; t += n_pairs, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, st, p.limit_ns, kSiteMmaAccEmpty)) {
@@ -220,19 +221,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t a0 = a_tile(stage), b0 = b_tile(stage);
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk)
-            umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * UK * 2), smem_desc_sw128(b0 + kk * UK * 2), IDESC,
-                      (kb | kk) != 0 ? 1u : 0u);
-          umma_commit(empty_bar(stage));
+            umma_bf16_pair(d_tmem, smem_desc_sw128(a0 + kk * UK * 2), smem_desc_sw128(b0 + kk * UK * 2), IDESC,
+                           (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair(empty_bar(stage), 0x3);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(accf_bar(acc));
+        umma_commit_pair(accf_bar(acc), 0x3);
       }
-      // Every MMA this thread issued must be complete before tensor memory is released.
-      umma_commit(drain_bar);
+      // Every MMA this thread issued must be complete before either CTA releases tensor memory or
+      // shared memory.
+      umma_commit_pair(drain_bar, 0x1);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(drain_bar, 0u))
         if (global_timer_ns() - t0 > p.limit_ns) {
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     int local = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+    for (int t = pair; t < p.num_tiles; t += n_pairs, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
       if (!warp_wait(accf_bar(acc), acc_phase, st, p.limit_ns, kSiteEpiAccFull)) break;
@@ -282,23 +284,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce_bar(acc));
+      if (lane == 0) mbar_arrive_remote(map_to_rank(acce_bar(acc), 0));
       double ds = static_cast<double>(sum);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ds = __dadd_rn(ds, __shfl_xor_sync(0xffffffffu, ds, off));
       if (lane == 0) {
         int band, nt;
         tile_coords(t, p, band, nt);
-        p.partials[(static_cast<int64_t>(band) * p.n_tiles_n + nt) * 4 + quarter] = ds;
+        p.partials[(static_cast<int64_t>(band) * p.n_tiles_n + nt) * PARTIALS_PER_TILE + rank * 4 + quarter] = ds;
       }
     }
   }
 
+  if (status_code(st) != 0u) {
+    // After a timeout some copies into this CTA's shared memory may still be in flight (their
+    // completion is counted on the even CTA's barrier, which may never be waited on): give them time
+    // to land before the pair releases its memory.
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 50000ull) __nanosleep(1000);
+  }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // no CTA of the pair leaves while its peer may still touch its memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
