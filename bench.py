@@ -17,7 +17,6 @@ CPU oracle on a bounded sample of the same workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
-import dataclasses
 import hashlib
 import json
 import os
@@ -34,7 +33,7 @@ sys.path.insert(0, ROOT)
 METRIC = "AWQ search candidates/sec per layer and effective TFLOP/s vs BF16 peak"
 UNIT = "candidates/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-GEMM_SOURCES = ["kernel_loss_gemm.cuh", "ptx.cuh"]
+GEMM_SOURCES = ["kernel_loss_gemm.cuh", "ptx.cuh", "kernels_simple.cuh", "numerics.cuh"]
 
 
 def parse_args():
@@ -233,15 +232,14 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
-    from weight_only_quantization_act_b200 import awq, inputs
+    from weight_only_quantization_act_b200 import awq, inputs, replicas  # noqa: F401
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     awq.load_library()
     wl = inputs.workload(args.workload)
     # each rank quantizes its own layer: same shapes, its own draw
-    seed_wl = wl if rank == 0 else dataclasses.replace(wl, number=wl.number + 1000 * rank)
-    X, W, _ = inputs.make_inputs(seed_wl)
+    X, W, _ = inputs.make_inputs(replicas.replica_workload(wl, rank))
     Xh = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16)
     Wh = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16)
     Xd, Wd = Xh.to(dev), Wh.to(dev)
@@ -299,28 +297,22 @@ def run_ours(args, rank, world, local_rank):
     search_ms = [e[1].elapsed_time(e[4]) for e in ev]
     gemm_ms = [e[2].elapsed_time(e[3]) for e in ev]
     pack_ms = [e[4].elapsed_time(e[5]) for e in ev]
-    total_ms = float(np.sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = replicas.max_over_ranks(float(np.sum(step_ms)), dev)
 
     # correctness guard on the timed result (cheap): a valid ratio and finite losses
     best = int(res.best_j.item())
     assert 0 <= best < J and torch.isfinite(res.losses).all()
 
     e2e = None if args.no_e2e else measure_e2e(args, Xh, Wh, dev, J)
-    if world > 1:
-        e2e_t = torch.tensor([e2e["ms"] if e2e else 0.0], dtype=torch.float64, device=dev)
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-        if e2e:
-            e2e["ms"] = float(e2e_t.item())
+    e2e_ms = replicas.max_over_ranks(e2e["ms"] if e2e else 0.0, dev)
+    if e2e:
+        e2e["ms"] = e2e_ms
 
     if rank != 0:
         return
     peaks, peaks_src = load_peaks()
     ms_per_step = total_ms / args.steps
-    value = J * world * args.steps / (total_ms / 1e3)
+    value = replicas.job_throughput(J * args.steps, world, total_ms / 1e3)
     flops = J * 2.0 * N * O * K
     gemm_avg_s = float(np.mean(gemm_ms)) / 1e3
     achieved_tflops = flops / gemm_avg_s / 1e12
@@ -356,7 +348,7 @@ def run_ours(args, rank, world, local_rank):
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if e2e is not None:
-        line["e2e"] = {"value": J * world / (e2e["ms"] / 1e3), "unit": UNIT,
+        line["e2e"] = {"value": replicas.job_throughput(J, world, e2e["ms"] / 1e3), "unit": UNIT,
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                        "ms_per_step": e2e["ms"]}
     print(json.dumps(line), flush=True)
