@@ -66,6 +66,8 @@ awq_status device_info(DeviceInfo** out) {
   if (!d.gemm_attr_set) {
     AWQ_CUDA(cudaFuncSetAttribute(awq::lg::loss_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   awq::lg::SMEM_BYTES));
+    AWQ_CUDA(cudaFuncSetAttribute(awq::act_chunk_sums_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::kActSmemBytes));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(d.sms & ~1));
     cfg.blockDim = dim3(awq::lg::THREADS);
@@ -154,7 +156,7 @@ SearchLayout search_layout(int64_t N, int64_t K, int64_t O, int n_grid) {
   l.tiles_o = l.O_pad / awq::lg::BN;
   l.sl = scale_layout(K, n_grid);
   size_t off = 0;
-  l.status_off = off;              // DeviceStatus (16 B)
+  l.status_off = off;              // DeviceStatus (16 B), then the finalize block counter (4 B)
   l.produced_off = off + 256;      // unsigned produced[AWQ_MAX_N_GRID]
   off += 512;
   l.table_off = off;
@@ -251,7 +253,8 @@ awq_status awq_act_stats(const void* X, int64_t N, int64_t K, int64_t ldx, void*
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   double* part = static_cast<double*>(workspace);
   dim3 grid(static_cast<unsigned>((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock), l.n_chunks);
-  awq::act_chunk_sums_kernel<<<grid, awq::kActThreads, 0, st>>>(static_cast<const uint16_t*>(X), N, K, ldx, part);
+  awq::act_chunk_sums_kernel<<<grid, awq::kActThreads, awq::kActSmemBytes, st>>>(static_cast<const uint16_t*>(X), N, K,
+                                                                                 ldx, part);
   AWQ_TRY(check_launch("act_chunk_sums_kernel"));
   awq::act_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(part, N, K, l.n_chunks, act_mean);
   AWQ_TRY(check_launch("act_finalize_kernel"));
@@ -365,6 +368,12 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   p.prod.exact = (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0;
   p.items_per_cand = l.O_pad * p.prod.segs;
   p.produced = produced;
+  // L2 residency (126 MB on B200): X is read by every candidate band and W once per candidate; keep
+  // them resident when they fit next to the streaming weight errors.
+  const double x_bytes = 2.0 * static_cast<double>(N) * static_cast<double>(K);
+  const double w_bytes = 2.0 * static_cast<double>(O) * static_cast<double>(K);
+  p.keep_x = x_bytes <= 64.0e6 ? 1 : 0;
+  p.prod.keep_w = (p.keep_x ? x_bytes : 0.0) + w_bytes <= 80.0e6 ? 1 : 0;
 
   // As many CTA pairs as fit at once, launched cooperatively: the TMA warps wait for rows that the
   // producer warps of every other CTA write, which is only safe when all CTAs are resident together.
@@ -383,9 +392,10 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   AWQ_TRY(check_launch("loss_gemm_kernel"));
   if (g_prof_after != nullptr) AWQ_CUDA(cudaEventRecord(g_prof_after, st));
 
-  awq::finalize_kernel<<<1, 1024, 0, st>>>(partials, l.tiles_o * l.tiles_n * awq::lg::PARTIALS_PER_TILE, n_grid,
-                                           static_cast<double>(N) * static_cast<double>(O), table, K, losses,
-                                           best_j, scales, status);
+  awq::finalize_kernel<<<n_grid, awq::kFinThreads, 0, st>>>(
+      partials, l.tiles_o * l.tiles_n * awq::lg::PARTIALS_PER_TILE, n_grid,
+      static_cast<double>(N) * static_cast<double>(O), table, K, losses, best_j, scales, status,
+      reinterpret_cast<unsigned int*>(ws + l.status_off + 16));
   AWQ_TRY(check_launch("finalize_kernel"));
   return ok();
 }
@@ -416,11 +426,12 @@ awq_status awq_quantize_pack_ex(const void* W, int64_t O, int64_t K, int64_t ldw
   if (K % 128 != 0) return fail(AWQ_ERR_INVALID_ARG, "K (%lld) must be a multiple of 128", static_cast<long long>(K));
   if (scales == nullptr || codes == nullptr || steps == nullptr || zeros == nullptr)
     return fail(AWQ_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(scales)) return fail(AWQ_ERR_INVALID_ARG, "scales is not 16-byte aligned");
+  if (!aligned16(scales) || !aligned16(codes))
+    return fail(AWQ_ERR_INVALID_ARG, "scales and codes must be 16-byte aligned");
   if (flags & ~AWQ_FLAG_EXACT_DIVISION) return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   DeviceInfo* d = nullptr;
   AWQ_TRY(device_info(&d));
-  const int64_t segs = (K + 255) / 256;
+  const int64_t segs = (K + awq::kPackWarpCols - 1) / awq::kPackWarpCols;
   const int64_t blocks = (O * segs * 32 + awq::kPackThreads - 1) / awq::kPackThreads;
   awq::quantize_pack_kernel<<<static_cast<unsigned>(blocks), awq::kPackThreads, 0,
                               reinterpret_cast<cudaStream_t>(stream)>>>(
@@ -496,7 +507,8 @@ extern "C" awq_status awq_act_stats_noalloc(const void* X, int64_t N, int64_t K,
   // Each (chunk, column) entry the finaliser reads is written first by this call, so the scratch needs
   // no clearing; what the previous call left there is simply overwritten.
   dim3 grid(static_cast<unsigned>((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock), l.n_chunks);
-  awq::act_chunk_sums_kernel<<<grid, awq::kActThreads, 0, st>>>(static_cast<const uint16_t*>(X), N, K, ldx, part);
+  awq::act_chunk_sums_kernel<<<grid, awq::kActThreads, awq::kActSmemBytes, st>>>(static_cast<const uint16_t*>(X), N, K,
+                                                                                 ldx, part);
   AWQ_TRY(check_launch("act_chunk_sums_kernel"));
   awq::act_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(part, N, K, l.n_chunks, act_mean);
   AWQ_TRY(check_launch("act_finalize_kernel"));

@@ -61,6 +61,7 @@ struct Params {
   ProducerArgs prod;         // weight-error production for every candidate
   int64_t items_per_cand;    // producer work items (warp x 512 in-features) per candidate
   unsigned int* produced;    // [n_grid] finished items per candidate (zeroed before launch)
+  int keep_x;                // X is re-read by every band: ask L2 to keep it (evict_last)
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& band, int& nt) {
@@ -165,6 +166,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       int ready = -1;  // candidates <= ready are known to be fully produced
+      const uint64_t pol_x = p.keep_x ? policy_evict_last() : policy_evict_normal();
+      const uint64_t pol_d = policy_evict_normal();
       for (int t = pair; ok && t < p.num_tiles; t += n_pairs) {
         int band, nt;
         tile_coords(t, p, band, nt);
@@ -185,8 +188,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
           if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-          tma_load_2d_pair(a_tile(stage), &tmX, kb * BK, a_row, fb);
-          tma_load_2d_pair(b_tile(stage), &tmD, kb * BK, b_row, fb);
+          tma_load_2d_pair_hint(a_tile(stage), &tmX, kb * BK, a_row, fb, pol_x);
+          tma_load_2d_pair_hint(b_tile(stage), &tmD, kb * BK, b_row, fb, pol_d);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;

@@ -14,42 +14,77 @@ namespace awq {
 // order (256-row chunks; rows in increasing order inside a chunk; chunk totals in chunk order).
 // ===================================================================================================
 constexpr int kMaxGrid = 64;  // largest n_grid (AWQ_MAX_N_GRID)
-constexpr int kActChunk = 256;
-constexpr int kActThreads = 256;
-constexpr int kActColsPerThread = 2;
-constexpr int kActColsPerBlock = kActThreads * kActColsPerThread;
-constexpr int kActUnroll = 32;
+constexpr int kActChunk = 256;          // rows per chunk of the fixed-order sum
+constexpr int kActThreads = 256;        // one column per thread
+constexpr int kActColsPerBlock = kActThreads;
+constexpr int kActStageRows = 16;       // rows per cp.async stage (16 x 512 B = 8 KB)
+constexpr int kActStages = 8;           // stages in flight per CTA (64 KB)
+constexpr int kActSmemBytes = kActStages * kActStageRows * kActColsPerBlock * 2;
 
-// grid (ceil(K / 512), n_chunks): thread owns 2 adjacent columns of one chunk and walks its rows.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int Pending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(Pending) : "memory");
+}
+
+// grid (ceil(K / 256), n_chunks). The CTA streams its chunk's 256-column slab through shared memory
+// with cp.async (8 stages of 16 rows in flight); thread t then adds column t's values in row order.
 __global__ void __launch_bounds__(kActThreads) act_chunk_sums_kernel(const uint16_t* __restrict__ X,
                                                                      int64_t N, int64_t K, int64_t ldx,
                                                                      double* __restrict__ part) {
-  const int64_t c = (static_cast<int64_t>(blockIdx.x) * kActThreads + threadIdx.x) * kActColsPerThread;
-  if (c >= K) return;
+  extern __shared__ __align__(16) uint16_t act_stage[];  // [kActStages][kActStageRows][256]
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kActColsPerBlock;
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kActChunk;
-  const int64_t r1 = min(N, r0 + kActChunk);
-  const int64_t stride = ldx / 2;  // in 32-bit words
-  const uint32_t* p = reinterpret_cast<const uint32_t*>(X + r0 * ldx + c);
-  double s0 = 0.0, s1 = 0.0;
-  int64_t i = r0;
-  for (; i + kActUnroll <= r1; i += kActUnroll) {
-    uint32_t v[kActUnroll];
+  const int rows = static_cast<int>(min(static_cast<int64_t>(kActChunk), N - r0));
+  const int n_stages = (rows + kActStageRows - 1) / kActStageRows;
+  // copy assignment: each thread moves 2 x 16 B of a stage (rows tid/32 and tid/32 + 8, piece tid%32)
+  const int piece = threadIdx.x & 31;
+  const int64_t pcol = c0 + piece * 8;
+  const uint32_t pbytes = pcol >= K ? 0u : static_cast<uint32_t>(min(static_cast<int64_t>(8), K - pcol) * 2);
+  const uint32_t smem0 = static_cast<uint32_t>(__cvta_generic_to_shared(act_stage));
+  auto issue = [&](int stg) {
+    if (stg < n_stages) {
+      const int slot = stg % kActStages;
 #pragma unroll
-    for (int u = 0; u < kActUnroll; ++u) v[u] = __ldcs(p + (i - r0 + u) * stride);
-#pragma unroll
-    for (int u = 0; u < kActUnroll; ++u) {
-      s0 = __dadd_rn(s0, fabs(static_cast<double>(bf16_lo(v[u]))));
-      s1 = __dadd_rn(s1, fabs(static_cast<double>(bf16_hi(v[u]))));
+      for (int h = 0; h < 2; ++h) {
+        const int rr = (threadIdx.x >> 5) + 8 * h;
+        const int row = stg * kActStageRows + rr;
+        const uint32_t dst = smem0 + static_cast<uint32_t>(((slot * kActStageRows + rr) * kActColsPerBlock +
+                                                            piece * 8) * 2);
+        const bool ok = row < rows && pbytes != 0u;
+        const uint16_t* src = ok ? X + (r0 + row) * ldx + pcol : X;
+        cp_async_16(dst, src, ok ? pbytes : 0u);
+      }
     }
+    cp_async_commit();  // an empty group keeps the wait arithmetic uniform
+  };
+#pragma unroll 1
+  for (int stg = 0; stg < kActStages - 1; ++stg) issue(stg);
+  const int64_t col = c0 + threadIdx.x;
+  double sum = 0.0;
+#pragma unroll 1
+  for (int stg = 0; stg < n_stages; ++stg) {
+    issue(stg + kActStages - 1);
+    cp_async_wait<kActStages - 1>();
+    __syncthreads();
+    const int slot = stg % kActStages;
+    const int nr = min(kActStageRows, rows - stg * kActStageRows);
+    const uint16_t* sp = act_stage + (slot * kActStageRows) * kActColsPerBlock + threadIdx.x;
+    if (nr == kActStageRows) {
+#pragma unroll
+      for (int r = 0; r < kActStageRows; ++r)
+        sum = __dadd_rn(sum, fabs(static_cast<double>(__uint_as_float(static_cast<uint32_t>(sp[r * kActColsPerBlock]) << 16))));
+    } else {
+      for (int r = 0; r < nr; ++r)
+        sum = __dadd_rn(sum, fabs(static_cast<double>(__uint_as_float(static_cast<uint32_t>(sp[r * kActColsPerBlock]) << 16))));
+    }
+    __syncthreads();  // the slot is refilled by the next iteration's issue
   }
-  for (; i < r1; ++i) {
-    const uint32_t v = __ldcs(p + (i - r0) * stride);
-    s0 = __dadd_rn(s0, fabs(static_cast<double>(bf16_lo(v))));
-    s1 = __dadd_rn(s1, fabs(static_cast<double>(bf16_hi(v))));
-  }
-  double* out = part + static_cast<int64_t>(blockIdx.y) * K + c;
-  out[0] = s0;
-  out[1] = s1;
+  cp_async_wait<0>();
+  if (col < K) part[static_cast<int64_t>(blockIdx.y) * K + col] = sum;
 }
 
 // grid ceil(K / 256): chunk totals in chunk order, then the mean.
@@ -157,6 +192,7 @@ struct ProducerArgs {
   const float* rtable;             // [n_grid][K] RN32(1 / scale)
   __nv_bfloat16* dW;               // [n_grid * O_pad][K]
   int exact;                       // AWQ_FLAG_EXACT_DIVISION
+  int keep_w;                      // W is re-read once per candidate: ask L2 to keep it (evict_last)
 };
 
 // Weight errors of one row of one 512-in-feature segment for candidate j, from the row's raw bf16 words.
@@ -219,19 +255,20 @@ __device__ __forceinline__ unsigned int produce_rows(const ProducerArgs& a, int6
     for (int i = 0; i < kProdCols; ++i) { s[i] = 1.0f; rs[i] = 1.0f; }
   }
   unsigned int count = 0;
+  const uint64_t pol = a.keep_w ? policy_evict_last() : policy_evict_normal();
   uint4 nxt[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
   if (o_first < a.O && active) {
     const uint4* src = reinterpret_cast<const uint4*>(a.W + o_first * a.ldw + k0);
-    nxt[0] = __ldg(src);
-    nxt[1] = __ldg(src + 1);
+    nxt[0] = ldg_v4_policy(src, pol);
+    nxt[1] = ldg_v4_policy(src + 1, pol);
   }
   for (int64_t o = o_first; o < a.O_pad; o += o_step) {
     const uint4 cur[2] = {nxt[0], nxt[1]};
     const int64_t on = o + o_step;
     if (on < a.O && active) {
       const uint4* src = reinterpret_cast<const uint4*>(a.W + on * a.ldw + k0);
-      nxt[0] = __ldg(src);
-      nxt[1] = __ldg(src + 1);
+      nxt[0] = ldg_v4_policy(src, pol);
+      nxt[1] = ldg_v4_policy(src + 1, pol);
     }
     uint32_t outw[8];
     produce_row(a, cur, s, rs, o < a.O, outw);
@@ -249,31 +286,48 @@ __device__ __forceinline__ unsigned int produce_rows(const ProducerArgs& a, int6
 // (4)-(5) finalisation: loss_j = (sum of the tile partials in a fixed order) / (N * O); best_j is the
 // first index of the minimum; scales = row best_j of the table. Single block of 1024 threads.
 // ===================================================================================================
-__global__ void __launch_bounds__(1024) finalize_kernel(const double* __restrict__ partials,
-                                                        int64_t per_cand, int n_grid, double denom,
-                                                        const float* __restrict__ table, int64_t K,
-                                                        double* __restrict__ losses, int* __restrict__ best_j,
-                                                        float* __restrict__ scales,
-                                                        const DeviceStatus* st) {
-  __shared__ double loss_sh[kMaxGrid];
+// grid n_grid blocks of 256: block j sums candidate j's tile partials in a fixed order (thread t takes
+// entries t, t + 256, ... in order; then a fixed tree), so the result does not depend on scheduling. The
+// last block to finish (counter in the zeroed status block) takes the first minimum and copies the
+// scales of the best ratio.
+constexpr int kFinThreads = 256;
+
+__global__ void __launch_bounds__(kFinThreads) finalize_kernel(const double* __restrict__ partials,
+                                                               int64_t per_cand, int n_grid, double denom,
+                                                               const float* __restrict__ table, int64_t K,
+                                                               double* __restrict__ losses, int* __restrict__ best_j,
+                                                               float* __restrict__ scales, const DeviceStatus* st,
+                                                               unsigned int* done_blocks) {
+  __shared__ double red[kFinThreads];
+  __shared__ int last_sh;
   __shared__ int best_sh;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x;
   const bool failed = status_code(st) != 0u;
-  for (int j = warp; j < n_grid; j += 32) {
-    double acc = 0.0;
-    const double* p = partials + static_cast<int64_t>(j) * per_cand;
-    for (int64_t i = lane; i < per_cand; i += 32) acc = __dadd_rn(acc, p[i]);
+  double acc = 0.0;
+  const double* p = partials + static_cast<int64_t>(j) * per_cand;
+  for (int64_t i = threadIdx.x; i < per_cand; i += kFinThreads) acc = __dadd_rn(acc, p[i]);
+  red[threadIdx.x] = acc;
+  __syncthreads();
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc = __dadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
-    if (lane == 0) loss_sh[j] = failed ? __longlong_as_double(0x7ff8000000000000ll) : __ddiv_rn(acc, denom);
+  for (int w = kFinThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] = __dadd_rn(red[threadIdx.x], red[threadIdx.x + w]);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    losses[j] = failed ? __longlong_as_double(0x7ff8000000000000ll) : __ddiv_rn(red[0], denom);
+    __threadfence();
+    last_sh = atomicAdd(done_blocks, 1u) == static_cast<unsigned int>(n_grid - 1);
   }
   __syncthreads();
-  if (warp == 0) {
+  if (!last_sh) return;
+  __threadfence();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
     double v = __longlong_as_double(0x7ff0000000000000ll);
     int idx = 0x7fffffff;
-    for (int j = lane; j < n_grid; j += 32) {
-      const double l = loss_sh[j];
-      if (l < v) { v = l; idx = j; }
+    for (int c = lane; c < n_grid; c += 32) {
+      const double l = *reinterpret_cast<volatile double*>(losses + c);
+      if (l < v) { v = l; idx = c; }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -288,10 +342,9 @@ __global__ void __launch_bounds__(1024) finalize_kernel(const double* __restrict
     }
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < n_grid; j += blockDim.x) losses[j] = loss_sh[j];
   const int b = best_sh;
   if (b >= 0)
-    for (int64_t k = threadIdx.x; k < K; k += blockDim.x) scales[k] = table[static_cast<int64_t>(b) * K + k];
+    for (int64_t k = threadIdx.x; k < K; k += kFinThreads) scales[k] = table[static_cast<int64_t>(b) * K + k];
 }
 
 // ===================================================================================================
@@ -299,51 +352,62 @@ __global__ void __launch_bounds__(1024) finalize_kernel(const double* __restrict
 // 16 lanes per group; one warp covers 256 in-features of one row.
 // ===================================================================================================
 constexpr int kPackThreads = 256;
+constexpr int kPackCols = 32;                    // in-features per lane (4 lanes per group of 128)
+constexpr int kPackWarpCols = 32 * kPackCols;    // 1024 in-features of one row per warp
 
 __global__ void __launch_bounds__(kPackThreads) quantize_pack_kernel(
     const uint16_t* __restrict__ W, int64_t O, int64_t K, int64_t ldw, const float* __restrict__ scales,
     int exact, uint32_t* __restrict__ codes, float* __restrict__ steps, float* __restrict__ zeros) {
-  const int64_t segs = (K + 255) / 256;
+  const int64_t segs = (K + kPackWarpCols - 1) / kPackWarpCols;
   const int64_t gw = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
-  if (gw >= O * segs) return;
+  if (gw >= O * segs) return;  // whole warps exit together
   const int lane = threadIdx.x & 31;
   const int64_t o = gw / segs;
-  const int64_t k0 = (gw - o * segs) * 256 + static_cast<int64_t>(lane) * 8;
-  const bool active = k0 < K;
-  float wp[8];
+  const int64_t k0 = (gw - o * segs) * kPackWarpCols + static_cast<int64_t>(lane) * kPackCols;
+  const bool active = k0 < K;  // K % 128 == 0: 4-lane groups are all active or all idle
+  float wp[kPackCols];
   float mx = -__int_as_float(0x7f800000), mn = __int_as_float(0x7f800000);
   if (active) {
-    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(W + o * ldw + k0));
-    const float4 s0 = __ldg(reinterpret_cast<const float4*>(scales + k0));
-    const float4 s1 = __ldg(reinterpret_cast<const float4*>(scales + k0) + 1);
-    const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-    const uint32_t u[4] = {a.x, a.y, a.z, a.w};
+    const uint4* src = reinterpret_cast<const uint4*>(W + o * ldw + k0);
+    const float4* ps = reinterpret_cast<const float4*>(scales + k0);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      wp[2 * i] = __fmul_rn(bf16_lo(u[i]), s[2 * i]);
-      wp[2 * i + 1] = __fmul_rn(bf16_hi(u[i]), s[2 * i + 1]);
+    for (int v = 0; v < 4; ++v) {
+      const uint4 u = __ldcs(src + v);
+      const float4 s0 = __ldg(ps + 2 * v), s1 = __ldg(ps + 2 * v + 1);
+      const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+      const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        wp[8 * v + 2 * i] = __fmul_rn(bf16_lo(uu[i]), ss[2 * i]);
+        wp[8 * v + 2 * i + 1] = __fmul_rn(bf16_hi(uu[i]), ss[2 * i + 1]);
+      }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kPackCols; ++i) {
       mx = fmaxf(mx, wp[i]);
       mn = fminf(mn, wp[i]);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) wp[i] = 0.0f;
+    for (int i = 0; i < kPackCols; ++i) wp[i] = 0.0f;
   }
 #pragma unroll
-  for (int off = 1; off < 16; off <<= 1) {
+  for (int off = 1; off < 4; off <<= 1) {
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
   }
   if (!active) return;
   const GroupParams g = group_params(mx, mn);
-  uint32_t word = 0;
+  uint32_t word[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) word |= static_cast<uint32_t>(code_of(wp[i], g, exact != 0)) << (4 * i);
-  __stcs(codes + o * (K / 8) + k0 / 8, word);
-  if ((lane & 15) == 0) {
+  for (int w = 0; w < 4; ++w) {
+    word[w] = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      word[w] |= static_cast<uint32_t>(code_of(wp[8 * w + i], g, exact != 0)) << (4 * i);
+  }
+  __stcs(reinterpret_cast<uint4*>(codes + o * (K / 8) + k0 / 8), make_uint4(word[0], word[1], word[2], word[3]));
+  if ((lane & 3) == 0) {
     const int64_t gi = o * (K / 128) + k0 / 128;
     steps[gi] = g.step;
     zeros[gi] = g.zero;

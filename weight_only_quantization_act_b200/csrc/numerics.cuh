@@ -172,17 +172,20 @@ __device__ __forceinline__ GroupParams group_params(float mx, float mn) {
   return g;
 }
 
-// rint(RN32(wp / step)) exactly. The product wp * RN32(1/step) differs from the IEEE quotient by less
-// than 1.5 * 2^-23 relative, so it rounds to the same integer unless it lies within |qa| * 2^-20 of a
-// half-integer (or is huge); those rare cases take the IEEE division.
+// Exact rint(RN32(wp / step)) through the IEEE division; kept out of line so that the common path
+// below issues no division instructions.
+__device__ __noinline__ float rint_quotient_exact(float wp, float step) { return rintf(__fdiv_rn(wp, step)); }
+
+// rint(RN32(wp / step)) exactly. For |qa| < 64 the product qa = wp * RN32(1/step) is within
+// 1.5 * 2^-23 * 64 < 1.2e-5 of the real quotient, and RN32 moves the quotient by at most 2^-18, so the
+// two round to the same integer whenever qa is farther than 2^-14 from a half-integer. Only the rare
+// remaining cases (about one element in 10^4, and groups with the step at its floor) take the division.
 __device__ __forceinline__ float rint_quotient(float wp, const GroupParams& g, bool exact) {
-  if (exact) return rintf(__fdiv_rn(wp, g.step));
   const float qa = __fmul_rn(wp, g.rstep);
-  const float n = rintf(qa);
+  float n = rintf(qa);
   const float d = fabsf(__fsub_rn(qa, n));  // exact: n is within a factor 2 of qa, or n = 0
-  const float margin = __fmul_rn(fabsf(qa), 0x1p-20f);
-  if (__fsub_rn(0.5f, d) > margin && fabsf(qa) < 0x1p21f) return n;
-  return rintf(__fdiv_rn(wp, g.step));
+  if (exact || !(d < 0.5f - 0x1p-14f && fabsf(qa) < 64.0f)) n = rint_quotient_exact(wp, g.step);
+  return n;
 }
 
 // Code q = min(max(RN32(rint(RN32(w'/step)) + z), 0), 15).
