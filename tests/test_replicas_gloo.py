@@ -27,7 +27,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_gloo_ranks_replicas_and_max_timing():
     port = 29500 + (os.getpid() % 2000)
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
         res = dict(out)
