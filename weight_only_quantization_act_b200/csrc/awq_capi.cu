@@ -156,7 +156,7 @@ SearchLayout search_layout(int64_t N, int64_t K, int64_t O, int n_grid) {
   l.tiles_o = l.O_pad / awq::lg::BN;
   l.sl = scale_layout(K, n_grid);
   size_t off = 0;
-  l.status_off = off;              // DeviceStatus (16 B), then the finalize block counter (4 B)
+  l.status_off = off;  // DeviceStatus (16 B), finalize block counter (4 B), tile counter (4 B)
   l.produced_off = off + 256;      // unsigned produced[AWQ_MAX_N_GRID]
   off += 512;
   l.table_off = off;
@@ -368,6 +368,7 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   p.prod.exact = (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0;
   p.items_per_cand = l.O_pad * p.prod.segs;
   p.produced = produced;
+  p.tile_counter = reinterpret_cast<unsigned int*>(ws + l.status_off + 20);
   // L2 residency (126 MB on B200): X is read by every candidate band and W once per candidate; keep
   // them resident when they fit next to the streaming weight errors.
   const double x_bytes = 2.0 * static_cast<double>(N) * static_cast<double>(K);

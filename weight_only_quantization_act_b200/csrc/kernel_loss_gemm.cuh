@@ -7,7 +7,10 @@
 // squares and sums each row in fp32 and adds the 32 rows of each warp in fp64. E is never written to
 // global memory.
 //
-// Persistent cooperative kernel, clusters of 2 CTAs, one CTA per SM, 14 warps per CTA:
+// Persistent cooperative kernel, clusters of 2 CTAs, one CTA per SM, 14 warps per CTA. Tiles are handed
+// out dynamically: the even CTA's TMA thread takes the next tile index from a global counter (the tiles
+// in flight are then always a contiguous stretch of the raster, whose operands the pairs share in L2)
+// and publishes it through an 8-slot ring in both CTAs' shared memory, one mbarrier per slot; -1 ends.
 //   warp 0      TMA: X tile [128 x 64] and dW tile [128 x 64] per stage for this CTA, 128-byte
 //               swizzle; the bytes of both CTAs are counted on the even CTA's barrier
 //   warp 1      pair-wide tensor memory (512 columns = two 256-column fp32 accumulators); in the even
@@ -44,6 +47,7 @@ constexpr int THREADS = 192 + 32 * PROD_WARPS;
 constexpr int BANDS_PER_GROUP = 8;               // tile raster: 8 dW bands advance together over X
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
 constexpr int PARTIALS_PER_TILE = 8;             // 2 CTAs x 4 lane quarters, 32 token rows each
+constexpr int RING = 8;                          // tile-index slots; producers run <= 4 tiles ahead
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 
 struct Params {
@@ -62,6 +66,7 @@ struct Params {
   int64_t items_per_cand;    // producer work items (warp x 512 in-features) per candidate
   unsigned int* produced;    // [n_grid] finished items per candidate (zeroed before launch)
   int keep_x;                // X is re-read by every band: ask L2 to keep it (evict_last)
+  unsigned int* tile_counter;  // tiles handed out after each pair's first one (zeroed before launch)
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& band, int& nt) {
@@ -115,8 +120,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                      Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[2 * STAGES + 2 * NUM_ACC + 2];
+  __shared__ __align__(8) uint64_t bars[2 * STAGES + 2 * NUM_ACC + 2 + RING];
   __shared__ uint32_t tmem_slot;
+  __shared__ int tile_ring[RING];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -128,6 +134,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   auto acce_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + NUM_ACC + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * NUM_ACC);
   const uint32_t never_bar = drain_bar + 8u;
+  auto tile_bar = [&](int slot) { return never_bar + 8u + 8u * slot; };
   const uint32_t smem_base = smem_u32(smem);
   auto a_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s) * STAGE_BYTES; };
   auto b_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s) * STAGE_BYTES + A_BYTES; };
@@ -143,6 +150,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     mbar_init(drain_bar, 1);
     mbar_init(never_bar, 1);
+    for (int r = 0; r < RING; ++r) mbar_init(tile_bar(r), 1);  // the even CTA's TMA thread arrives
     fence_barrier_init();
     fence_proxy_async_smem();
   }
@@ -159,6 +167,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int n_pairs = static_cast<int>(gridDim.x >> 1);
 
+  // Tile index of this CTA's local tile i (waits for the even CTA's TMA thread to publish it).
+  auto ring_wait_thread = [&](int i, bool& ok) -> int {
+    const int slot = i % RING;
+    const uint32_t par = static_cast<uint32_t>(i / RING) & 1u;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait_cluster(tile_bar(slot), par)) {
+      if (status_code(st) != 0u || global_timer_ns() - t0 > p.limit_ns) {
+        if (status_code(st) == 0u) raise_timeout(st, kSiteTileRing);
+        ok = false;
+        return -1;
+      }
+    }
+    return *reinterpret_cast<volatile int*>(&tile_ring[slot]);
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------------------------ TMA
     if (elect_one()) {
@@ -168,7 +191,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int ready = -1;  // candidates <= ready are known to be fully produced
       const uint64_t pol_x = p.keep_x ? policy_evict_last() : policy_evict_normal();
       const uint64_t pol_d = policy_evict_normal();
-      for (int t = pair; ok && t < p.num_tiles; t += n_pairs) {
+      for (int i = 0; ok; ++i) {
+        int t;
+        if (rank == 0) {
+          // hand out the next tile: the pair's own first tile, then the shared counter
+          t = i == 0 ? pair : n_pairs + static_cast<int>(atomicAdd(p.tile_counter, 1u));
+          if (t >= p.num_tiles) t = -1;
+          const int slot = i % RING;
+          tile_ring[slot] = t;
+          st_shared_cluster_u32(map_to_rank(smem_u32(&tile_ring[slot]), 1), static_cast<uint32_t>(t));
+          mbar_arrive(tile_bar(slot));
+          mbar_arrive_remote(map_to_rank(tile_bar(slot), 1));
+        } else {
+          t = ring_wait_thread(i, ok);
+          if (!ok) break;
+        }
+        if (t < 0) break;
         int band, nt;
         tile_coords(t, p, band, nt);
         const int cand = band / p.tiles_o;
@@ -205,10 +243,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       if (p.flags & AWQ_FLAG_INJECT_STALL) ok = mbar_wait(never_bar, 0u, st, p.limit_ns, kSiteMmaInjected);
-      int local = 0;
-      for (int t = pair; ok && t < p.num_tiles; t += n_pairs, ++local) {
-        const int acc = local & 1;
-        const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
+      for (int i = 0; ok; ++i) {
+        const int t = ring_wait_thread(i, ok);
+        if (!ok || t < 0) break;
+        const int acc = i & 1;
+        const uint32_t acc_phase = static_cast<uint32_t>(i >> 1) & 1u;
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, st, p.limit_ns, kSiteMmaAccEmpty)) {
           ok = false;
           break;
@@ -269,10 +308,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else {
     // ------------------------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
-    int local = 0;
-    for (int t = pair; t < p.num_tiles; t += n_pairs, ++local) {
-      const int acc = local & 1;
-      const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
+    for (int i = 0;; ++i) {
+      // the tile's index (all lanes wait on the ring slot; the outcome is warp-uniform)
+      const int slot = i % RING;
+      const uint32_t par = static_cast<uint32_t>(i / RING) & 1u;
+      bool got = false;
+      {
+        uint64_t t0 = 0;
+        if (lane == 0) t0 = global_timer_ns();
+        for (uint32_t it = 0;; ++it) {
+          const bool done = mbar_try_wait_cluster(tile_bar(slot), par);
+          if (__all_sync(0xffffffffu, done)) {
+            got = true;
+            break;
+          }
+          int give_up = 0;
+          if (lane == 0 && (it & 63u) == 63u) {
+            if (status_code(st) != 0u) give_up = 1;
+            else if (global_timer_ns() - t0 > p.limit_ns) {
+              raise_timeout(st, kSiteTileRing);
+              give_up = 1;
+            }
+          }
+          if (__shfl_sync(0xffffffffu, give_up, 0)) break;
+        }
+      }
+      if (!got) break;
+      const int t = *reinterpret_cast<volatile int*>(&tile_ring[slot]);
+      if (t < 0) break;
+      const int acc = i & 1;
+      const uint32_t acc_phase = static_cast<uint32_t>(i >> 1) & 1u;
       if (!warp_wait(accf_bar(acc), acc_phase, st, p.limit_ns, kSiteEpiAccFull)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
@@ -283,7 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         float v[32];
         tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sum = fmaf(v[i], v[i], sum);
+        for (int k = 0; k < 32; ++k) sum = fmaf(v[k], v[k], sum);
       }
       tc_fence_before();
       __syncwarp();
