@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -432,8 +433,11 @@ awq_status awq_quantize_pack_ex(const void* W, int64_t O, int64_t K, int64_t ldw
   if (flags & ~AWQ_FLAG_EXACT_DIVISION) return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   DeviceInfo* d = nullptr;
   AWQ_TRY(device_info(&d));
+  // one resident wave of warps; each warp then walks rows of its segment
   const int64_t segs = (K + awq::kPackWarpCols - 1) / awq::kPackWarpCols;
-  const int64_t blocks = (O * segs * 32 + awq::kPackThreads - 1) / awq::kPackThreads;
+  const int64_t items = O * segs;
+  const int64_t max_blocks = static_cast<int64_t>(d->sms) * 2;  // 2 blocks of 256 threads fit per SM
+  const int64_t blocks = std::min<int64_t>(max_blocks, (items * 32 + awq::kPackThreads - 1) / awq::kPackThreads);
   awq::quantize_pack_kernel<<<static_cast<unsigned>(blocks), awq::kPackThreads, 0,
                               reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint16_t*>(W), O, K, ldw, scales, (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0, codes, steps,

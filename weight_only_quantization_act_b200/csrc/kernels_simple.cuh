@@ -353,64 +353,99 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(const double* __r
 // ===================================================================================================
 constexpr int kPackThreads = 256;
 constexpr int kPackCols = 32;                    // in-features per lane (4 lanes per group of 128)
-constexpr int kPackWarpCols = 32 * kPackCols;    // 1024 in-features of one row per warp
+constexpr int kPackWarpCols = 32 * kPackCols;    // 1024 in-features (one segment) per warp
 
+// Warp v owns segment v % segs and rows v / segs, v / segs + wps, ... (wps = warps per segment): the
+// segment's scales stay in registers and the next row's weights are loaded while the current row is
+// quantized. With fewer warps than segments a warp walks several whole segments.
 __global__ void __launch_bounds__(kPackThreads) quantize_pack_kernel(
     const uint16_t* __restrict__ W, int64_t O, int64_t K, int64_t ldw, const float* __restrict__ scales,
     int exact, uint32_t* __restrict__ codes, float* __restrict__ steps, float* __restrict__ zeros) {
   const int64_t segs = (K + kPackWarpCols - 1) / kPackWarpCols;
-  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
-  if (gw >= O * segs) return;  // whole warps exit together
+  const int64_t v = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
+  const int64_t total = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t o = gw / segs;
-  const int64_t k0 = (gw - o * segs) * kPackWarpCols + static_cast<int64_t>(lane) * kPackCols;
-  const bool active = k0 < K;  // K % 128 == 0: 4-lane groups are all active or all idle
-  float wp[kPackCols];
-  float mx = -__int_as_float(0x7f800000), mn = __int_as_float(0x7f800000);
-  if (active) {
-    const uint4* src = reinterpret_cast<const uint4*>(W + o * ldw + k0);
-    const float4* ps = reinterpret_cast<const float4*>(scales + k0);
+  int64_t seg_first, seg_step, row_first, row_step;
+  if (total >= segs) {
+    const int64_t wps = total / segs;
+    if (v >= wps * segs) return;  // whole warps exit together
+    seg_first = v % segs;
+    seg_step = segs;  // one segment
+    row_first = v / segs;
+    row_step = wps;
+  } else {
+    seg_first = v;
+    seg_step = total;
+    row_first = 0;
+    row_step = 1;
+  }
+  for (int64_t seg = seg_first; seg < segs; seg += seg_step) {
+    const int64_t k0 = seg * kPackWarpCols + static_cast<int64_t>(lane) * kPackCols;
+    const bool active = k0 < K;  // K % 128 == 0: 4-lane groups are all active or all idle
+    float s[kPackCols];
+    if (active) {
+      const float4* ps = reinterpret_cast<const float4*>(scales + k0);
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const uint4 u = __ldcs(src + v);
-      const float4 s0 = __ldg(ps + 2 * v), s1 = __ldg(ps + 2 * v + 1);
-      const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
-      const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      for (int i = 0; i < kPackCols / 4; ++i) {
+        const float4 x = __ldg(ps + i);
+        s[4 * i] = x.x; s[4 * i + 1] = x.y; s[4 * i + 2] = x.z; s[4 * i + 3] = x.w;
+      }
+    } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        wp[8 * v + 2 * i] = __fmul_rn(bf16_lo(uu[i]), ss[2 * i]);
-        wp[8 * v + 2 * i + 1] = __fmul_rn(bf16_hi(uu[i]), ss[2 * i + 1]);
+      for (int i = 0; i < kPackCols; ++i) s[i] = 1.0f;
+    }
+    uint4 nxt[4] = {};
+    if (row_first < O && active) {
+      const uint4* src = reinterpret_cast<const uint4*>(W + row_first * ldw + k0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) nxt[i] = __ldcs(src + i);
+    }
+    for (int64_t o = row_first; o < O; o += row_step) {
+      const uint4 cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
+      const int64_t on = o + row_step;
+      if (on < O && active) {
+        const uint4* src = reinterpret_cast<const uint4*>(W + on * ldw + k0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) nxt[i] = __ldcs(src + i);
+      }
+      float wp[kPackCols];
+      float mx = -__int_as_float(0x7f800000), mn = __int_as_float(0x7f800000);
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4) {
+        const uint32_t uu[4] = {cur[v4].x, cur[v4].y, cur[v4].z, cur[v4].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          wp[8 * v4 + 2 * i] = __fmul_rn(bf16_lo(uu[i]), s[8 * v4 + 2 * i]);
+          wp[8 * v4 + 2 * i + 1] = __fmul_rn(bf16_hi(uu[i]), s[8 * v4 + 2 * i + 1]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kPackCols; ++i) {
+        mx = fmaxf(mx, wp[i]);
+        mn = fminf(mn, wp[i]);
+      }
+#pragma unroll
+      for (int off = 1; off < 4; off <<= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      }
+      if (!active) continue;
+      const GroupParams g = group_params(mx, mn);
+      uint32_t word[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        word[w] = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          word[w] |= static_cast<uint32_t>(code_of(wp[8 * w + i], g, exact != 0)) << (4 * i);
+      }
+      __stcs(reinterpret_cast<uint4*>(codes + o * (K / 8) + k0 / 8), make_uint4(word[0], word[1], word[2], word[3]));
+      if ((lane & 3) == 0) {
+        const int64_t gi = o * (K / 128) + k0 / 128;
+        steps[gi] = g.step;
+        zeros[gi] = g.zero;
       }
     }
-#pragma unroll
-    for (int i = 0; i < kPackCols; ++i) {
-      mx = fmaxf(mx, wp[i]);
-      mn = fminf(mn, wp[i]);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < kPackCols; ++i) wp[i] = 0.0f;
-  }
-#pragma unroll
-  for (int off = 1; off < 4; off <<= 1) {
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-  }
-  if (!active) return;
-  const GroupParams g = group_params(mx, mn);
-  uint32_t word[4];
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    word[w] = 0u;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      word[w] |= static_cast<uint32_t>(code_of(wp[8 * w + i], g, exact != 0)) << (4 * i);
-  }
-  __stcs(reinterpret_cast<uint4*>(codes + o * (K / 8) + k0 / 8), make_uint4(word[0], word[1], word[2], word[3]));
-  if ((lane & 3) == 0) {
-    const int64_t gi = o * (K / 128) + k0 / 128;
-    steps[gi] = g.step;
-    zeros[gi] = g.zero;
   }
 }
 
