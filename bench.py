@@ -303,6 +303,7 @@ def run_ours(args, rank, world, local_rank):
     best = int(res.best_j.item())
     assert 0 <= best < J and torch.isfinite(res.losses).all()
 
+    fold_ms = measure_fold(Wd, res.scales)
     e2e = None if args.no_e2e else measure_e2e(args, Xh, Wh, dev, J)
     e2e_ms = replicas.max_over_ranks(e2e["ms"] if e2e else 0.0, dev)
     if e2e:
@@ -339,6 +340,7 @@ def run_ours(args, rank, world, local_rank):
         "hbm": {"act_stats_gbs": (2.0 * N * K + 4.0 * K) / (np.mean(act_ms) / 1e3) / 1e9,
                 "quantize_pack_gbs": (2.0 * O * K + 4.0 * K + O * K / 2.0 + 8.0 * O * K / 128)
                 / (np.mean(pack_ms) / 1e3) / 1e9,
+                "fold_gbs": (4.0 * O * K + 4.0 * K) / (fold_ms / 1e3) / 1e9,
                 "peak_gbs": peaks.get("hbm_gbs")},
         "gpu_launches": launches_per_step(J) * args.steps,
         "clocks": clocks,
@@ -352,6 +354,27 @@ def run_ours(args, rank, world, local_rank):
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                        "ms_per_step": e2e["ms"]}
     print(json.dumps(line), flush=True)
+
+
+def measure_fold(Wd, scales):
+    """Applying the chosen scales to W (W diag(s), bf16 out): an HBM-bound step after the search."""
+    import torch
+
+    from weight_only_quantization_act_b200 import awq
+
+    out = torch.empty_like(Wd)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=Wd.device)
+    times = []
+    for i in range(6):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        awq.scale_columns(Wd, scales, out=out)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            times.append(e0.elapsed_time(e1))
+    return float(np.mean(times))
 
 
 def launches_per_step(n_grid: int) -> int:

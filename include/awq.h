@@ -193,6 +193,26 @@ AWQ_API awq_status awq_quantize_pack_ex(const void *W, int64_t O, int64_t K, int
                                 int group, unsigned flags, uint32_t *codes, float *steps, float *zeros,
                                 awq_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------------------
+ * Applying the chosen scales (SubgraphFusionFactory step of 缩放因子搜索流程 on the msModelSlim page):
+ * the target linears get forward scaling of their input columns, W' = W diag(s); the producer of their
+ * input gets the inverse: the norm weight gamma' = gamma / s (NormLinearSubgraph), or the output rows
+ * (and bias) of the source linear divided by s (LinearLinearSubgraph linear1, OVSubgraph v_proj for
+ * multi-head attention, UpDownSubgraph up_proj), so that section 一's identity
+ * X W^T = (X diag(s)^-1)(diag(s) W)^T keeps the subgraph's output.
+ *   awq_scale_columns: out[r, c] = bf16(RN32(A[r, c] op s[c]))
+ *   awq_scale_rows:    out[r, c] = bf16(RN32(A[r, c] op s[r]))
+ * op = AWQ_SCALE_MULTIPLY or AWQ_SCALE_DIVIDE (IEEE fp32 division); A, out bf16 row-major with row
+ * strides lda, ldo (multiples of 8); C % 8 == 0; out may equal A (in place). A norm weight or a bias is
+ * a 1 x C matrix. Bit-exact.
+ * ------------------------------------------------------------------------------------------------- */
+#define AWQ_SCALE_MULTIPLY 0
+#define AWQ_SCALE_DIVIDE 1
+AWQ_API awq_status awq_scale_columns(const void *A, int64_t R, int64_t C, int64_t lda, const float *s, int op,
+                                     void *out, int64_t ldo, awq_stream_t stream);
+AWQ_API awq_status awq_scale_rows(const void *A, int64_t R, int64_t C, int64_t lda, const float *s, int op,
+                                  void *out, int64_t ldo, awq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

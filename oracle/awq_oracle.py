@@ -274,3 +274,33 @@ def quantize_pack(w_bits, s, group: int = GROUP):
     """Codes, steps and zeros of W at scales s, codes packed (the artefact of the search)."""
     _, q, step, z = pseudo_quantize(w_bits, s, group)
     return pack_codes(q.astype(np.uint32)), step, z
+
+
+# ---------------------------------------------------------------------------------------------------
+# (6) applying the scales to the subgraph            [P4 缩放因子搜索流程 (SubgraphFusionFactory), 支持的子图类型]
+#     forward scaling of the target linears' input columns, inverse scaling of the producer of that input
+#     (norm weight, or the rows and bias of the source linear); outputs are bfloat16.
+# ---------------------------------------------------------------------------------------------------
+def round_f32_to_bf16(x) -> np.ndarray:
+    """float32 -> bfloat16 bit patterns, round to nearest, ties to even (finite inputs)."""
+    u = np.ascontiguousarray(x, dtype=F32).view(np.uint32).astype(np.uint64)
+    keep = u >> np.uint64(16)
+    rest = u & np.uint64(0xFFFF)
+    up = (rest > 0x8000) | ((rest == 0x8000) & ((keep & np.uint64(1)) == 1))
+    return (keep + up.astype(np.uint64)).astype(np.uint16)
+
+
+def fold_columns(a_bits, s, divide: bool) -> np.ndarray:
+    """out[r, c] = bf16(RN32(a[r, c] * s[c])) or bf16(RN32(a[r, c] / s[c]))."""
+    a = widen_bf16(a_bits)
+    s = np.asarray(s, F32)[None, :]
+    r = (a / s) if divide else (a * s)
+    return round_f32_to_bf16(r.astype(F32))
+
+
+def fold_rows(a_bits, s, divide: bool) -> np.ndarray:
+    """out[r, c] = bf16(RN32(a[r, c] * s[r])) or bf16(RN32(a[r, c] / s[r]))."""
+    a = widen_bf16(a_bits)
+    s = np.asarray(s, F32)[:, None]
+    r = (a / s) if divide else (a * s)
+    return round_f32_to_bf16(r.astype(F32))

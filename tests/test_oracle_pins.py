@@ -401,3 +401,68 @@ def test_shared_input_concatenation_is_one_search():
         lq = orc.loss_of(X, Wq, orc.pseudo_quantize(Wq, T[j])[0])
         lk = orc.loss_of(X, Wk, orc.pseudo_quantize(Wk, T[j])[0])
         assert abs(res["losses"][j] - (128 * lq + 64 * lk) / 192) <= 1e-12 * res["losses"][j]
+
+
+# ------------------------------------------------------------------------------------------ folding
+def test_bf16_rounding_is_nearest_even():
+    rng = np.random.default_rng(91)
+    x = (rng.standard_normal(4000) * 10.0 ** rng.uniform(-6, 6, 4000)).astype(F32)
+    got = inputs.bf16_bits_to_f32(orc.round_f32_to_bf16(x))
+    for v, g in zip(x[:500], got[:500]):
+        lo = np.float32(inputs.bf16_bits_to_f32(np.array([orc.round_f32_to_bf16(np.array([v]))[0]]))[0])
+        assert g == lo
+        # exact check: no bf16 value is strictly closer
+        up = inputs.bf16_bits_to_f32((orc.round_f32_to_bf16(np.array([v])).astype(np.uint32) + 1).astype(np.uint16))[0]
+        dn = inputs.bf16_bits_to_f32((orc.round_f32_to_bf16(np.array([v])).astype(np.int64) - 1).astype(np.uint16))[0]
+        d = abs(Fraction(float(g)) - Fraction(float(v)))
+        assert d <= abs(Fraction(float(up)) - Fraction(float(v))) and d <= abs(Fraction(float(dn)) - Fraction(float(v)))
+    # ties go to the even pattern: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7
+    assert orc.round_f32_to_bf16(np.array([1 + 2.0 ** -8], F32))[0] == 0x3F80
+    assert orc.round_f32_to_bf16(np.array([1 + 3 * 2.0 ** -8], F32))[0] == 0x3F82
+
+
+def test_fold_identity_and_powers_of_two():
+    A = inputs.random_bf16((7, 64), 92, scale=0.5)
+    one = np.ones(64, F32)
+    assert np.array_equal(orc.fold_columns(A, one, False), A)
+    assert np.array_equal(orc.fold_rows(A, np.ones(7, F32), True), A)
+    two = np.full(64, 4.0, F32)
+    assert np.array_equal(inputs.bf16_bits_to_f32(orc.fold_columns(A, two, False)), inputs.bf16_bits_to_f32(A) * 4)
+    assert np.array_equal(inputs.bf16_bits_to_f32(orc.fold_columns(A, two, True)), inputs.bf16_bits_to_f32(A) / 4)
+
+
+def test_folded_norm_linear_keeps_the_output():
+    """gamma / s on the norm and W diag(s) on the linear give the same output (section 一 of the gsyq.cn
+    AWQ page), up to the bf16 rounding of the folded parameters."""
+    rng = np.random.default_rng(93)
+    K, O = 256, 64
+    xn = inputs.random_bf16((32, K), 94)                       # normalised activations before gamma
+    gamma = inputs.f32_to_bf16_bits((1 + 0.1 * rng.standard_normal(K)).astype(F32))
+    W = inputs.random_bf16((O, K), 95, scale=0.02)
+    act = orc.act_mean(inputs.random_bf16((200, K), 96, outliers=3, factor=50))
+    s = orc.scale_candidates(act, orc.ratio(11, 20))
+    g2 = orc.fold_columns(gamma[None, :], s, True)[0]
+    W2 = orc.fold_columns(W, s, False)
+    f = lambda b: inputs.bf16_bits_to_f32(b).astype(np.float64)  # noqa: E731
+    ref = (f(xn) * f(gamma)[None, :]) @ f(W).T
+    alt = (f(xn) * f(g2)[None, :]) @ f(W2).T
+    mag = np.abs(f(xn) * f(gamma)[None, :]) @ np.abs(f(W)).T
+    assert np.all(np.abs(alt - ref) <= 2 * 2.0 ** -8 * mag)
+
+
+def test_folded_linear_linear_keeps_the_output():
+    """Rows (and bias) of linear1 divided by s, columns of linear2 multiplied by s."""
+    K, H, O = 128, 256, 96
+    x = inputs.random_bf16((16, K), 97)
+    W1 = inputs.random_bf16((H, K), 98, scale=0.05)
+    b1 = inputs.random_bf16((1, H), 99, scale=0.1)[0]
+    W2 = inputs.random_bf16((O, H), 100, scale=0.05)
+    act = orc.act_mean(inputs.random_bf16((64, H), 101, outliers=2, factor=30))
+    s = orc.scale_candidates(act, orc.ratio(15, 20))
+    f = lambda b: inputs.bf16_bits_to_f32(b).astype(np.float64)  # noqa: E731
+    h = f(x) @ f(W1).T + f(b1)[None, :]
+    ref = h @ f(W2).T
+    h2 = f(x) @ f(orc.fold_rows(W1, s, True)).T + f(orc.fold_columns(b1[None, :], s, True)[0])[None, :]
+    alt = h2 @ f(orc.fold_columns(W2, s, False)).T
+    mag = np.abs(h) @ np.abs(f(W2)).T
+    assert np.all(np.abs(alt - ref) <= 3 * 2.0 ** -8 * mag + 1e-12)

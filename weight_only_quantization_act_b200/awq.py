@@ -48,6 +48,8 @@ SIGNATURES = {
     "awq_search_get_layout": (_I, [_I64, _I64, _I64, _I, _I, _P]),
     "awq_quantize_pack": (_I, [_P, _I64, _I64, _I64, _P, _I, _P, _P, _P, _P]),
     "awq_quantize_pack_ex": (_I, [_P, _I64, _I64, _I64, _P, _I, _U, _P, _P, _P, _P]),
+    "awq_scale_columns": (_I, [_P, _I64, _I64, _I64, _P, _I, _P, _I64, _P]),
+    "awq_scale_rows": (_I, [_P, _I64, _I64, _I64, _P, _I, _P, _I64, _P]),
 }
 
 
@@ -271,3 +273,63 @@ def quantize_layer(X: torch.Tensor, W, n_grid: int = 20, group: int = 128, strea
     codes, steps, zeros = quantize_pack(W, res.scales, group=group, stream=stream)
     return dict(act_mean=act, losses=res.losses, best_j=res.best_j, scales=res.scales, codes=codes,
                 steps=steps, zeros=zeros)
+
+
+# --------------------------------------------------------------------------------------------- (6)
+SCALE_MULTIPLY = 0
+SCALE_DIVIDE = 1
+
+
+def _as_matrix(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError("expected a CUDA bfloat16 tensor")
+    return t.view(1, -1) if t.dim() == 1 else t
+
+
+def scale_columns(A: torch.Tensor, s: torch.Tensor, divide: bool = False, out: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """out[r, c] = bf16(A[r, c] * s[c]) (or / s[c]); a 1-D tensor is one row. ``out=A`` works in place."""
+    lib = load_library()
+    A2 = _as_matrix(A)
+    if out is None:
+        out = torch.empty_like(A)
+    O2 = _as_matrix(out)
+    R, C = A2.shape
+    _check("awq_scale_columns", lib.awq_scale_columns(_ptr(A2), R, C, A2.stride(0), _ptr(s),
+                                                      SCALE_DIVIDE if divide else SCALE_MULTIPLY, _ptr(O2),
+                                                      O2.stride(0), _stream(stream)))
+    return out
+
+
+def scale_rows(A: torch.Tensor, s: torch.Tensor, divide: bool = False, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """out[r, c] = bf16(A[r, c] * s[r]) (or / s[r]); a 1-D tensor is scaled element-wise."""
+    lib = load_library()
+    one_d = A.dim() == 1
+    A2 = A.view(-1, 1) if one_d else A
+    if one_d:
+        # a vector scaled element-wise by s is a 1 x C column scaling
+        return scale_columns(A, s, divide=divide, out=out, stream=stream)
+    if out is None:
+        out = torch.empty_like(A)
+    R, C = A2.shape
+    _check("awq_scale_rows", lib.awq_scale_rows(_ptr(A2), R, C, A2.stride(0), _ptr(s),
+                                                SCALE_DIVIDE if divide else SCALE_MULTIPLY, _ptr(out),
+                                                out.stride(0), _stream(stream)))
+    return out
+
+
+def fold_norm_linear(norm_weight: torch.Tensor, linears: Sequence[torch.Tensor], s: torch.Tensor, stream=None):
+    """NormLinearSubgraph: gamma / s for the norm, W diag(s) for every linear reading its output (in place)."""
+    scale_columns(norm_weight, s, divide=True, out=norm_weight, stream=stream)
+    for w in linears:
+        scale_columns(w, s, out=w, stream=stream)
+
+
+def fold_linear_linear(w1: torch.Tensor, b1: torch.Tensor | None, w2: torch.Tensor, s: torch.Tensor, stream=None):
+    """LinearLinearSubgraph / OVSubgraph (multi-head) / UpDownSubgraph: rows (and bias) of the source linear
+    divided by s, columns of the target linear multiplied by s (in place)."""
+    scale_rows(w1, s, divide=True, out=w1, stream=stream)
+    if b1 is not None:
+        scale_columns(b1, s, divide=True, out=b1, stream=stream)
+    scale_columns(w2, s, out=w2, stream=stream)

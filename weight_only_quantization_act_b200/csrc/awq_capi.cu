@@ -519,3 +519,38 @@ extern "C" awq_status awq_act_stats_noalloc(const void* X, int64_t N, int64_t K,
   AWQ_TRY(check_launch("act_finalize_kernel"));
   return ok();
 }
+
+namespace {
+awq_status scale_fold(bool columns, const void* A, int64_t R, int64_t C, int64_t lda, const float* s, int op, void* out,
+                      int64_t ldo, awq_stream_t stream) {
+  AWQ_TRY(check_matrix("A", A, R, C, lda));
+  AWQ_TRY(check_matrix("out", out, R, C, ldo));
+  if (C % 8 != 0) return fail(AWQ_ERR_INVALID_ARG, "C (%lld) must be a multiple of 8", static_cast<long long>(C));
+  if (s == nullptr || (columns && !aligned16(s))) return fail(AWQ_ERR_INVALID_ARG, "s is null or not 16-byte aligned");
+  if (op != AWQ_SCALE_MULTIPLY && op != AWQ_SCALE_DIVIDE) return fail(AWQ_ERR_INVALID_ARG, "unknown op %d", op);
+  if (A == out && lda != ldo) return fail(AWQ_ERR_INVALID_ARG, "in-place scaling needs lda == ldo");
+  DeviceInfo* d = nullptr;
+  AWQ_TRY(device_info(&d));
+  const int64_t vecs = R * (C / 8);
+  const int64_t blocks = std::min<int64_t>(static_cast<int64_t>(d->sms) * 16, (vecs + awq::kFoldThreads - 1) / awq::kFoldThreads);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (columns)
+    awq::scale_fold_kernel<true><<<static_cast<unsigned>(blocks), awq::kFoldThreads, 0, st>>>(
+        static_cast<const uint16_t*>(A), R, C, lda, s, op == AWQ_SCALE_DIVIDE, static_cast<uint16_t*>(out), ldo);
+  else
+    awq::scale_fold_kernel<false><<<static_cast<unsigned>(blocks), awq::kFoldThreads, 0, st>>>(
+        static_cast<const uint16_t*>(A), R, C, lda, s, op == AWQ_SCALE_DIVIDE, static_cast<uint16_t*>(out), ldo);
+  AWQ_TRY(check_launch("scale_fold_kernel"));
+  return ok();
+}
+}  // namespace
+
+extern "C" awq_status awq_scale_columns(const void* A, int64_t R, int64_t C, int64_t lda, const float* s, int op,
+                                        void* out, int64_t ldo, awq_stream_t stream) {
+  return scale_fold(true, A, R, C, lda, s, op, out, ldo, stream);
+}
+
+extern "C" awq_status awq_scale_rows(const void* A, int64_t R, int64_t C, int64_t lda, const float* s, int op,
+                                     void* out, int64_t ldo, awq_stream_t stream) {
+  return scale_fold(false, A, R, C, lda, s, op, out, ldo, stream);
+}

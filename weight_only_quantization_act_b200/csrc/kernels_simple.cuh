@@ -449,4 +449,45 @@ __global__ void __launch_bounds__(kPackThreads) quantize_pack_kernel(
   }
 }
 
+// ===================================================================================================
+// Scale folding: out = bf16(RN32(A op s)) with s per column or per row. 8 elements per thread.
+// ===================================================================================================
+constexpr int kFoldThreads = 256;
+
+template <bool kColumns>
+__global__ void __launch_bounds__(kFoldThreads) scale_fold_kernel(const uint16_t* __restrict__ A, int64_t R,
+                                                                  int64_t C, int64_t lda,
+                                                                  const float* __restrict__ s, int divide,
+                                                                  uint16_t* __restrict__ out, int64_t ldo) {
+  const int64_t vec_per_row = C / 8;
+  const int64_t total = R * vec_per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kFoldThreads + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * kFoldThreads) {
+    const int64_t r = i / vec_per_row;
+    const int64_t c0 = (i - r * vec_per_row) * 8;
+    const uint4 u = *reinterpret_cast<const uint4*>(A + r * lda + c0);
+    float sv[8];
+    if (kColumns) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(s + c0));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(s + c0) + 1);
+      sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w; sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
+    } else {
+      const float x = __ldg(s + r);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sv[k] = x;
+    }
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float lo = bf16_lo(w[k]), hi = bf16_hi(w[k]);
+      const float rl = divide ? __fdiv_rn(lo, sv[2 * k]) : __fmul_rn(lo, sv[2 * k]);
+      const float rh = divide ? __fdiv_rn(hi, sv[2 * k + 1]) : __fmul_rn(hi, sv[2 * k + 1]);
+      const __nv_bfloat162 pr = __floats2bfloat162_rn(rl, rh);
+      o[k] = *reinterpret_cast<const uint32_t*>(&pr);
+    }
+    *reinterpret_cast<uint4*>(out + r * ldo + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 }  // namespace awq
