@@ -304,6 +304,7 @@ def run_ours(args, rank, world, local_rank):
     assert 0 <= best < J and torch.isfinite(res.losses).all()
 
     fold_ms = measure_fold(Wd, res.scales)
+    w4 = measure_w4a16(Xd, Wd, res.scales)
     e2e = None if args.no_e2e else measure_e2e(args, Xh, Wh, dev, J)
     e2e_ms = replicas.max_over_ranks(e2e["ms"] if e2e else 0.0, dev)
     if e2e:
@@ -342,6 +343,11 @@ def run_ours(args, rank, world, local_rank):
                 / (np.mean(pack_ms) / 1e3) / 1e9,
                 "fold_gbs": (4.0 * O * K + 4.0 * K) / (fold_ms / 1e3) / 1e9,
                 "peak_gbs": peaks.get("hbm_gbs")},
+        "w4a16": {"prefill_tokens": N, "prefill_ms": w4["prefill_ms"],
+                  "prefill_tflops": 2.0 * N * O * K / (w4["prefill_ms"] / 1e3) / 1e12,
+                  "prefill_frac_of_peak": 2.0 * N * O * K / (w4["prefill_ms"] / 1e3) / 1e12 / peaks["bf16_tflops"],
+                  "decode_tokens": 16, "decode_ms": w4["decode_ms"],
+                  "decode_weight_gbs": (0.5 * O * K + 8.0 * O * K / 128) / (w4["decode_ms"] / 1e3) / 1e9},
         "gpu_launches": launches_per_step(J) * args.steps,
         "clocks": clocks,
         "best_j": best,
@@ -375,6 +381,35 @@ def measure_fold(Wd, scales):
         if i >= 2:
             times.append(e0.elapsed_time(e1))
     return float(np.mean(times))
+
+
+def measure_w4a16(Xd, Wd, scales):
+    """The deployment GEMM on the quantized layer: a prefill of all N calibration tokens and a 16-token
+    decode step, each timed alone (L2 flushed before every launch)."""
+    import torch
+
+    from weight_only_quantization_act_b200 import awq
+
+    codes, steps, zeros = awq.quantize_pack(Wd, scales)
+    Xs = awq.scale_columns(Xd, scales, divide=True)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=Xd.device)
+    ws = torch.empty(awq.load_library().awq_w4a16_workspace_size(Xd.shape[1], codes.shape[0]), dtype=torch.uint8,
+                     device=Xd.device)
+    out = {}
+    for name, X in (("prefill_ms", Xs), ("decode_ms", Xs[:16].contiguous())):
+        Y = torch.empty((X.shape[0], codes.shape[0]), dtype=torch.bfloat16, device=Xd.device)
+        times = []
+        for i in range(6):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            awq.w4a16_gemm(X, codes, steps, zeros, out=Y, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                times.append(e0.elapsed_time(e1))
+        out[name] = float(np.mean(times))
+    return out
 
 
 def launches_per_step(n_grid: int) -> int:

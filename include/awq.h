@@ -213,6 +213,25 @@ AWQ_API awq_status awq_scale_columns(const void *A, int64_t R, int64_t C, int64_
 AWQ_API awq_status awq_scale_rows(const void *A, int64_t R, int64_t C, int64_t lda, const float *s, int op,
                                   void *out, int64_t ldo, awq_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------------------
+ * Deployment GEMM of a quantized linear (W4A16): Y = X' deq(W)^T, the weights read as the packed codes,
+ * steps and zeros of awq_quantize_pack and dequantized on the fly ("GPU 硬件级反量化算子内联融合" on the
+ * bjdmk.com.cn AWQ article): deq(W)[o, k] = bf16(RN32(RN32(q[o,k] - z[o,g]) * step[o,g])), g = k / 128.
+ * X' is the layer input with the AWQ scales already folded out (X diag(s)^-1, e.g. by awq_scale_columns
+ * on the previous norm weight). bf16 x bf16 products, fp32 accumulation on the tensor cores, bf16 output.
+ *   X       device bf16 [M, K], row stride ldx (multiple of 8)
+ *   codes   device uint32 [O, K/8], steps / zeros device float [O, K/128] (contiguous, as packed)
+ *   Y       device bf16 [M, O], row stride ldy (multiple of 8)
+ *   workspace  device, >= awq_w4a16_workspace_size(K, O) bytes (status word, tile counter and a
+ *              group-major copy of steps and zeros, rewritten every call)
+ * Requires K % 128 == 0, O % 8 == 0, M >= 1. A device timeout is reported by awq_search_status() on the
+ * same workspace.
+ * ------------------------------------------------------------------------------------------------- */
+AWQ_API size_t awq_w4a16_workspace_size(int64_t K, int64_t O);
+AWQ_API awq_status awq_w4a16_gemm(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *codes,
+                                  const float *steps, const float *zeros, int64_t O, void *Y, int64_t ldy,
+                                  void *workspace, size_t ws_bytes, awq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

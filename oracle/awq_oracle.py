@@ -304,3 +304,23 @@ def fold_rows(a_bits, s, divide: bool) -> np.ndarray:
     s = np.asarray(s, F32)[:, None]
     r = (a / s) if divide else (a * s)
     return round_f32_to_bf16(r.astype(F32))
+
+
+# ---------------------------------------------------------------------------------------------------
+# (7) deployment GEMM of the quantized linear (W4A16)   [P2 GPU 硬件级反量化算子内联融合]
+#     the weights are restored from the packed codes with the group step and zero, to a 16-bit float
+#     (bfloat16 here), and multiplied with the activations; here exactly, in fp64.
+# ---------------------------------------------------------------------------------------------------
+def dequant_w4(words, steps, zeros, group: int = GROUP) -> np.ndarray:
+    """float32 [O, K]: RN32(RN32(q - z) * step) per element, q unpacked from the words."""
+    q = unpack_codes(words, np.asarray(words).shape[1] * 8).astype(F32)
+    st = np.repeat(np.asarray(steps, F32), group, axis=1)
+    z = np.repeat(np.asarray(zeros, F32), group, axis=1)
+    return ((q - z) * st).astype(F32)
+
+
+def w4a16_matmul(x_bits, words, steps, zeros, group: int = GROUP) -> np.ndarray:
+    """fp64 [M, O] = X' @ bf16(deq(W))^T, with the bf16 weight operand the GPU feeds its tensor cores."""
+    deq16 = widen_bf16(round_f32_to_bf16(dequant_w4(words, steps, zeros, group))).astype(F64)
+    x = widen_bf16(x_bits).astype(F64)
+    return x @ deq16.T

@@ -1,0 +1,62 @@
+"""The W4A16 deployment GEMM (a 'next' row) against the oracle, and the whole deploy path end to end."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import awq_oracle as orc
+from tests._helpers import bf16_to_device
+from weight_only_quantization_act_b200 import awq, inputs
+
+pytestmark = pytest.mark.gpu
+F32 = np.float32
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    awq.load_library()
+
+
+def check_against_oracle(Xp, words, steps, zeros, Y):
+    """|Y - ref| <= 2^-8 |ref| + (K/16 + 16) 2^-23 sum_k |x w|: bf16 output rounding plus fp32 accumulation."""
+    K = Xp.shape[1]
+    ref = orc.w4a16_matmul(Xp, words, steps, zeros)
+    deq16 = inputs.bf16_bits_to_f32(orc.round_f32_to_bf16(orc.dequant_w4(words, steps, zeros))).astype(np.float64)
+    mag = np.abs(inputs.bf16_bits_to_f32(Xp).astype(np.float64)) @ np.abs(deq16).T
+    got = Y.float().cpu().numpy().astype(np.float64)
+    tol = 2.0 ** -8 * np.abs(ref) + (K / 16 + 16) * 2.0 ** -23 * mag
+    bad = np.abs(got - ref) > tol
+    assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], ref[bad][:5])
+
+
+def quantized(O, K, seed):
+    W = inputs.random_bf16((O, K), seed, scale=0.02)
+    s = orc.scale_candidates(orc.act_mean(inputs.random_bf16((64, K), seed + 1, outliers=3, factor=40)),
+                             orc.ratio(8, 20))
+    return W, s, orc.quantize_pack(W, s)
+
+
+@pytest.mark.parametrize("M,K,O", [(300, 384, 600), (1, 128, 8), (256, 256, 256), (513, 4096, 1032)])
+def test_w4a16_matches_oracle(M, K, O):
+    _, _, (words, steps, zeros) = quantized(O, K, M + K + O)
+    Xp = inputs.random_bf16((M, K), 7 * M + 1, scale=1.0)
+    Y = awq.w4a16_gemm(bf16_to_device(Xp), torch.from_numpy(words.view(np.int32)).cuda(),
+                       torch.from_numpy(steps).cuda(), torch.from_numpy(zeros).cuda())
+    torch.cuda.synchronize()
+    check_against_oracle(Xp, words, steps, zeros, Y)
+
+
+def test_deploy_path_end_to_end():
+    """search -> pack -> fold the scales out of X -> W4A16 GEMM reproduces X W^T up to the quantization
+    error the search measured (mean squared output error within 25% of the search's best loss)."""
+    X = inputs.random_bf16((1024, 1024), 31, outliers=10, factor=40)
+    W = inputs.random_bf16((512, 1024), 32, scale=0.02)
+    Xd, Wd = bf16_to_device(X), bf16_to_device(W)
+    out = awq.quantize_layer(Xd, Wd)
+    Xs = awq.scale_columns(Xd, out["scales"], divide=True)
+    Y = awq.w4a16_gemm(Xs, out["codes"], out["steps"], out["zeros"]).double()
+    ref = Xd.double() @ Wd.double().T
+    mse = float(((Y - ref) ** 2).mean())
+    best = float(out["losses"][int(out["best_j"].item())])
+    assert 0.5 * best < mse < 1.25 * best, (mse, best)

@@ -466,3 +466,28 @@ def test_folded_linear_linear_keeps_the_output():
     alt = h2 @ f(orc.fold_columns(W2, s, False)).T
     mag = np.abs(h) @ np.abs(f(W2)).T
     assert np.all(np.abs(alt - ref) <= 3 * 2.0 ** -8 * mag + 1e-12)
+
+
+# ------------------------------------------------------------------------------------------ W4A16
+def test_dequant_from_packed_codes_equals_the_quantizers_dequant():
+    W = inputs.random_bf16((48, 384), 111, scale=0.03)
+    s = orc.scale_candidates(orc.act_mean(inputs.random_bf16((64, 384), 112, outliers=2, factor=40)),
+                             orc.ratio(9, 20))
+    wp = (inputs.bf16_bits_to_f32(W) * s[None, :]).astype(F32)
+    _, _, _, deq = orc.quantize_groups(wp)
+    words, steps, zeros = orc.quantize_pack(W, s)
+    assert np.array_equal(orc.dequant_w4(words, steps, zeros), deq)
+
+
+def test_w4a16_hand_examples():
+    O, K = 8, 128
+    q = np.full((O, K), 8, np.uint8)
+    words = orc.pack_codes(q)
+    zeros = np.full((O, 1), 8.0, F32)
+    steps = np.full((O, 1), 0.25, F32)
+    x = inputs.random_bf16((3, K), 113)
+    assert np.all(orc.w4a16_matmul(x, words, steps, zeros) == 0.0)
+    rng = np.random.default_rng(114)
+    q = rng.integers(0, 16, (O, K)).astype(np.uint8)
+    y = orc.w4a16_matmul(x, orc.pack_codes(q), np.ones((O, 1), F32), np.zeros((O, 1), F32))
+    assert np.array_equal(y, inputs.bf16_bits_to_f32(x).astype(np.float64) @ q.T.astype(np.float64))

@@ -50,6 +50,8 @@ SIGNATURES = {
     "awq_quantize_pack_ex": (_I, [_P, _I64, _I64, _I64, _P, _I, _U, _P, _P, _P, _P]),
     "awq_scale_columns": (_I, [_P, _I64, _I64, _I64, _P, _I, _P, _I64, _P]),
     "awq_scale_rows": (_I, [_P, _I64, _I64, _I64, _P, _I, _P, _I64, _P]),
+    "awq_w4a16_workspace_size": (_SZ, [_I64, _I64]),
+    "awq_w4a16_gemm": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I64, _P, _I64, _P, _SZ, _P]),
 }
 
 
@@ -333,3 +335,21 @@ def fold_linear_linear(w1: torch.Tensor, b1: torch.Tensor | None, w2: torch.Tens
     if b1 is not None:
         scale_columns(b1, s, divide=True, out=b1, stream=stream)
     scale_columns(w2, s, out=w2, stream=stream)
+
+
+# --------------------------------------------------------------------------------------------- (7)
+def w4a16_gemm(X: torch.Tensor, codes: torch.Tensor, steps: torch.Tensor, zeros: torch.Tensor,
+               out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = X' deq(W)^T (bf16 [M, O]) from packed codes [O, K/8], steps and zeros [O, K/128]."""
+    lib = load_library()
+    X = _bf16_matrix("X", X)
+    M, K = X.shape
+    O = codes.shape[0]
+    if out is None:
+        out = torch.empty((M, O), dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(lib.awq_w4a16_workspace_size(K, O), dtype=torch.uint8, device=X.device)
+    _check("awq_w4a16_gemm", lib.awq_w4a16_gemm(_ptr(X), M, K, X.stride(0), _ptr(codes), _ptr(steps), _ptr(zeros),
+                                                O, _ptr(out), out.stride(0), _ptr(workspace), workspace.numel(),
+                                                _stream(stream)))
+    return out

@@ -13,6 +13,7 @@
 
 #include "awq.h"
 #include "kernel_loss_gemm.cuh"
+#include "kernel_w4a16.cuh"
 #include "kernels_simple.cuh"
 
 namespace {
@@ -46,6 +47,7 @@ struct DeviceInfo {
   int cc_major = 0;
   bool gemm_attr_set = false;
   int gemm_clusters = 0;  // CTA pairs of the loss GEMM that fit on the device at once
+  int w4_clusters = 0;    // CTA pairs of the W4A16 GEMM that fit on the device at once
 };
 
 constexpr int kMaxDevices = 64;
@@ -82,6 +84,12 @@ awq_status device_info(DeviceInfo** out) {
     cfg.numAttrs = 1;
     AWQ_CUDA(cudaOccupancyMaxActiveClusters(&d.gemm_clusters, awq::lg::loss_gemm_kernel, &cfg));
     if (d.gemm_clusters < 1) return fail(AWQ_ERR_UNSUPPORTED, "the loss GEMM does not fit on this device");
+    AWQ_CUDA(cudaFuncSetAttribute(awq::dq::w4a16_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::dq::SMEM_BYTES));
+    cfg.blockDim = dim3(awq::dq::THREADS);
+    cfg.dynamicSmemBytes = awq::dq::SMEM_BYTES;
+    AWQ_CUDA(cudaOccupancyMaxActiveClusters(&d.w4_clusters, awq::dq::w4a16_gemm_kernel, &cfg));
+    if (d.w4_clusters < 1) return fail(AWQ_ERR_UNSUPPORTED, "the W4A16 GEMM does not fit on this device");
     d.gemm_attr_set = true;
   }
   *out = &d;
@@ -113,6 +121,21 @@ awq_status make_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t c
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return AWQ_OK;
+}
+
+// Generic row-major 2-D map without swizzle: [rows][cols] of elements of `esize` bytes.
+awq_status make_tmap_plain(CUtensorMap* map, const void* base, CUtensorMapDataType type, int esize, int64_t rows,
+                           int64_t cols, int64_t ld, int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * static_cast<cuuint64_t>(esize)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
   return AWQ_OK;
 }
@@ -553,4 +576,85 @@ extern "C" awq_status awq_scale_columns(const void* A, int64_t R, int64_t C, int
 extern "C" awq_status awq_scale_rows(const void* A, int64_t R, int64_t C, int64_t lda, const float* s, int op,
                                      void* out, int64_t ldo, awq_stream_t stream) {
   return scale_fold(false, A, R, C, lda, s, op, out, ldo, stream);
+}
+
+namespace {
+struct W4Layout {
+  int64_t O_pad, G;
+  size_t steps_off, zeros_off, bytes;
+};
+W4Layout w4_layout(int64_t K, int64_t O) {
+  W4Layout l;
+  l.O_pad = (O + awq::lg::BN - 1) / awq::lg::BN * awq::lg::BN;
+  l.G = K / 128;
+  l.steps_off = 512;
+  l.zeros_off = align_up(l.steps_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
+  l.bytes = align_up(l.zeros_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
+  return l;
+}
+}  // namespace
+
+extern "C" size_t awq_w4a16_workspace_size(int64_t K, int64_t O) {
+  if (K < 128 || O < 1) return 0;
+  return w4_layout(K, O).bytes;
+}
+
+extern "C" awq_status awq_w4a16_gemm(const void* X, int64_t M, int64_t K, int64_t ldx, const uint32_t* codes,
+                                     const float* steps, const float* zeros, int64_t O, void* Y, int64_t ldy,
+                                     void* workspace, size_t ws_bytes, awq_stream_t stream) {
+  AWQ_TRY(check_matrix("X", X, M, K, ldx));
+  AWQ_TRY(check_matrix("Y", Y, M, O, ldy));
+  if (K % 128 != 0) return fail(AWQ_ERR_INVALID_ARG, "K (%lld) must be a multiple of 128", static_cast<long long>(K));
+  if (O % 8 != 0) return fail(AWQ_ERR_INVALID_ARG, "O (%lld) must be a multiple of 8", static_cast<long long>(O));
+  if (codes == nullptr || steps == nullptr || zeros == nullptr || !aligned16(codes))
+    return fail(AWQ_ERR_INVALID_ARG, "codes (16-byte aligned), steps and zeros must be given");
+  const W4Layout l = w4_layout(K, O);
+  if (workspace == nullptr || ws_bytes < l.bytes)
+    return fail(AWQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", l.bytes, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(AWQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  const int64_t n_tiles_m = (M + awq::lg::BM - 1) / awq::lg::BM;
+  const int64_t n_bands = l.O_pad / awq::lg::BN;
+  if (n_tiles_m * n_bands >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "too many tiles");
+  DeviceInfo* d = nullptr;
+  AWQ_TRY(device_info(&d));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  float* steps_t = reinterpret_cast<float*>(ws + l.steps_off);
+  float* zeros_t = reinterpret_cast<float*>(ws + l.zeros_off);
+  CUtensorMap tmX, tmC, tmS, tmZ;
+  AWQ_TRY(make_tmap(&tmX, X, M, K, ldx, awq::lg::HALF));
+  AWQ_TRY(make_tmap_plain(&tmC, codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, O, K / 8, K / 8, awq::lg::BK / 8,
+                          awq::lg::HALF));
+  AWQ_TRY(make_tmap_plain(&tmS, steps_t, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, l.G, l.O_pad, l.O_pad, awq::lg::HALF, 1));
+  AWQ_TRY(make_tmap_plain(&tmZ, zeros_t, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, l.G, l.O_pad, l.O_pad, awq::lg::HALF, 1));
+  AWQ_CUDA(cudaMemsetAsync(ws, 0, 512, st));
+  awq::dq::transpose_groups_kernel<<<dim3(static_cast<unsigned>(l.O_pad / 256), static_cast<unsigned>(l.G)), 256, 0,
+                                     st>>>(steps, zeros, O, l.O_pad, l.G, steps_t, zeros_t);
+  AWQ_TRY(check_launch("transpose_groups_kernel"));
+  awq::dq::Params p;
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.M = M;
+  p.O = O;
+  p.K = K;
+  p.ldy = ldy;
+  p.n_tiles_m = static_cast<int>(n_tiles_m);
+  p.n_bands = static_cast<int>(n_bands);
+  p.num_kb = static_cast<int>(K / awq::lg::BK);
+  p.num_tiles = static_cast<int>(n_tiles_m * n_bands);
+  p.tile_counter = reinterpret_cast<unsigned int*>(ws + 20);
+  p.status = reinterpret_cast<awq::DeviceStatus*>(ws);
+  p.limit_ns = g_wait_limit_ns.load();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * d->w4_clusters));
+  cfg.blockDim = dim3(awq::dq::THREADS);
+  cfg.dynamicSmemBytes = awq::dq::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  AWQ_CUDA(cudaLaunchKernelEx(&cfg, awq::dq::w4a16_gemm_kernel, tmX, tmC, tmS, tmZ, p));
+  AWQ_TRY(check_launch("w4a16_gemm_kernel"));
+  return ok();
 }

@@ -1,0 +1,398 @@
+// kernel_w4a16.cuh - the deployment GEMM of an AWQ-quantized linear: Y = X' deq(W)^T with the weights
+// read as packed 4-bit codes and dequantized on the fly ("GPU 硬件级反量化算子内联融合" on the bjdmk.com.cn
+// AWQ article: 4-bit weights loaded compactly, unpacked with shifts and masks, converted, multiplied by
+// the group scale and offset, then fed to the tensor cores). X' is the layer input already divided by
+// the AWQ scales (folded into the previous operation); deq(W)[o, k] = bf16(RN32(RN32(q - z) * step)).
+//
+// Persistent cooperative kernel, clusters of 2 CTAs, one CTA per SM, 18 warps per CTA; tiles of 256
+// tokens x 256 output rows handed out dynamically through an 8-slot ring (as in the loss kernel):
+//   warp 0      TMA: X' tile [128 x 64] per stage for this CTA (128-byte swizzle; both CTAs' bytes are
+//               counted on the even CTA's barrier), and the stage's code words [128 rows x 8 words]
+//               plus the group steps and zeros of those rows (from a group-major copy) into this CTA's
+//               shared memory, counted on a barrier of this CTA
+//   warp 1      pair-wide tensor memory (two 256-column fp32 accumulators); the even CTA issues the pair
+//               MMAs (tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16)
+//   warps 2-5   epilogue: fp32 accumulator -> bf16, stored to Y (each lane one row, 64-byte pieces)
+//   warps 6-17  dequantizers, two per pipeline stage: warps 6+s and 12+s fill every use of stage s with
+//               the CTA's 128 weight rows x 64 in-features from the staged codes, in the 128-byte swizzled
+//               K-major layout the MMA descriptor expects (64 rows each), then one proxy fence and one
+//               arrive on the even CTA's full barrier. Owning whole stages lets the six stages fill
+//               concurrently and pays the fence once per 8 KB; the warps issue no global loads (the
+//               fence would wait for them too).
+// Every wait is bounded.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "kernel_loss_gemm.cuh"
+#include "ptx.cuh"
+
+namespace awq {
+namespace dq {
+
+using lg::BK;
+using lg::BM;
+using lg::BN;
+using lg::HALF;
+using lg::NUM_ACC;
+using lg::RING;
+using lg::TMEM_COLS;
+using lg::UK;
+
+constexpr int STAGES = 6;
+constexpr int A_BYTES = HALF * BK * 2;            // 16 KB  X' rows
+constexpr int B_BYTES = HALF * BK * 2;            // 16 KB  dequantized weight rows
+constexpr int C_BYTES = HALF * (BK / 8) * 4;      // 4 KB   code words of those rows
+constexpr int S_BYTES = HALF * 4;                 // 512 B  step of each row (this k-block's group)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES + 2 * S_BYTES;  // 37 KB per CTA
+constexpr int DQ_PER_STAGE = 2;                   // dequantizer warps per stage (each half the rows)
+constexpr int DQ_WARPS = STAGES * DQ_PER_STAGE;
+constexpr int THREADS = 192 + 32 * DQ_WARPS;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+constexpr int BANDS_PER_GROUP = 8;                // raster: 8 weight bands advance together over X'
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+struct Params {
+  __nv_bfloat16* Y;        // [M][ldy]
+  int64_t M, O, K, ldy;
+  int n_tiles_m;           // ceil(M / 256)
+  int n_bands;             // ceil(O / 256)
+  int num_kb;              // K / 64
+  int num_tiles;
+  unsigned int* tile_counter;  // zeroed before launch
+  DeviceStatus* status;
+  uint64_t limit_ns;
+};
+
+__device__ __forceinline__ void tile_coords(int t, const Params& p, int& band, int& mt) {
+  const int per_group = BANDS_PER_GROUP * p.n_tiles_m;
+  const int g = t / per_group;
+  const int local = t - g * per_group;
+  const int bands_in_g = min(BANDS_PER_GROUP, p.n_bands - g * BANDS_PER_GROUP);
+  band = g * BANDS_PER_GROUP + local % bands_in_g;
+  mt = local / bands_in_g;
+}
+
+// Warp-uniform bounded wait (all lanes poll), with cluster-scope acquire when `cluster` is set.
+__device__ __forceinline__ bool warp_wait_any(uint32_t bar, uint32_t parity, DeviceStatus* st, uint64_t limit,
+                                              unsigned where, bool cluster) {
+  uint64_t t0 = 0;
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) t0 = global_timer_ns();
+#pragma unroll 1
+  for (uint32_t it = 0;; ++it) {
+    const bool done = cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    int give_up = 0;
+    if (lane == 0 && (it & 63u) == 63u) {
+      if (status_code(st) != 0u) give_up = 1;
+      else if (global_timer_ns() - t0 > limit) {
+        raise_timeout(st, where);
+        give_up = 1;
+      }
+    }
+    if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+  }
+}
+
+// Group-major copy of the per-group steps and zeros: [O][G] -> [G][O_pad] (rows past O are zeros), so that
+// one TMA box brings the steps of 128 consecutive weight rows for one group.
+__global__ void __launch_bounds__(256) transpose_groups_kernel(const float* __restrict__ steps,
+                                                               const float* __restrict__ zeros, int64_t O,
+                                                               int64_t O_pad, int64_t G, float* __restrict__ steps_t,
+                                                               float* __restrict__ zeros_t) {
+  const int64_t o = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  const int64_t g = blockIdx.y;
+  if (o >= O_pad) return;
+  const bool real = o < O;
+  steps_t[g * O_pad + o] = real ? steps[o * G + g] : 0.0f;
+  zeros_t[g * O_pad + o] = real ? zeros[o * G + g] : 0.0f;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
+                      const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bars[3 * STAGES + 2 * NUM_ACC + 1 + RING];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int tile_ring[RING];
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const uint32_t bar0 = smem_u32(&bars[0]);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + NUM_ACC + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * NUM_ACC);
+  auto tile_bar = [&](int slot) { return drain_bar + 8u + 8u * slot; };
+  auto cfull_bar = [&](int s) { return drain_bar + 8u + 8u * RING + 8u * s; };
+  const uint32_t smem_base = smem_u32(smem);
+  auto a_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s) * STAGE_BYTES; };
+  auto b_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s) * STAGE_BYTES + A_BYTES; };
+  auto c_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s) * STAGE_BYTES + A_BYTES + B_BYTES; };
+  auto s_tile = [&](int s) { return c_tile(s) + C_BYTES; };
+  auto z_tile = [&](int s) { return c_tile(s) + C_BYTES + S_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1 + 2 * DQ_PER_STAGE);  // TMA arm + the stage's dequantizer warps of both CTAs
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < NUM_ACC; ++a) {
+      mbar_init(accf_bar(a), 1);
+      mbar_init(acce_bar(a), 8);
+    }
+    mbar_init(drain_bar, 1);
+    for (int r = 0; r < RING; ++r) mbar_init(tile_bar(r), 1);
+    for (int st2 = 0; st2 < STAGES; ++st2) mbar_init(cfull_bar(st2), 1);  // this CTA's TMA thread arms it
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) tmem_alloc_pair(smem_u32(&tmem_slot), TMEM_COLS);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmC);
+    tma_prefetch_desc(&tmS);
+    tma_prefetch_desc(&tmZ);
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  DeviceStatus* st = p.status;
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int n_pairs = static_cast<int>(gridDim.x >> 1);
+
+  auto ring_wait_thread = [&](int i, bool& ok) -> int {
+    const int slot = i % RING;
+    const uint32_t par = static_cast<uint32_t>(i / RING) & 1u;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait_cluster(tile_bar(slot), par)) {
+      if (status_code(st) != 0u || global_timer_ns() - t0 > p.limit_ns) {
+        if (status_code(st) == 0u) raise_timeout(st, kSiteTileRing);
+        ok = false;
+        return -1;
+      }
+    }
+    return *reinterpret_cast<volatile int*>(&tile_ring[slot]);
+  };
+  auto ring_wait_warp = [&](int i, bool& ok) -> int {
+    const int slot = i % RING;
+    const uint32_t par = static_cast<uint32_t>(i / RING) & 1u;
+    if (!warp_wait_any(tile_bar(slot), par, st, p.limit_ns, kSiteTileRing, true)) {
+      ok = false;
+      return -1;
+    }
+    return *reinterpret_cast<volatile int*>(&tile_ring[slot]);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------------------ TMA (X')
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      const uint64_t pol_x = policy_evict_normal();
+      for (int i = 0; ok; ++i) {
+        int t;
+        if (rank == 0) {
+          t = i == 0 ? pair : n_pairs + static_cast<int>(atomicAdd(p.tile_counter, 1u));
+          if (t >= p.num_tiles) t = -1;
+          const int slot = i % RING;
+          tile_ring[slot] = t;
+          st_shared_cluster_u32(map_to_rank(smem_u32(&tile_ring[slot]), 1), static_cast<uint32_t>(t));
+          mbar_arrive(tile_bar(slot));
+          mbar_arrive_remote(map_to_rank(tile_bar(slot), 1));
+        } else {
+          t = ring_wait_thread(i, ok);
+          if (!ok) break;
+        }
+        if (t < 0) break;
+        int band, mt;
+        tile_coords(t, p, band, mt);
+        const int32_t a_row = mt * BM + static_cast<int32_t>(rank) * HALF;
+        const int32_t w_row = band * BN + static_cast<int32_t>(rank) * HALF;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, st, p.limit_ns, kSiteTmaEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = map_to_rank(full_bar(stage), 0);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * A_BYTES);
+          tma_load_2d_pair_hint(a_tile(stage), &tmX, kb * BK, a_row, fb, pol_x);
+          mbar_arrive_expect_tx(cfull_bar(stage), C_BYTES + 2 * S_BYTES);
+          tma_load_2d(c_tile(stage), &tmC, kb * (BK / 8), w_row, cfull_bar(stage));
+          tma_load_2d(s_tile(stage), &tmS, w_row, (kb * BK) >> 7, cfull_bar(stage));
+          tma_load_2d(z_tile(stage), &tmZ, w_row, (kb * BK) >> 7, cfull_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------------------ MMA (even CTA)
+    if (rank == 0 && elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; ok; ++i) {
+        const int t = ring_wait_thread(i, ok);
+        if (!ok || t < 0) break;
+        const int acc = i & 1;
+        const uint32_t acc_phase = static_cast<uint32_t>(i >> 1) & 1u;
+        if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, st, p.limit_ns, kSiteMmaAccEmpty)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, st, p.limit_ns, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = a_tile(stage), b0 = b_tile(stage);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk)
+            umma_bf16_pair(d_tmem, smem_desc_sw128(a0 + kk * UK * 2), smem_desc_sw128(b0 + kk * UK * 2), IDESC,
+                           (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair(empty_bar(stage), 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(accf_bar(acc), 0x3);
+      }
+      umma_commit_pair(drain_bar, 0x1);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain_bar, 0u))
+        if (global_timer_ns() - t0 > p.limit_ns) {
+          raise_timeout(st, kSiteDrainMma);
+          break;
+        }
+    }
+    __syncwarp();
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------------------------ dequantizers
+    // Warp 6+s owns stage s: the pipeline's k-blocks are numbered continuously over this pair's tiles
+    // (tile i, k-block kb -> i * num_kb + kb), and stage s carries the numbers congruent to s mod STAGES.
+    const int s_own = (warp - 6) % STAGES;
+    const int part = (warp - 6) / STAGES;  // which HALF / DQ_PER_STAGE rows of the stage this warp fills
+    bool ok = true;
+    int known_tile = -1;  // tiles < known_tile + 1 exist (the ring told us)
+    for (int64_t g = s_own, use = 0; ok; g += STAGES, ++use) {
+      const int i = static_cast<int>(g / p.num_kb);
+      if (i > known_tile) {
+        const int t = ring_wait_warp(i, ok);
+        if (!ok || t < 0) break;
+        known_tile = i;
+      }
+      if (!warp_wait_any(cfull_bar(s_own), static_cast<uint32_t>(use) & 1u, st, p.limit_ns, kSiteTmaEmpty, false)) {
+        ok = false;
+        break;
+      }
+      const uint32_t cbase = c_tile(s_own), bbase = b_tile(s_own);
+#pragma unroll 1
+      for (int rr = 0; rr < HALF / 32 / DQ_PER_STAGE; ++rr) {
+        const int r = lane + 32 * (rr + part * (HALF / 32 / DQ_PER_STAGE));
+        uint32_t w[8];
+        float z, stp;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "r"(cbase + static_cast<uint32_t>(r * 32)));
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                     : "r"(cbase + static_cast<uint32_t>(r * 32 + 16)));
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(stp) : "r"(s_tile(s_own) + static_cast<uint32_t>(r * 4)));
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(z) : "r"(z_tile(s_own) + static_cast<uint32_t>(r * 4)));
+        // (2^23 + q) - (2^23 + z) = q - z exactly; then one fp32 rounding for the step, one for bf16.
+        // Rows past O arrive as zero codes with zero step and zero: they dequantize to 0.
+        const float zb = __fadd_rn(8388608.0f, z);
+        const uint32_t row_base = bbase + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {  // code word c = in-features 8c..8c+7 = 16-byte chunk c of the row
+          uint32_t o4[4];
+#pragma unroll
+          for (int n = 0; n < 8; n += 2) {
+            const float q0 = __uint_as_float(0x4B000000u | ((w[c] >> (4 * n)) & 0xFu));
+            const float q1 = __uint_as_float(0x4B000000u | ((w[c] >> (4 * n + 4)) & 0xFu));
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(__fmul_rn(__fsub_rn(q0, zb), stp),
+                                                            __fmul_rn(__fsub_rn(q1, zb), stp));
+            o4[n / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+          }
+          const uint32_t chunk = static_cast<uint32_t>(c) ^ static_cast<uint32_t>(r & 7);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row_base + (chunk << 4)), "r"(o4[0]),
+                       "r"(o4[1]), "r"(o4[2]), "r"(o4[3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();  // the tensor cores read these bytes through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_rank(full_bar(s_own), 0));
+    }
+  } else {
+    // ------------------------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      const int t = ring_wait_warp(i, ok);
+      if (!ok || t < 0) break;
+      const int acc = i & 1;
+      const uint32_t acc_phase = static_cast<uint32_t>(i >> 1) & 1u;
+      if (!warp_wait_any(accf_bar(acc), acc_phase, st, p.limit_ns, kSiteEpiAccFull, false)) break;
+      tc_fence_after();
+      int band, mt;
+      tile_coords(t, p, band, mt);
+      const int64_t row = static_cast<int64_t>(mt) * BM + static_cast<int64_t>(rank) * HALF + quarter * 32 + lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
+        const int64_t col0 = static_cast<int64_t>(band) * BN + c * 32;
+        if (row < p.M && col0 < p.O) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+            packed[k] = *reinterpret_cast<const uint32_t*>(&pr);
+          }
+          __nv_bfloat16* dst = p.Y + row * p.ldy + col0;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (col0 + 8 * q < p.O)  // O % 8 == 0: 16-byte pieces are all in or all out
+              *reinterpret_cast<uint4*>(dst + 8 * q) =
+                  make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_rank(acce_bar(acc), 0));
+    }
+  }
+
+  if (status_code(st) != 0u) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 50000ull) __nanosleep(1000);
+  }
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace dq
+}  // namespace awq
