@@ -304,6 +304,7 @@ def run_ours(args, rank, world, local_rank):
     assert 0 <= best < J and torch.isfinite(res.losses).all()
 
     fold_ms = measure_fold(Wd, res.scales)
+    rules_ms = measure_rules(Xd, Wd, act, J)
     w4 = measure_w4a16(Xd, Wd, res.scales)
     e2e = None if args.no_e2e else measure_e2e(args, Xh, Wh, dev, J)
     e2e_ms = replicas.max_over_ranks(e2e["ms"] if e2e else 0.0, dev)
@@ -343,6 +344,7 @@ def run_ours(args, rank, world, local_rank):
                 / (np.mean(pack_ms) / 1e3) / 1e9,
                 "fold_gbs": (4.0 * O * K + 4.0 * K) / (fold_ms / 1e3) / 1e9,
                 "peak_gbs": peaks.get("hbm_gbs")},
+        "search_ms_by_rule": rules_ms,
         "w4a16": {"prefill_tokens": N, "prefill_ms": w4["prefill_ms"],
                   "prefill_tflops": 2.0 * N * O * K / (w4["prefill_ms"] / 1e3) / 1e12,
                   "prefill_frac_of_peak": 2.0 * N * O * K / (w4["prefill_ms"] / 1e3) / 1e12 / peaks["bf16_tflops"],
@@ -381,6 +383,29 @@ def measure_fold(Wd, scales):
         if i >= 2:
             times.append(e0.elapsed_time(e1))
     return float(np.mean(times))
+
+
+def measure_rules(Xd, Wd, act, J):
+    """awq_search time with each candidate-scale rule (the default, page 2's weight-aware rule, page 1's
+    RMS-normalised 11-point grid)."""
+    import torch
+
+    from weight_only_quantization_act_b200 import awq
+
+    out = {}
+    for rule, n in (("p4", J), ("weight_aware", J), ("rms", 11)):
+        res = awq.search(Xd, Wd, act, n_grid=n, rule=rule)
+        times = []
+        for i in range(4):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            awq.search(Xd, Wd, act, n_grid=n, rule=rule, workspace=res.workspace, out=res)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 1:
+                times.append(e0.elapsed_time(e1))
+        out[f"{rule}_n{n}"] = float(np.mean(times))
+    return out
 
 
 def measure_w4a16(Xd, Wd, scales):

@@ -71,6 +71,9 @@ typedef enum awq_status {
 #define AWQ_FLAG_EXACT_DIVISION 0x1u /* every w'/step quotient by IEEE division, no reciprocal fast path */
 #define AWQ_FLAG_EXACT_POW 0x2u      /* every act_mean^ratio by the double-double path, no fp64 pow */
 #define AWQ_FLAG_INJECT_STALL 0x100u /* test hook: the loss GEMM waits on a barrier nobody signals */
+/* Candidate-scale rule of the search (default: 原理 on the msModelSlim page, see (2) below). */
+#define AWQ_FLAG_SCALES_WEIGHT_AWARE 0x10u /* AWQChannelScaler on the bjdmk.com.cn article: see (2) */
+#define AWQ_FLAG_SCALES_RMS 0x20u          /* search_smooth_scaling_factors, gsyq.cn section 二: see (2) */
 
 #define AWQ_MAX_N_GRID 64
 
@@ -123,11 +126,22 @@ AWQ_API awq_status awq_act_stats_noalloc(const void *X, int64_t N, int64_t K, in
  * the candidates). Row j of table (device, float [n_grid, K]) receives, with r = RN32(j / n_grid):
  *   t = correctly rounded fp32 of act_mean[k]^r (0^0 = 1), t = max(t, RN32(1e-4)),
  *   d = RN32(sqrt(RN32(max_k t * min_k t))), s = RN32(t / d).
- * flags: 0 or AWQ_FLAG_EXACT_POW. 1 <= n_grid <= AWQ_MAX_N_GRID.
+ * flags: 0 or AWQ_FLAG_EXACT_POW, optionally with one of the alternative rules (also accepted by
+ * awq_search_ex), all bit-exact, P_j = RN32(j / (n_grid - 1)) (linspace(0, 1, n_grid), 1.0 included):
+ *   AWQ_FLAG_SCALES_WEIGHT_AWARE: t = max(RN32(CR32(a^P) / RN32(CR32(wm^RN32(1 - P)) + RN32(1e-6))), 1e-4),
+ *     then the same geometric normalisation; wm[k] = mean_o |W[o,k]| (fixed order as in (1)); only through
+ *     awq_scale_table_ex (which takes wm) or awq_search_ex.
+ *   AWQ_FLAG_SCALES_RMS: t = CR32(max(a, RN32(1e-5))^P); m = RN32(RN64(S / K)), S = fp64 sum of RN32(t^2)
+ *     in 256-column chunks (in order, chunk totals in order); s = max(RN32(t / RN32(sqrt(m))), 1e-4)
+ *     (n_grid = 11 gives the page's 0, 0.1, ..., 1.0).
+ * 1 <= n_grid <= AWQ_MAX_N_GRID.
  * ------------------------------------------------------------------------------------------------- */
 AWQ_API size_t awq_scale_table_workspace_size(int64_t K, int n_grid);
 AWQ_API awq_status awq_scale_table(const float *act_mean, int64_t K, int n_grid, unsigned flags, void *workspace,
                            size_t ws_bytes, float *table, awq_stream_t stream);
+AWQ_API awq_status awq_scale_table_ex(const float *act_mean, const float *weight_mean, int64_t K, int n_grid,
+                                      unsigned flags, void *workspace, size_t ws_bytes, float *table,
+                                      awq_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------------
  * (2)-(4) The search. For every candidate j it forms the weight error dW_j = W - W_hat_j (fp32, rounded
@@ -148,7 +162,8 @@ AWQ_API size_t awq_search_workspace_size(int64_t N, int64_t K, int64_t O, int gr
 AWQ_API awq_status awq_search(const void *X, int64_t N, int64_t K, int64_t ldx, const void *W, int64_t O,
                       int64_t ldw, const float *act_mean, int group, int n_grid, void *workspace,
                       size_t ws_bytes, double *losses, int *best_j, float *scales, awq_stream_t stream);
-/* Same, with flags (AWQ_FLAG_EXACT_DIVISION, AWQ_FLAG_EXACT_POW, AWQ_FLAG_INJECT_STALL). */
+/* Same, with flags (AWQ_FLAG_EXACT_DIVISION, AWQ_FLAG_EXACT_POW, AWQ_FLAG_INJECT_STALL, and one of
+ * AWQ_FLAG_SCALES_WEIGHT_AWARE / AWQ_FLAG_SCALES_RMS to search the alternative candidate scales). */
 AWQ_API awq_status awq_search_ex(const void *X, int64_t N, int64_t K, int64_t ldx, const void *W, int64_t O,
                          int64_t ldw, const float *act_mean, int group, int n_grid, unsigned flags,
                          void *workspace, size_t ws_bytes, double *losses, int *best_j, float *scales,

@@ -229,14 +229,22 @@ def argmin_first(losses) -> int:
     return best_j
 
 
-def search(x_bits, w_bits, n_grid: int = 20, group: int = GROUP, act=None, table=None):
+def search(x_bits, w_bits, n_grid: int = 20, group: int = GROUP, act=None, table=None, mode: str = "p4"):
     """The whole search for one linear (or several sharing X, rows of W concatenated).
 
+    mode selects the candidate scales: "p4" (default), "weight_aware" or "rms" (see the variants below).
     Returns dict(act_mean, table [n_grid,K], losses [n_grid] fp64, best_j, scales, codes, steps, zeros)."""
     if act is None:
         act = act_mean(x_bits)
     if table is None:
-        table = scale_table(act, n_grid)
+        if mode == "p4":
+            table = scale_table(act, n_grid)
+        elif mode == "weight_aware":
+            table = scale_table_weight_aware(act, weight_mean(w_bits), n_grid)
+        elif mode == "rms":
+            table = scale_table_rms(act, n_grid)
+        else:
+            raise ValueError(mode)
     losses = np.empty(n_grid, F64)
     for j in range(n_grid):
         w_hat, _, _, _ = pseudo_quantize(w_bits, table[j], group)
@@ -324,3 +332,71 @@ def w4a16_matmul(x_bits, words, steps, zeros, group: int = GROUP) -> np.ndarray:
     deq16 = widen_bf16(round_f32_to_bf16(dequant_w4(words, steps, zeros, group))).astype(F64)
     x = widen_bf16(x_bits).astype(F64)
     return x @ deq16.T
+
+
+# ---------------------------------------------------------------------------------------------------
+# (8) variants of the candidate scales
+#   weight-aware [P2 数学等价变换与通道自适应缩放, AWQChannelScaler]: s = clamp(act^p / (wmean^(1-p) + 1e-6),
+#       1e-4), s /= sqrt(max(s) min(s)), p over linspace(0, 1, n): p_j = RN32(j / (n - 1)) (1.0 included);
+#       wmean[k] = mean_o |W[o, k]| (the same fixed-order mean as the activation statistic).
+#   RMS-normalised [P1 section 二, search_smooth_scaling_factors]: a = clamp(act, 1e-5); s = a^alpha;
+#       s /= sqrt(mean(s^2)); s = clamp(s, 1e-4); alpha_j = RN32(j / (n - 1)) (n = 11 gives 0, 0.1, ..., 1.0).
+#       mean(s^2) = RN32(RN64(S / K)) with S the fp64 sum of RN32(s_k^2) in 256-column chunks (columns in
+#       order inside a chunk, chunk totals in order); the root and the division are single fp32 operations.
+# The quantizer and the loss are the ones above in both cases.
+# ---------------------------------------------------------------------------------------------------
+WEIGHT_EPS = F32(1e-6)
+RMS_ACT_FLOOR = F32(1e-5)
+
+
+def weight_mean(w_bits) -> np.ndarray:
+    """mean over output rows of |W[o, k]|, float32 [K] (same fixed order as act_mean)."""
+    return act_mean(w_bits)
+
+
+def closed_grid(j: int, n_grid: int) -> np.float32:
+    """Point j of linspace(0, 1, n_grid): RN32(j / (n_grid - 1)); a single point is 0."""
+    if n_grid == 1:
+        return F32(0)
+    return F32(F32(j) / F32(n_grid - 1))
+
+
+def scale_table_weight_aware(act, wmean, n_grid: int) -> np.ndarray:
+    act = np.asarray(act, F32)
+    wmean = np.asarray(wmean, F32)
+    cache_a: dict = {}
+    cache_w: dict = {}
+    rows = []
+    for j in range(n_grid):
+        p = closed_grid(j, n_grid)
+        q = F32(F32(1) - p)
+        t = _cr_pow_row(act, p, cache_a)
+        u = _cr_pow_row(wmean, q, cache_w)
+        s = np.maximum((t / (u + WEIGHT_EPS)).astype(F32), SCALE_FLOOR)
+        d = np.sqrt(F32(s.max() * s.min()))
+        rows.append((s / d).astype(F32))
+    return np.stack(rows)
+
+
+def _sum_sq_fixed(t: np.ndarray, chunk: int = 256) -> np.float64:
+    sq = (t * t).astype(F32).astype(F64)
+    total = F64(0)
+    for c0 in range(0, sq.shape[0], chunk):
+        part = F64(0)
+        for v in sq[c0:c0 + chunk]:
+            part = part + v
+        total = total + part
+    return total
+
+
+def scale_table_rms(act, n_grid: int) -> np.ndarray:
+    act = np.maximum(np.asarray(act, F32), RMS_ACT_FLOOR)
+    K = act.shape[0]
+    cache: dict = {}
+    rows = []
+    for j in range(n_grid):
+        t = _cr_pow_row(act, closed_grid(j, n_grid), cache)
+        m = F32(_sum_sq_fixed(t) / F64(K))
+        d = np.sqrt(m)
+        rows.append(np.maximum((t / d).astype(F32), SCALE_FLOOR))
+    return np.stack(rows)

@@ -216,3 +216,32 @@ def test_tile_partials_match_oracle():
                     blk = E[r0:r0 + rows, a * lay.tile_o:(a + 1) * lay.tile_o]
                     want = float((blk * blk).sum())
                     assert abs(parts[j, a, b, q] - want) <= LOSS_RTOL * want + 1e-300, (j, a, b, q)
+
+
+# ------------------------------------------------------------------------------------------------ scale rules
+@pytest.mark.parametrize("exact_pow", [False, True])
+def test_scale_table_rules_bit_exact(exact_pow):
+    act = edge_act_vector()
+    rng = np.random.default_rng(131)
+    wm = np.concatenate([rng.random(act.shape[0] - 2) * 0.05, [0.0, 1e-30]]).astype(F32)
+    got = awq.scale_table(torch.from_numpy(act).cuda(), 20, exact_pow=exact_pow, rule="weight_aware",
+                          weight_mean=torch.from_numpy(wm).cuda())
+    assert_bits_equal(got, orc.scale_table_weight_aware(act, wm, 20), "weight-aware table")
+    got = awq.scale_table(torch.from_numpy(act).cuda(), 11, exact_pow=exact_pow, rule="rms")
+    assert_bits_equal(got, orc.scale_table_rms(act, 11), "rms table")
+
+
+@pytest.mark.parametrize("rule,n_grid", [("weight_aware", 20), ("rms", 11)])
+def test_search_with_alternative_rules(rule, n_grid):
+    X = inputs.random_bf16((300, 384), seed=61, outliers=4, factor=50)
+    W = inputs.random_bf16((600, 384), seed=62, scale=0.02)
+    Xd, Wd = bf16_to_device(X), bf16_to_device(W)
+    act = awq.act_stats(Xd)
+    res = awq.search(Xd, Wd, act, n_grid=n_grid, rule=rule)
+    assert awq.search_status(res) == 0
+    ref = orc.search(X, W, n_grid=n_grid, mode=rule)
+    losses = res.losses.cpu().numpy()
+    assert np.all(loss_rel_err(losses, ref["losses"]) <= LOSS_RTOL)
+    best = int(res.best_j.item())
+    check_argmin_rule(best, ref["losses"])
+    assert_bits_equal(res.scales, ref["table"][best], "scales")

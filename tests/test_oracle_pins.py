@@ -491,3 +491,53 @@ def test_w4a16_hand_examples():
     q = rng.integers(0, 16, (O, K)).astype(np.uint8)
     y = orc.w4a16_matmul(x, orc.pack_codes(q), np.ones((O, 1), F32), np.zeros((O, 1), F32))
     assert np.array_equal(y, inputs.bf16_bits_to_f32(x).astype(np.float64) @ q.T.astype(np.float64))
+
+
+# ------------------------------------------------------------------------------------------ scale rules
+def test_closed_grid_points():
+    assert [orc.closed_grid(j, 11) for j in (0, 10)] == [0.0, 1.0]
+    for j in range(11):
+        assert orc.closed_grid(j, 11) == nearest_f32_of_fraction(Fraction(j, 10))
+    assert orc.closed_grid(0, 1) == 0.0
+
+
+def test_weight_aware_rule_end_points():
+    """p = 1 leaves act / (1 + 1e-6) (wmean^0 = 1); p = 0 leaves 1 / (wmean + 1e-6); both normalised."""
+    rng = np.random.default_rng(121)
+    act = (rng.random(200) * 3 + 0.01).astype(F32)
+    wm = (rng.random(200) * 0.05 + 0.001).astype(F32)
+    T = orc.scale_table_weight_aware(act, wm, 5)
+    for row, expect_order in ((T[-1], act), (T[0], -wm)):
+        order = np.argsort(expect_order, kind="stable")
+        assert np.all(np.diff(row[order]) >= 0)
+        assert abs(float(row.max()) * float(row.min()) - 1) <= 4 * 2.0 ** -23
+    eps = Fraction(float(F32(1e-6)))
+    one_plus = nearest_f32_of_fraction(1 + eps)
+    t = [nearest_f32_of_fraction(Fraction(float(a)) / Fraction(float(one_plus))) for a in act]
+    t = np.maximum(np.array(t, F32), F32(1e-4))
+    d = np.sqrt(F32(t.max() * t.min()))
+    assert np.array_equal(T[-1], (t / d).astype(F32))
+
+
+def test_rms_rule_end_points_and_sum():
+    rng = np.random.default_rng(122)
+    act = np.concatenate([rng.random(300) * 4, [0.0, 1e-7]]).astype(F32)
+    T = orc.scale_table_rms(act, 11)
+    assert np.all(T[0] == F32(1.0)), "alpha = 0 must give scales of exactly one"
+    a = np.maximum(act, F32(1e-5))
+    rms = np.sqrt(np.mean(T[-1].astype(np.float64) ** 2))
+    assert abs(rms - 1) < 1e-5
+    order = np.argsort(a, kind="stable")
+    for j in range(11):
+        assert np.all(np.diff(T[j][order]) >= 0)
+    # the fixed-order fp64 sum of the fp32 squares is within one fp64 rounding per chunk of the exact sum
+    sq = (a * a).astype(F32)
+    exact = sum(Fraction(float(v)) for v in sq)
+    assert abs(Fraction(float(orc._sum_sq_fixed(a))) - exact) <= exact * Fraction(1, 2 ** 45)
+
+
+def test_search_rules_pick_a_ratio_that_beats_rtn():
+    X, W, _ = inputs.make_inputs(inputs.workload(1))
+    for mode in ("weight_aware", "rms"):
+        res = orc.search(X, W, n_grid=11 if mode == "rms" else 20, mode=mode)
+        assert res["losses"][res["best_j"]] <= res["losses"][0]

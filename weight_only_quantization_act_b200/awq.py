@@ -26,6 +26,8 @@ STATUS_NAMES = {0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_UNSUPPORTED",
 FLAG_EXACT_DIVISION = 0x1
 FLAG_EXACT_POW = 0x2
 FLAG_INJECT_STALL = 0x100
+FLAG_SCALES_WEIGHT_AWARE = 0x10
+FLAG_SCALES_RMS = 0x20
 MAX_N_GRID = 64
 
 # name -> (restype, argtypes)
@@ -41,6 +43,7 @@ SIGNATURES = {
     "awq_act_stats_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P]),
     "awq_scale_table_workspace_size": (_SZ, [_I64, _I]),
     "awq_scale_table": (_I, [_P, _I64, _I, _U, _P, _SZ, _P, _P]),
+    "awq_scale_table_ex": (_I, [_P, _P, _I64, _I, _U, _P, _SZ, _P, _P]),
     "awq_search_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I]),
     "awq_search": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I, _I, _P, _SZ, _P, _P, _P, _P]),
     "awq_search_ex": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I, _I, _U, _P, _SZ, _P, _P, _P, _P]),
@@ -174,16 +177,22 @@ def act_stats_noalloc(X: torch.Tensor, out: torch.Tensor, stream=None) -> torch.
 
 
 # --------------------------------------------------------------------------------------------- (2)
-def scale_table(act_mean: torch.Tensor, n_grid: int = 20, exact_pow: bool = False, stream=None) -> torch.Tensor:
-    """float32 [n_grid, K] table of candidate scales."""
+def scale_table(act_mean: torch.Tensor, n_grid: int = 20, exact_pow: bool = False, rule: str = "p4",
+                weight_mean: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """float32 [n_grid, K] table of candidate scales; rule "p4" (default), "weight_aware" (needs
+    weight_mean) or "rms"."""
     lib = load_library()
     K = act_mean.shape[0]
     table = torch.empty((n_grid, K), dtype=torch.float32, device=act_mean.device)
     ws = _workspace(lib.awq_scale_table_workspace_size(K, n_grid), act_mean.device, None)
-    flags = FLAG_EXACT_POW if exact_pow else 0
-    _check("awq_scale_table", lib.awq_scale_table(_ptr(act_mean), K, n_grid, flags, _ptr(ws), ws.numel(),
-                                                  _ptr(table), _stream(stream)))
+    flags = (FLAG_EXACT_POW if exact_pow else 0) | RULE_FLAGS[rule]
+    wm = _ptr(weight_mean) if weight_mean is not None else None
+    _check("awq_scale_table_ex", lib.awq_scale_table_ex(_ptr(act_mean), wm, K, n_grid, flags, _ptr(ws), ws.numel(),
+                                                        _ptr(table), _stream(stream)))
     return table
+
+
+RULE_FLAGS = {"p4": 0, "weight_aware": FLAG_SCALES_WEIGHT_AWARE, "rms": FLAG_SCALES_RMS}
 
 
 # --------------------------------------------------------------------------------------------- (3)-(4)
@@ -218,9 +227,12 @@ def search_layout(N: int, K: int, O: int, n_grid: int = 20, group: int = 128) ->
 
 
 def search(X: torch.Tensor, W, act_mean: torch.Tensor, n_grid: int = 20, group: int = 128, flags: int = 0,
-           workspace: torch.Tensor | None = None, out: SearchResult | None = None, stream=None) -> SearchResult:
-    """Grid search of the AWQ scale ratio for one linear (or stacked linears sharing X)."""
+           workspace: torch.Tensor | None = None, out: SearchResult | None = None, rule: str = "p4",
+           stream=None) -> SearchResult:
+    """Grid search of the AWQ scale ratio for one linear (or stacked linears sharing X); rule selects the
+    candidate scales ("p4" default, "weight_aware", "rms")."""
     lib = load_library()
+    flags |= RULE_FLAGS[rule]
     X = _bf16_matrix("X", X)
     W = stack_weights(W)
     N, K = X.shape

@@ -170,7 +170,7 @@ ScaleLayout scale_layout(int64_t K, int n_grid) {
 
 struct SearchLayout {
   int64_t O_pad, tiles_n, tiles_o;
-  size_t status_off, produced_off, table_off, rtable_off, spart_off, partials_off, dw_off, bytes;
+  size_t status_off, produced_off, table_off, rtable_off, spart_off, wmean_off, wpart_off, partials_off, dw_off, bytes;
   ScaleLayout sl;
 };
 SearchLayout search_layout(int64_t N, int64_t K, int64_t O, int n_grid) {
@@ -189,6 +189,10 @@ SearchLayout search_layout(int64_t N, int64_t K, int64_t O, int n_grid) {
   off = align_up(off + static_cast<size_t>(n_grid) * K * sizeof(float), 256);
   l.spart_off = off;
   off = align_up(off + l.sl.bytes, 256);
+  l.wmean_off = off;  // weight-aware rule: mean |W| per column and its fixed-order chunk sums
+  off = align_up(off + static_cast<size_t>(K) * sizeof(float), 256);
+  l.wpart_off = off;
+  off = align_up(off + act_layout(O, K).bytes, 256);
   l.partials_off = off;
   off = align_up(off + static_cast<size_t>(n_grid) * l.tiles_o * l.tiles_n * awq::lg::PARTIALS_PER_TILE *
                            sizeof(double), 1024);
@@ -233,14 +237,21 @@ awq_status check_launch(const char* what) {
     if (s_ != AWQ_OK) return s_;        \
   } while (0)
 
-awq_status launch_scale_table(const float* act, int64_t K, int n_grid, bool exact_pow, float* table, float* rtable,
-                              float2* part, cudaStream_t st) {
+awq_status launch_scale_table(const float* act, const float* wmean, int64_t K, int n_grid, int mode, bool exact_pow,
+                              float* table, float* rtable, float2* part, cudaStream_t st) {
   const int nblk = static_cast<int>((K + awq::kScaleThreads - 1) / awq::kScaleThreads);
   dim3 grid(nblk, n_grid);
-  awq::scale_pow_kernel<<<grid, awq::kScaleThreads, 0, st>>>(act, K, n_grid, exact_pow ? 1 : 0, table, part);
+  awq::scale_pow_kernel<<<grid, awq::kScaleThreads, 0, st>>>(act, wmean, K, n_grid, mode, exact_pow ? 1 : 0, table,
+                                                              part);
   AWQ_TRY(check_launch("scale_pow_kernel"));
-  awq::scale_normalize_kernel<<<grid, awq::kScaleThreads, 0, st>>>(table, rtable, part, K, nblk);
+  awq::scale_normalize_kernel<<<grid, awq::kScaleThreads, 0, st>>>(table, rtable, part, K, nblk, mode);
   return check_launch("scale_normalize_kernel");
+}
+
+int scale_mode_of(unsigned flags) {
+  if (flags & AWQ_FLAG_SCALES_WEIGHT_AWARE) return awq::kScalesWeightAware;
+  if (flags & AWQ_FLAG_SCALES_RMS) return awq::kScalesRms;
+  return awq::kScalesP4;
 }
 
 }  // namespace
@@ -290,21 +301,33 @@ size_t awq_scale_table_workspace_size(int64_t K, int n_grid) {
   return scale_layout(K, n_grid).bytes;
 }
 
-awq_status awq_scale_table(const float* act_mean, int64_t K, int n_grid, unsigned flags, void* workspace,
-                           size_t ws_bytes, float* table, awq_stream_t stream) {
+awq_status awq_scale_table_ex(const float* act_mean, const float* weight_mean, int64_t K, int n_grid, unsigned flags,
+                              void* workspace, size_t ws_bytes, float* table, awq_stream_t stream) {
   if (act_mean == nullptr || table == nullptr) return fail(AWQ_ERR_INVALID_ARG, "null pointer");
   if (K < 1 || K >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "bad K");
   AWQ_TRY(check_grid(n_grid));
-  if (flags & ~AWQ_FLAG_EXACT_POW) return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~(AWQ_FLAG_EXACT_POW | AWQ_FLAG_SCALES_WEIGHT_AWARE | AWQ_FLAG_SCALES_RMS))
+    return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if ((flags & AWQ_FLAG_SCALES_WEIGHT_AWARE) && (flags & AWQ_FLAG_SCALES_RMS))
+    return fail(AWQ_ERR_INVALID_ARG, "choose one candidate-scale rule");
+  if ((flags & AWQ_FLAG_SCALES_WEIGHT_AWARE) && weight_mean == nullptr)
+    return fail(AWQ_ERR_INVALID_ARG, "the weight-aware rule needs weight_mean");
   const ScaleLayout l = scale_layout(K, n_grid);
   if (workspace == nullptr || ws_bytes < l.bytes)
     return fail(AWQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", l.bytes, workspace ? ws_bytes : 0);
   DeviceInfo* d = nullptr;
   AWQ_TRY(device_info(&d));
-  AWQ_TRY(launch_scale_table(act_mean, K, n_grid, (flags & AWQ_FLAG_EXACT_POW) != 0, table, nullptr,
-                             reinterpret_cast<float2*>(static_cast<char*>(workspace) + l.part_off),
+  AWQ_TRY(launch_scale_table(act_mean, weight_mean, K, n_grid, scale_mode_of(flags), (flags & AWQ_FLAG_EXACT_POW) != 0,
+                             table, nullptr, reinterpret_cast<float2*>(static_cast<char*>(workspace) + l.part_off),
                              reinterpret_cast<cudaStream_t>(stream)));
   return ok();
+}
+
+awq_status awq_scale_table(const float* act_mean, int64_t K, int n_grid, unsigned flags, void* workspace,
+                           size_t ws_bytes, float* table, awq_stream_t stream) {
+  if (flags & AWQ_FLAG_SCALES_WEIGHT_AWARE)
+    return fail(AWQ_ERR_INVALID_ARG, "the weight-aware rule needs awq_scale_table_ex");
+  return awq_scale_table_ex(act_mean, nullptr, K, n_grid, flags, workspace, ws_bytes, table, stream);
 }
 
 size_t awq_search_workspace_size(int64_t N, int64_t K, int64_t O, int group, int n_grid) {
@@ -338,8 +361,11 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   if (K % 128 != 0) return fail(AWQ_ERR_INVALID_ARG, "K (%lld) must be a multiple of 128", static_cast<long long>(K));
   if (act_mean == nullptr || losses == nullptr || best_j == nullptr || scales == nullptr)
     return fail(AWQ_ERR_INVALID_ARG, "null output or act_mean pointer");
-  if (flags & ~(AWQ_FLAG_EXACT_DIVISION | AWQ_FLAG_EXACT_POW | AWQ_FLAG_INJECT_STALL))
+  if (flags & ~(AWQ_FLAG_EXACT_DIVISION | AWQ_FLAG_EXACT_POW | AWQ_FLAG_INJECT_STALL | AWQ_FLAG_SCALES_WEIGHT_AWARE |
+                AWQ_FLAG_SCALES_RMS))
     return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if ((flags & AWQ_FLAG_SCALES_WEIGHT_AWARE) && (flags & AWQ_FLAG_SCALES_RMS))
+    return fail(AWQ_ERR_INVALID_ARG, "choose one candidate-scale rule");
   const SearchLayout l = search_layout(N, K, O, n_grid);
   if (static_cast<int64_t>(n_grid) * l.O_pad >= (1ll << 31))
     return fail(AWQ_ERR_INVALID_ARG, "n_grid * O is too large");
@@ -366,7 +392,21 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   auto* produced = reinterpret_cast<unsigned int*>(ws + l.produced_off);
 
   AWQ_CUDA(cudaMemsetAsync(ws + l.status_off, 0, 512, st));  // status word and production counters
-  AWQ_TRY(launch_scale_table(act_mean, K, n_grid, (flags & AWQ_FLAG_EXACT_POW) != 0, table, rtable, spart, st));
+  const int mode = scale_mode_of(flags);
+  float* wmean = reinterpret_cast<float*>(ws + l.wmean_off);
+  if (mode == awq::kScalesWeightAware) {
+    // mean |W| per column: the activation statistic's fixed-order kernels run on W
+    const ActLayout wl = act_layout(O, K);
+    double* wpart = reinterpret_cast<double*>(ws + l.wpart_off);
+    dim3 wgrid(static_cast<unsigned>((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock), wl.n_chunks);
+    awq::act_chunk_sums_kernel<<<wgrid, awq::kActThreads, awq::kActSmemBytes, st>>>(static_cast<const uint16_t*>(W), O,
+                                                                                     K, ldw, wpart);
+    AWQ_TRY(check_launch("act_chunk_sums_kernel"));
+    awq::act_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(wpart, O, K, wl.n_chunks, wmean);
+    AWQ_TRY(check_launch("act_finalize_kernel"));
+  }
+  AWQ_TRY(launch_scale_table(act_mean, wmean, K, n_grid, mode, (flags & AWQ_FLAG_EXACT_POW) != 0, table, rtable, spart,
+                             st));
 
   awq::lg::Params p;
   p.n_tiles_n = static_cast<int>(l.tiles_n);

@@ -127,49 +127,93 @@ __device__ __forceinline__ void block_max_min(float& mx, float& mn, float* red /
   }
 }
 
-// grid (ceil(K / 256), n_grid)
-__global__ void __launch_bounds__(kScaleThreads) scale_pow_kernel(const float* __restrict__ act, int64_t K,
-                                                                  int n_grid, int force_slow,
+// Candidate-scale rules (the `mode` of the scale kernels).
+enum ScaleMode : int {
+  kScalesP4 = 0,           // clamp(act^(j/n), 1e-4) / sqrt(max * min)
+  kScalesWeightAware = 1,  // clamp(act^p / (wmean^(1-p) + 1e-6), 1e-4) / sqrt(max * min), p = j/(n-1)
+  kScalesRms = 2,          // clamp(max(act, 1e-5)^a / sqrt(mean(s^2)), 1e-4), a = j/(n-1)
+};
+
+__device__ __forceinline__ float closed_grid(int j, int n_grid) {
+  return n_grid == 1 ? 0.0f : __fdiv_rn(static_cast<float>(j), static_cast<float>(n_grid - 1));
+}
+
+// grid (ceil(K / 256), n_grid). Modes P4 / weight-aware: t (clamped) to the table, per-block max/min to
+// part (float2). RMS mode: t (unclamped) to the table, the fp64 sum of RN32(t^2) over the block's 256
+// columns in column order to part (as a double).
+__global__ void __launch_bounds__(kScaleThreads) scale_pow_kernel(const float* __restrict__ act,
+                                                                  const float* __restrict__ wmean, int64_t K,
+                                                                  int n_grid, int mode, int force_slow,
                                                                   float* __restrict__ table,
                                                                   float2* __restrict__ part) {
   __shared__ float red[64];
+  __shared__ float sq[kScaleThreads];
   const int j = blockIdx.y;
   const int64_t k = static_cast<int64_t>(blockIdx.x) * kScaleThreads + threadIdx.x;
-  const float r = __fdiv_rn(static_cast<float>(j), static_cast<float>(n_grid));
-  float mx = 0.0f, mn = __int_as_float(0x7f800000);
+  const bool slow = force_slow != 0;
+  float t = 0.0f;
   if (k < K) {
-    const float t = fmaxf(pow_f32_cr(act[k], r, force_slow != 0), AWQ_SCALE_FLOOR);
+    if (mode == kScalesP4) {
+      const float r = __fdiv_rn(static_cast<float>(j), static_cast<float>(n_grid));
+      t = fmaxf(pow_f32_cr(act[k], r, slow), AWQ_SCALE_FLOOR);
+    } else if (mode == kScalesWeightAware) {
+      const float p = closed_grid(j, n_grid);
+      const float tp = pow_f32_cr_full(act[k], p, slow);
+      const float u = pow_f32_cr_full(wmean[k], __fsub_rn(1.0f, p), slow);
+      t = fmaxf(__fdiv_rn(tp, __fadd_rn(u, AWQ_WEIGHT_EPS)), AWQ_SCALE_FLOOR);
+    } else {
+      t = pow_f32_cr_full(fmaxf(act[k], AWQ_RMS_ACT_FLOOR), closed_grid(j, n_grid), slow);
+    }
     table[static_cast<int64_t>(j) * K + k] = t;
-    mx = t;
-    mn = t;
   }
+  if (mode == kScalesRms) {
+    sq[threadIdx.x] = __fmul_rn(t, t);  // columns past K contribute +0
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double acc = 0.0;
+      for (int i = 0; i < kScaleThreads; ++i) acc = __dadd_rn(acc, static_cast<double>(sq[i]));
+      reinterpret_cast<double*>(part)[static_cast<int64_t>(j) * gridDim.x + blockIdx.x] = acc;
+    }
+    return;
+  }
+  float mx = k < K ? t : 0.0f, mn = k < K ? t : __int_as_float(0x7f800000);
   block_max_min(mx, mn, red);
   if (threadIdx.x == 0) part[static_cast<int64_t>(j) * gridDim.x + blockIdx.x] = make_float2(mx, mn);
 }
 
-// grid (ceil(K / 256), n_grid): every block reduces the row's partial max/min (cheap, <= a few hundred
-// entries) and normalises its 256 columns in place. Optionally also writes RN32(1/s) for the producer.
+// grid (ceil(K / 256), n_grid): every block reduces the row's partials (cheap, <= a few hundred entries)
+// and normalises its 256 columns in place. Optionally also writes RN32(1/s) for the producer.
 __global__ void __launch_bounds__(kScaleThreads) scale_normalize_kernel(float* __restrict__ table,
                                                                         float* __restrict__ rtable,
                                                                         const float2* __restrict__ part,
-                                                                        int64_t K, int nblk) {
+                                                                        int64_t K, int nblk, int mode) {
   __shared__ float red[64];
-  const int j = blockIdx.y;
-  float mx = 0.0f, mn = __int_as_float(0x7f800000);
-  for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
-    const float2 v = part[static_cast<int64_t>(j) * nblk + b];
-    mx = fmaxf(mx, v.x);
-    mn = fminf(mn, v.y);
-  }
-  block_max_min(mx, mn, red);
   __shared__ float d_sh;
-  if (threadIdx.x == 0) d_sh = __fsqrt_rn(__fmul_rn(mx, mn));
+  const int j = blockIdx.y;
+  if (mode == kScalesRms) {
+    if (threadIdx.x == 0) {
+      double S = 0.0;  // chunk totals in chunk order
+      const double* ps = reinterpret_cast<const double*>(part) + static_cast<int64_t>(j) * nblk;
+      for (int b = 0; b < nblk; ++b) S = __dadd_rn(S, ps[b]);
+      d_sh = __fsqrt_rn(__double2float_rn(__ddiv_rn(S, static_cast<double>(K))));
+    }
+  } else {
+    float mx = 0.0f, mn = __int_as_float(0x7f800000);
+    for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+      const float2 v = part[static_cast<int64_t>(j) * nblk + b];
+      mx = fmaxf(mx, v.x);
+      mn = fminf(mn, v.y);
+    }
+    block_max_min(mx, mn, red);
+    if (threadIdx.x == 0) d_sh = __fsqrt_rn(__fmul_rn(mx, mn));
+  }
   __syncthreads();
   const float d = d_sh;
   const int64_t k = static_cast<int64_t>(blockIdx.x) * kScaleThreads + threadIdx.x;
   if (k < K) {
     const int64_t idx = static_cast<int64_t>(j) * K + k;
-    const float s = __fdiv_rn(table[idx], d);
+    float s = __fdiv_rn(table[idx], d);
+    if (mode == kScalesRms) s = fmaxf(s, AWQ_SCALE_FLOOR);
     table[idx] = s;
     if (rtable != nullptr) rtable[idx] = __frcp_rn(s);
   }

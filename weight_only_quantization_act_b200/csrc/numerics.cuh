@@ -155,6 +155,24 @@ __device__ __forceinline__ float pow_f32_cr(float a, float r, bool force_slow) {
   return pow_f32_slow(a, r);
 }
 
+// Same correctly rounded power for results that matter below the 1e-4 floor as well (the scale variants
+// divide or normalise before clamping): no shortcut for small results, and every result below the
+// smallest normal fp32 (where fewer mantissa bits remain) goes through the double-double path.
+__device__ __forceinline__ float pow_f32_cr_full(float a, float r, bool force_slow) {
+  if (r == 0.0f) return 1.0f;
+  if (a == 0.0f) return 0.0f;
+  const double y = pow(static_cast<double>(a), static_cast<double>(r));
+  if (!force_slow && y >= 0x1p-126) {
+    const uint64_t low = static_cast<uint64_t>(__double_as_longlong(y)) & ((1ull << 29) - 1ull);
+    const int64_t off = static_cast<int64_t>(low) - (1ll << 28);
+    if (off > (1ll << 11) || off < -(1ll << 11)) return __double2float_rn(y);
+  }
+  return pow_f32_slow(a, r);
+}
+
+#define AWQ_WEIGHT_EPS 0x1.0c6f7ap-20f   // 1e-6 added to the powered weight mean (weight-aware scales)
+#define AWQ_RMS_ACT_FLOOR 0x1.4f8b58p-17f  // 1e-5 floor of the statistic (RMS-normalised scales)
+
 // ===================================================================================================
 // Asymmetric 4-bit group quantizer (section 二 of the gsyq.cn AWQ page), fp32, one rounding per step.
 // ===================================================================================================
