@@ -229,10 +229,13 @@ def argmin_first(losses) -> int:
     return best_j
 
 
-def search(x_bits, w_bits, n_grid: int = 20, group: int = GROUP, act=None, table=None, mode: str = "p4"):
+def search(x_bits, w_bits, n_grid: int = 20, group: int = GROUP, act=None, table=None, mode: str = "p4",
+           quant: str = "int4"):
     """The whole search for one linear (or several sharing X, rows of W concatenated).
 
     mode selects the candidate scales: "p4" (default), "weight_aware" or "rms" (see the variants below).
+    quant selects the weight quantizer: "int4" (asymmetric, groups of ``group``) or "int8" (symmetric
+    per output channel, section (9); zeros is then None and codes are int8).
     Returns dict(act_mean, table [n_grid,K], losses [n_grid] fp64, best_j, scales, codes, steps, zeros)."""
     if act is None:
         act = act_mean(x_bits)
@@ -246,13 +249,16 @@ def search(x_bits, w_bits, n_grid: int = 20, group: int = GROUP, act=None, table
         else:
             raise ValueError(mode)
     losses = np.empty(n_grid, F64)
+    if quant not in ("int4", "int8"):
+        raise ValueError(quant)
+    pq = pseudo_quantize if quant == "int4" else (lambda w, s, g: pseudo_quantize_int8(w, s) + (None,))
     for j in range(n_grid):
-        w_hat, _, _, _ = pseudo_quantize(w_bits, table[j], group)
+        w_hat = pq(w_bits, table[j], group)[0]
         losses[j] = loss_of(x_bits, w_bits, w_hat)
     best = argmin_first(losses)
-    _, q, step, z = pseudo_quantize(w_bits, table[best], group)
+    _, q, step, z = pq(w_bits, table[best], group)
     return dict(act_mean=act, table=table, losses=losses, best_j=best, scales=table[best].copy(),
-                codes=q.astype(np.uint8), steps=step, zeros=z)
+                codes=q.astype(np.uint8 if quant == "int4" else np.int8), steps=step, zeros=z)
 
 
 # ---------------------------------------------------------------------------------------------------
@@ -400,3 +406,36 @@ def scale_table_rms(act, n_grid: int) -> np.ndarray:
         d = np.sqrt(m)
         rows.append(np.maximum((t / d).astype(F32), SCALE_FLOOR))
     return np.stack(rows)
+
+
+# ---------------------------------------------------------------------------------------------------
+# (9) INT8 symmetric per-channel quantizer for the search   [P4 YAML weight_qconfig: per_channel, int8,
+#     symmetric, minmax; P5 section 2.1: q = clamp(round(x / s), -127, 127), s = max|x| / 127]
+#     per output row o of W' = W diag(s): step = max(RN32(max_k |w'| / 127), 1e-5) (the 1e-5 floor as in the
+#     INT4 quantizer, so an all-zero row stays finite); q = min(max(rint(RN32(w' / step)), -127), 127);
+#     deq = RN32(q * step).
+# ---------------------------------------------------------------------------------------------------
+QMAX8 = F32(127)
+
+
+def quantize_rows_int8(wp):
+    wp = np.asarray(wp, F32)
+    amax = np.abs(wp).max(axis=1)
+    step = np.maximum((amax / QMAX8).astype(F32), STEP_FLOOR).astype(F32)
+    q = np.minimum(np.maximum(np.rint(wp / step[:, None]), -QMAX8), QMAX8).astype(F32)
+    deq = (q * step[:, None]).astype(F32)
+    return q, step, deq
+
+
+def pseudo_quantize_int8(w_bits_or_f32, s):
+    """w_hat = RN32(deq / s) with the INT8 per-channel quantizer on W diag(s). Returns (w_hat, q, step)."""
+    w = _as_f32_weight(w_bits_or_f32)
+    s = np.asarray(s, F32)
+    q, step, deq = quantize_rows_int8((w * s[None, :]).astype(F32))
+    return (deq / s[None, :]).astype(F32), q, step
+
+
+def quantize_pack_int8(w_bits, s):
+    """(codes int8 [O, K], steps float32 [O]) of W at scales s."""
+    _, q, step = pseudo_quantize_int8(w_bits, s)
+    return q.astype(np.int8), step

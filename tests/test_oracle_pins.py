@@ -541,3 +541,72 @@ def test_search_rules_pick_a_ratio_that_beats_rtn():
     for mode in ("weight_aware", "rms"):
         res = orc.search(X, W, n_grid=11 if mode == "rms" else 20, mode=mode)
         assert res["losses"][res["best_j"]] <= res["losses"][0]
+
+
+# ------------------------------------------------------------------------------------------------ f4
+def test_int8_worked_example_of_the_outlier_page():
+    """The page's two cases: one outlier of 23 wipes 0.03 out (code 0); without it 0.03 keeps code 38."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "int8_outlier_example.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        wp = np.array([[c["max_abs"], c["x"], -c["max_abs"] / 4, 0.0]], F32)
+        q, step, deq = orc.quantize_rows_int8(wp)
+        assert round(float(step[0]), c["scale_digits"]) == c["scale_printed"]
+        assert int(q[0, 1]) == c["code"]
+        assert q[0, 0] == 127
+        if "dequant_printed" in c:
+            assert round(float(deq[0, 1]), c["dequant_digits"]) == c["dequant_printed"]
+            assert abs(float(deq[0, 1]) - c["x"]) / c["x"] < c["relative_error_below"]
+        else:
+            assert float(deq[0, 1]) == c["dequant"]
+
+
+def test_int8_step_is_exact_division_and_codes_nearest_of_255_levels():
+    """step = nearest fp32 of max|w'| / 127; each code is the nearest of the 255 levels by exact arithmetic
+    (a near-tie may go either way); the row's max |w'| gets code +-127."""
+    rng = np.random.default_rng(131)
+    wp = (rng.standard_normal((12, 96)) * rng.uniform(0.001, 4, (12, 1))).astype(F32)
+    q, step, deq = orc.quantize_rows_int8(wp)
+    for o in range(wp.shape[0]):
+        amax = max(abs(Fraction(float(v))) for v in wp[o])
+        assert step[o] == max(nearest_f32_of_fraction(amax / 127), F32(1e-5))
+        st = Fraction(float(step[o]))
+        for k in range(wp.shape[1]):
+            w = Fraction(float(wp[o, k]))
+            quo = w / st
+            nearest = min(range(-127, 128), key=lambda lvl: abs(quo - lvl))
+            if int(q[o, k]) != nearest:
+                half = Fraction(int(np.floor(float(quo)))) + Fraction(1, 2)
+                assert abs(quo - half) <= 2 * abs(quo) * Fraction(1, 2 ** 23), (o, k)
+            assert deq[o, k] == nearest_f32_of_fraction(Fraction(int(q[o, k])) * st)
+        kmax = int(np.argmax(np.abs(wp[o])))
+        assert abs(int(q[o, kmax])) == 127 and np.sign(q[o, kmax]) == np.sign(wp[o, kmax])
+
+
+def test_int8_symmetry_zero_rows_and_error_bound():
+    rng = np.random.default_rng(132)
+    wp = (rng.standard_normal((8, 256)) * 0.3).astype(F32)
+    wp[3] = 0.0
+    q, step, deq = orc.quantize_rows_int8(wp)
+    qn, stepn, _ = orc.quantize_rows_int8(-wp)
+    assert np.array_equal(step, stepn) and np.array_equal(q, -qn), "the quantizer is odd-symmetric"
+    assert step[3] == F32(1e-5) and np.all(q[3] == 0)
+    assert q.min() >= -127 and q.max() <= 127
+    err = np.abs(wp.astype(np.float64) - deq.astype(np.float64))
+    assert np.all(err <= step[:, None].astype(np.float64) / 2 * (1 + 2.0 ** -21) + 1e-30)
+
+
+def test_int8_search_ratio_zero_is_per_channel_rtn_and_beats_int4():
+    X, W, _ = inputs.make_inputs(inputs.workload(1))
+    res8 = orc.search(X, W, n_grid=20, quant="int8")
+    res4 = orc.search(X, W, n_grid=20)
+    w = inputs.bf16_bits_to_f32(W)
+    q, step, deq = orc.quantize_rows_int8(w)  # s = 1 at ratio 0 (act^0 = 1, normalised to 1)
+    assert np.all(res8["table"][0] == F32(1))
+    assert res8["losses"][0] == orc.loss_of(X, W, deq)
+    assert res8["codes"].dtype == np.int8 and res8["zeros"] is None
+    assert res8["losses"][res8["best_j"]] <= res8["losses"][0]
+    # 255 levels per channel against 16 per group of 128: far smaller error on these Gaussian rows
+    assert res8["losses"].min() < res4["losses"].min() / 10
