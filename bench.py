@@ -305,6 +305,7 @@ def run_ours(args, rank, world, local_rank):
 
     fold_ms = measure_fold(Wd, res.scales)
     rules_ms = measure_rules(Xd, Wd, act, J)
+    int8_pack_ms = measure_int8_pack(Wd, res.scales)
     w4 = measure_w4a16(Xd, Wd, res.scales)
     e2e = None if args.no_e2e else measure_e2e(args, Xh, Wh, dev, J)
     e2e_ms = replicas.max_over_ranks(e2e["ms"] if e2e else 0.0, dev)
@@ -343,6 +344,7 @@ def run_ours(args, rank, world, local_rank):
                 "quantize_pack_gbs": (2.0 * O * K + 4.0 * K + O * K / 2.0 + 8.0 * O * K / 128)
                 / (np.mean(pack_ms) / 1e3) / 1e9,
                 "fold_gbs": (4.0 * O * K + 4.0 * K) / (fold_ms / 1e3) / 1e9,
+                "int8_pack_gbs": (2.0 * O * K + 4.0 * K + 1.0 * O * K + 4.0 * O) / (int8_pack_ms / 1e3) / 1e9,
                 "peak_gbs": peaks.get("hbm_gbs")},
         "search_ms_by_rule": rules_ms,
         "w4a16": {"prefill_tokens": N, "prefill_ms": w4["prefill_ms"],
@@ -387,25 +389,45 @@ def measure_fold(Wd, scales):
 
 def measure_rules(Xd, Wd, act, J):
     """awq_search time with each candidate-scale rule (the default, page 2's weight-aware rule, page 1's
-    RMS-normalised 11-point grid)."""
+    RMS-normalised 11-point grid), and with the INT8 per-channel quantizer in place of INT4."""
     import torch
 
     from weight_only_quantization_act_b200 import awq
 
     out = {}
-    for rule, n in (("p4", J), ("weight_aware", J), ("rms", 11)):
-        res = awq.search(Xd, Wd, act, n_grid=n, rule=rule)
+    for rule, n, quant in (("p4", J, "int4"), ("weight_aware", J, "int4"), ("rms", 11, "int4"), ("p4", J, "int8")):
+        res = awq.search(Xd, Wd, act, n_grid=n, rule=rule, quant=quant)
         times = []
         for i in range(4):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            awq.search(Xd, Wd, act, n_grid=n, rule=rule, workspace=res.workspace, out=res)
+            awq.search(Xd, Wd, act, n_grid=n, rule=rule, quant=quant, workspace=res.workspace, out=res)
             e1.record()
             torch.cuda.synchronize()
             if i >= 1:
                 times.append(e0.elapsed_time(e1))
-        out[f"{rule}_n{n}"] = float(np.mean(times))
+        out[f"{rule}_n{n}" if quant == "int4" else f"{quant}_{rule}_n{n}"] = float(np.mean(times))
     return out
+
+
+def measure_int8_pack(Wd, scales):
+    """awq_quantize_pack_int8 alone (L2 flushed before every launch), in ms."""
+    import torch
+
+    from weight_only_quantization_act_b200 import awq
+
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=Wd.device)
+    times = []
+    for i in range(6):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        awq.quantize_pack_int8(Wd, scales)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            times.append(e0.elapsed_time(e1))
+    return float(np.mean(times))
 
 
 def measure_w4a16(Xd, Wd, scales):

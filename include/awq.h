@@ -61,7 +61,7 @@ typedef struct CUstream_st *awq_stream_t; /* identical to cudaStream_t */
 typedef enum awq_status {
   AWQ_OK = 0,
   AWQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, misalignment, n_grid out of range */
-  AWQ_ERR_UNSUPPORTED = 2, /* group != 128, or a device other than sm_100 */
+  AWQ_ERR_UNSUPPORTED = 2, /* group not 128 (0 with AWQ_FLAG_QUANT_INT8), or a device other than sm_100 */
   AWQ_ERR_WORKSPACE = 3,   /* workspace null or smaller than the *_workspace_size() query */
   AWQ_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed; message from the runtime */
   AWQ_ERR_TIMEOUT = 5      /* a bounded device wait gave up (reported by awq_search_status) */
@@ -74,6 +74,8 @@ typedef enum awq_status {
 /* Candidate-scale rule of the search (default: 原理 on the msModelSlim page, see (2) below). */
 #define AWQ_FLAG_SCALES_WEIGHT_AWARE 0x10u /* AWQChannelScaler on the bjdmk.com.cn article: see (2) */
 #define AWQ_FLAG_SCALES_RMS 0x20u          /* search_smooth_scaling_factors, gsyq.cn section 二: see (2) */
+/* Weight quantizer of the search (default: asymmetric INT4 in groups of 128, see (3)). */
+#define AWQ_FLAG_QUANT_INT8 0x40u /* symmetric INT8, one step per output channel: see (5b); group must be 0 */
 
 #define AWQ_MAX_N_GRID 64
 
@@ -157,13 +159,16 @@ AWQ_API awq_status awq_scale_table_ex(const float *act_mean, const float *weight
  * The scales, and the codes/steps/zeros that awq_quantize_pack derives from them, are bit-exact
  * functions of (act_mean, W); the losses carry bf16 rounding of dW and fp32 tensor-core accumulation.
  * Requires N >= 1, O >= 1, K >= 128, K % 128 == 0, N, O, K < 2^31, 1 <= n_grid <= AWQ_MAX_N_GRID.
+ * group: 128 (INT4 groups of 128 in-features), or 0 (per output channel) together with
+ * AWQ_FLAG_QUANT_INT8; the workspace size is the same for both.
  * ------------------------------------------------------------------------------------------------- */
 AWQ_API size_t awq_search_workspace_size(int64_t N, int64_t K, int64_t O, int group, int n_grid);
 AWQ_API awq_status awq_search(const void *X, int64_t N, int64_t K, int64_t ldx, const void *W, int64_t O,
                       int64_t ldw, const float *act_mean, int group, int n_grid, void *workspace,
                       size_t ws_bytes, double *losses, int *best_j, float *scales, awq_stream_t stream);
-/* Same, with flags (AWQ_FLAG_EXACT_DIVISION, AWQ_FLAG_EXACT_POW, AWQ_FLAG_INJECT_STALL, and one of
- * AWQ_FLAG_SCALES_WEIGHT_AWARE / AWQ_FLAG_SCALES_RMS to search the alternative candidate scales). */
+/* Same, with flags (AWQ_FLAG_EXACT_DIVISION, AWQ_FLAG_EXACT_POW, AWQ_FLAG_INJECT_STALL, one of
+ * AWQ_FLAG_SCALES_WEIGHT_AWARE / AWQ_FLAG_SCALES_RMS to search the alternative candidate scales, and
+ * AWQ_FLAG_QUANT_INT8 with group 0 to search with the INT8 per-channel quantizer of (5b)). */
 AWQ_API awq_status awq_search_ex(const void *X, int64_t N, int64_t K, int64_t ldx, const void *W, int64_t O,
                          int64_t ldw, const float *act_mean, int group, int n_grid, unsigned flags,
                          void *workspace, size_t ws_bytes, double *losses, int *best_j, float *scales,
@@ -207,6 +212,23 @@ AWQ_API awq_status awq_quantize_pack(const void *W, int64_t O, int64_t K, int64_
 AWQ_API awq_status awq_quantize_pack_ex(const void *W, int64_t O, int64_t K, int64_t ldw, const float *scales,
                                 int group, unsigned flags, uint32_t *codes, float *steps, float *zeros,
                                 awq_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------------
+ * (5b) Symmetric INT8 codes of W at given scales, one step per output channel (formula of section 2.1
+ * of the hncyxsy.com large-model outlier article, with the per-channel weight setting of the
+ * quantization YAML on the msModelSlim page). With w' = RN32(w * s_k) over the row's K in-features:
+ *   step_o = max(RN32(max_k |w'| / 127), RN32(1e-5))    q = min(max(rint(RN32(w' / step_o)), -127), 127)
+ * and the dequantized value is RN32(q * step_o). The search with AWQ_FLAG_QUANT_INT8 scores exactly this
+ * quantizer (w_hat = RN32(q * step_o) * RN32(1 / s_k), as for INT4).
+ *   W      device bf16 [O, ldw] as in awq_search
+ *   scales device float [K], 16-byte aligned
+ *   codes  device int8 [O, K] row-major (row stride K), 8-byte aligned (output)
+ *   steps  device float [O] (output)
+ *   flags  0 or AWQ_FLAG_EXACT_DIVISION
+ * Bit-exact: every operation is one IEEE fp32 operation in the order above. Requires K % 8 == 0.
+ * ------------------------------------------------------------------------------------------------- */
+AWQ_API awq_status awq_quantize_pack_int8(const void *W, int64_t O, int64_t K, int64_t ldw, const float *scales,
+                                          unsigned flags, int8_t *codes, float *steps, awq_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------------
  * Applying the chosen scales (SubgraphFusionFactory step of 缩放因子搜索流程 on the msModelSlim page):

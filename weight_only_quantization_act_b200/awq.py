@@ -28,6 +28,7 @@ FLAG_EXACT_POW = 0x2
 FLAG_INJECT_STALL = 0x100
 FLAG_SCALES_WEIGHT_AWARE = 0x10
 FLAG_SCALES_RMS = 0x20
+FLAG_QUANT_INT8 = 0x40
 MAX_N_GRID = 64
 
 # name -> (restype, argtypes)
@@ -51,6 +52,7 @@ SIGNATURES = {
     "awq_search_get_layout": (_I, [_I64, _I64, _I64, _I, _I, _P]),
     "awq_quantize_pack": (_I, [_P, _I64, _I64, _I64, _P, _I, _P, _P, _P, _P]),
     "awq_quantize_pack_ex": (_I, [_P, _I64, _I64, _I64, _P, _I, _U, _P, _P, _P, _P]),
+    "awq_quantize_pack_int8": (_I, [_P, _I64, _I64, _I64, _P, _U, _P, _P, _P]),
     "awq_scale_columns": (_I, [_P, _I64, _I64, _I64, _P, _I, _P, _I64, _P]),
     "awq_scale_rows": (_I, [_P, _I64, _I64, _I64, _P, _I, _P, _I64, _P]),
     "awq_w4a16_workspace_size": (_SZ, [_I64, _I64]),
@@ -228,11 +230,17 @@ def search_layout(N: int, K: int, O: int, n_grid: int = 20, group: int = 128) ->
 
 def search(X: torch.Tensor, W, act_mean: torch.Tensor, n_grid: int = 20, group: int = 128, flags: int = 0,
            workspace: torch.Tensor | None = None, out: SearchResult | None = None, rule: str = "p4",
-           stream=None) -> SearchResult:
+           quant: str = "int4", stream=None) -> SearchResult:
     """Grid search of the AWQ scale ratio for one linear (or stacked linears sharing X); rule selects the
-    candidate scales ("p4" default, "weight_aware", "rms")."""
+    candidate scales ("p4" default, "weight_aware", "rms"); quant the weight quantizer ("int4" in groups
+    of `group`, or "int8" symmetric per output channel, for which group is ignored)."""
     lib = load_library()
     flags |= RULE_FLAGS[rule]
+    if quant == "int8":
+        flags |= FLAG_QUANT_INT8
+        group = 0
+    elif quant != "int4":
+        raise ValueError(f"quant must be 'int4' or 'int8', not {quant!r}")
     X = _bf16_matrix("X", X)
     W = stack_weights(W)
     N, K = X.shape
@@ -278,6 +286,18 @@ def quantize_pack(W: torch.Tensor, scales: torch.Tensor, group: int = 128, flags
         _ptr(W), O, K, W.stride(0), _ptr(scales), group, flags, _ptr(codes), _ptr(steps), _ptr(zeros),
         _stream(stream)))
     return codes, steps, zeros
+
+
+def quantize_pack_int8(W: torch.Tensor, scales: torch.Tensor, flags: int = 0, stream=None):
+    """(codes int8 [O, K], steps float32 [O]): symmetric INT8, one step per output channel."""
+    lib = load_library()
+    W = stack_weights(W)
+    O, K = W.shape
+    codes = torch.empty((O, K), dtype=torch.int8, device=W.device)
+    steps = torch.empty(O, dtype=torch.float32, device=W.device)
+    _check("awq_quantize_pack_int8", lib.awq_quantize_pack_int8(
+        _ptr(W), O, K, W.stride(0), _ptr(scales), flags, _ptr(codes), _ptr(steps), _stream(stream)))
+    return codes, steps
 
 
 def quantize_layer(X: torch.Tensor, W, n_grid: int = 20, group: int = 128, stream=None):

@@ -170,7 +170,8 @@ ScaleLayout scale_layout(int64_t K, int n_grid) {
 
 struct SearchLayout {
   int64_t O_pad, tiles_n, tiles_o;
-  size_t status_off, produced_off, table_off, rtable_off, spart_off, wmean_off, wpart_off, partials_off, dw_off, bytes;
+  size_t status_off, produced_off, table_off, rtable_off, spart_off, wmean_off, wpart_off, rowstep_off, partials_off,
+      dw_off, bytes;
   ScaleLayout sl;
 };
 SearchLayout search_layout(int64_t N, int64_t K, int64_t O, int n_grid) {
@@ -193,6 +194,8 @@ SearchLayout search_layout(int64_t N, int64_t K, int64_t O, int n_grid) {
   off = align_up(off + static_cast<size_t>(K) * sizeof(float), 256);
   l.wpart_off = off;
   off = align_up(off + act_layout(O, K).bytes, 256);
+  l.rowstep_off = off;  // INT8 quantizer: per-candidate, per-row steps
+  off = align_up(off + static_cast<size_t>(n_grid) * l.O_pad * sizeof(float), 256);
   l.partials_off = off;
   off = align_up(off + static_cast<size_t>(n_grid) * l.tiles_o * l.tiles_n * awq::lg::PARTIALS_PER_TILE *
                            sizeof(double), 1024);
@@ -331,13 +334,13 @@ awq_status awq_scale_table(const float* act_mean, int64_t K, int n_grid, unsigne
 }
 
 size_t awq_search_workspace_size(int64_t N, int64_t K, int64_t O, int group, int n_grid) {
-  if (N < 1 || K < 1 || O < 1 || group != 128 || n_grid < 1 || n_grid > AWQ_MAX_N_GRID) return 0;
+  if (N < 1 || K < 1 || O < 1 || (group != 128 && group != 0) || n_grid < 1 || n_grid > AWQ_MAX_N_GRID) return 0;
   return search_layout(N, K, O, n_grid).bytes;
 }
 
 awq_status awq_search_get_layout(int64_t N, int64_t K, int64_t O, int group, int n_grid, awq_search_layout* out) {
   if (out == nullptr) return fail(AWQ_ERR_INVALID_ARG, "out is null");
-  AWQ_TRY(check_group(group));
+  if (group != 0) AWQ_TRY(check_group(group));
   AWQ_TRY(check_grid(n_grid));
   if (N < 1 || K < 1 || O < 1) return fail(AWQ_ERR_INVALID_ARG, "empty shape");
   const SearchLayout l = search_layout(N, K, O, n_grid);
@@ -354,7 +357,10 @@ awq_status awq_search_get_layout(int64_t N, int64_t K, int64_t O, int group, int
 awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const void* W, int64_t O, int64_t ldw,
                          const float* act_mean, int group, int n_grid, unsigned flags, void* workspace,
                          size_t ws_bytes, double* losses, int* best_j, float* scales, awq_stream_t stream) {
-  AWQ_TRY(check_group(group));
+  const bool int8 = (flags & AWQ_FLAG_QUANT_INT8) != 0;
+  if (int8 && group != 0)
+    return fail(AWQ_ERR_UNSUPPORTED, "group %d: the INT8 quantizer is per channel (pass group 0)", group);
+  if (!int8) AWQ_TRY(check_group(group));
   AWQ_TRY(check_grid(n_grid));
   AWQ_TRY(check_matrix("X", X, N, K, ldx));
   AWQ_TRY(check_matrix("W", W, O, K, ldw));
@@ -362,7 +368,7 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   if (act_mean == nullptr || losses == nullptr || best_j == nullptr || scales == nullptr)
     return fail(AWQ_ERR_INVALID_ARG, "null output or act_mean pointer");
   if (flags & ~(AWQ_FLAG_EXACT_DIVISION | AWQ_FLAG_EXACT_POW | AWQ_FLAG_INJECT_STALL | AWQ_FLAG_SCALES_WEIGHT_AWARE |
-                AWQ_FLAG_SCALES_RMS))
+                AWQ_FLAG_SCALES_RMS | AWQ_FLAG_QUANT_INT8))
     return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if ((flags & AWQ_FLAG_SCALES_WEIGHT_AWARE) && (flags & AWQ_FLAG_SCALES_RMS))
     return fail(AWQ_ERR_INVALID_ARG, "choose one candidate-scale rule");
@@ -407,6 +413,15 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   }
   AWQ_TRY(launch_scale_table(act_mean, wmean, K, n_grid, mode, (flags & AWQ_FLAG_EXACT_POW) != 0, table, rtable, spart,
                              st));
+  float* rowstep = nullptr;
+  if (int8) {
+    // The per-channel step needs the whole row's max |w'| before any element is coded.
+    rowstep = reinterpret_cast<float*>(ws + l.rowstep_off);
+    dim3 rgrid(static_cast<unsigned>(l.O_pad * 32 / awq::kRowThreads), static_cast<unsigned>(n_grid));
+    awq::int8_rowstep_kernel<<<rgrid, awq::kRowThreads, 0, st>>>(static_cast<const uint16_t*>(W), O, l.O_pad, K, ldw,
+                                                                 table, rowstep);
+    AWQ_TRY(check_launch("int8_rowstep_kernel"));
+  }
 
   awq::lg::Params p;
   p.n_tiles_n = static_cast<int>(l.tiles_n);
@@ -430,6 +445,7 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   p.prod.rtable = rtable;
   p.prod.dW = dw;
   p.prod.exact = (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0;
+  p.prod.rowstep = rowstep;
   p.items_per_cand = l.O_pad * p.prod.segs;
   p.produced = produced;
   p.tile_counter = reinterpret_cast<unsigned int*>(ws + l.status_off + 20);
@@ -512,6 +528,26 @@ awq_status awq_quantize_pack_ex(const void* W, int64_t O, int64_t K, int64_t ldw
 awq_status awq_quantize_pack(const void* W, int64_t O, int64_t K, int64_t ldw, const float* scales, int group,
                              uint32_t* codes, float* steps, float* zeros, awq_stream_t stream) {
   return awq_quantize_pack_ex(W, O, K, ldw, scales, group, 0u, codes, steps, zeros, stream);
+}
+
+awq_status awq_quantize_pack_int8(const void* W, int64_t O, int64_t K, int64_t ldw, const float* scales,
+                                  unsigned flags, int8_t* codes, float* steps, awq_stream_t stream) {
+  AWQ_TRY(check_matrix("W", W, O, K, ldw));
+  if (K % 8 != 0) return fail(AWQ_ERR_INVALID_ARG, "K (%lld) must be a multiple of 8", static_cast<long long>(K));
+  if (scales == nullptr || codes == nullptr || steps == nullptr) return fail(AWQ_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(scales) || (reinterpret_cast<uintptr_t>(codes) & 7u) != 0)
+    return fail(AWQ_ERR_INVALID_ARG, "scales must be 16-byte and codes 8-byte aligned");
+  if (flags & ~AWQ_FLAG_EXACT_DIVISION) return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  DeviceInfo* d = nullptr;
+  AWQ_TRY(device_info(&d));
+  // one warp per row, grid-stride; 8 warps of a block and up to 8 blocks per SM resident at once
+  const int64_t rows_per_block = awq::kRowThreads / 32;
+  const int64_t blocks = std::min<int64_t>(static_cast<int64_t>(d->sms) * 8, (O + rows_per_block - 1) / rows_per_block);
+  awq::quantize_pack_int8_kernel<<<static_cast<unsigned>(blocks), awq::kRowThreads, 0,
+                                   reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(W), O, K, ldw, scales, (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0, codes, steps);
+  AWQ_TRY(check_launch("quantize_pack_int8_kernel"));
+  return ok();
 }
 
 }  // extern "C"

@@ -237,11 +237,13 @@ struct ProducerArgs {
   __nv_bfloat16* dW;               // [n_grid * O_pad][K]
   int exact;                       // AWQ_FLAG_EXACT_DIVISION
   int keep_w;                      // W is re-read once per candidate: ask L2 to keep it (evict_last)
+  const float* rowstep;            // INT8 per-channel quantizer: [n_grid][O_pad] steps, else null
 };
 
 // Weight errors of one row of one 512-in-feature segment for candidate j, from the row's raw bf16 words.
 __device__ __forceinline__ void produce_row(const ProducerArgs& a, const uint4 (&u)[2], const float (&s)[kProdCols],
-                                            const float (&rs)[kProdCols], bool real_row, uint32_t (&outw)[8]) {
+                                            const float (&rs)[kProdCols], bool real_row, float row_step,
+                                            uint32_t (&outw)[8]) {
   if (!real_row) {  // padding rows (o >= O) are zeros; warp-uniform
 #pragma unroll
     for (int i = 0; i < 8; ++i) outw[i] = 0u;
@@ -260,6 +262,21 @@ __device__ __forceinline__ void produce_row(const ProducerArgs& a, const uint4 (
     wp[i] = __fmul_rn(w[i], s[i]);
     mx = fmaxf(mx, wp[i]);
     mn = fminf(mn, wp[i]);
+  }
+  if (a.rowstep != nullptr) {  // INT8 per-channel: the row's step comes from the pre-pass
+    GroupParams g;
+    g.step = row_step;
+    g.zero = 0.0f;
+    g.rstep = __frcp_rn(row_step);
+#pragma unroll
+    for (int i = 0; i < kProdCols; i += 2) {
+      const float q0 = code_of_int8(wp[i], g, a.exact != 0), q1 = code_of_int8(wp[i + 1], g, a.exact != 0);
+      const float h0 = __fmul_rn(__fmul_rn(q0, g.step), rs[i]);
+      const float h1 = __fmul_rn(__fmul_rn(q1, g.step), rs[i + 1]);
+      const __nv_bfloat162 pr = __floats2bfloat162_rn(__fsub_rn(w[i], h0), __fsub_rn(w[i + 1], h1));
+      outw[i / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+    }
+    return;
   }
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) {
@@ -315,7 +332,8 @@ __device__ __forceinline__ unsigned int produce_rows(const ProducerArgs& a, int6
       nxt[1] = ldg_v4_policy(src + 1, pol);
     }
     uint32_t outw[8];
-    produce_row(a, cur, s, rs, o < a.O, outw);
+    const float row_step = a.rowstep != nullptr ? __ldg(a.rowstep + static_cast<int64_t>(j) * a.O_pad + o) : 0.0f;
+    produce_row(a, cur, s, rs, o < a.O, row_step, outw);
     if (active) {
       uint4* dst = reinterpret_cast<uint4*>(a.dW + (static_cast<int64_t>(j) * a.O_pad + o) * a.K + k0);
       dst[0] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
@@ -531,6 +549,84 @@ __global__ void __launch_bounds__(kFoldThreads) scale_fold_kernel(const uint16_t
       o[k] = *reinterpret_cast<const uint32_t*>(&pr);
     }
     *reinterpret_cast<uint4*>(out + r * ldo + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ===================================================================================================
+// INT8 per-channel quantizer: per-row steps of every candidate, and the INT8 pack.
+// ===================================================================================================
+constexpr int kRowThreads = 256;  // one warp per (candidate, row)
+
+// rowstep[j][o] = max(RN32(max_k |RN32(w[o,k] * s_j[k])| / 127), 1e-5); rows o >= O get 1.
+__global__ void __launch_bounds__(kRowThreads) int8_rowstep_kernel(const uint16_t* __restrict__ W, int64_t O,
+                                                                   int64_t O_pad, int64_t K, int64_t ldw,
+                                                                   const float* __restrict__ table,
+                                                                   float* __restrict__ rowstep) {
+  const int64_t o = (static_cast<int64_t>(blockIdx.x) * kRowThreads + threadIdx.x) >> 5;
+  const int j = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  if (o >= O_pad) return;
+  float amax = 0.0f;
+  if (o < O) {
+    const float* sj = table + static_cast<int64_t>(j) * K;
+    for (int64_t k0 = static_cast<int64_t>(lane) * 8; k0 < K; k0 += 256) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(W + o * ldw + k0));
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(sj + k0));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(sj + k0) + 1);
+      const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+      const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        amax = fmaxf(amax, fabsf(__fmul_rn(bf16_lo(uu[i]), ss[2 * i])));
+        amax = fmaxf(amax, fabsf(__fmul_rn(bf16_hi(uu[i]), ss[2 * i + 1])));
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if (lane == 0) rowstep[static_cast<int64_t>(j) * O_pad + o] = o < O ? int8_params(amax).step : 1.0f;
+}
+
+// One warp per row (grid-stride): the row's max |w'|, then its codes (int8) and step.
+__global__ void __launch_bounds__(kRowThreads) quantize_pack_int8_kernel(
+    const uint16_t* __restrict__ W, int64_t O, int64_t K, int64_t ldw, const float* __restrict__ scales, int exact,
+    int8_t* __restrict__ codes, float* __restrict__ steps) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * kRowThreads) >> 5;
+  for (int64_t o = (static_cast<int64_t>(blockIdx.x) * kRowThreads + threadIdx.x) >> 5; o < O; o += warps) {
+    float amax = 0.0f;
+    for (int64_t k0 = static_cast<int64_t>(lane) * 8; k0 < K; k0 += 256) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(W + o * ldw + k0));
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(scales + k0));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(scales + k0) + 1);
+      const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+      const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        amax = fmaxf(amax, fabsf(__fmul_rn(bf16_lo(uu[i]), ss[2 * i])));
+        amax = fmaxf(amax, fabsf(__fmul_rn(bf16_hi(uu[i]), ss[2 * i + 1])));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const GroupParams g = int8_params(amax);
+    for (int64_t k0 = static_cast<int64_t>(lane) * 8; k0 < K; k0 += 256) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(W + o * ldw + k0));
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(scales + k0));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(scales + k0) + 1);
+      const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+      const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q0 = static_cast<int>(code_of_int8(__fmul_rn(bf16_lo(uu[i]), ss[2 * i]), g, exact != 0));
+        const int q1 = static_cast<int>(code_of_int8(__fmul_rn(bf16_hi(uu[i]), ss[2 * i + 1]), g, exact != 0));
+        packed[i / 2] |= (static_cast<uint32_t>(q0) & 0xFFu) << (16 * (i & 1));
+        packed[i / 2] |= (static_cast<uint32_t>(q1) & 0xFFu) << (16 * (i & 1) + 8);
+      }
+      *reinterpret_cast<uint2*>(codes + o * K + k0) = make_uint2(packed[0], packed[1]);
+    }
+    if (lane == 0) steps[o] = g.step;
   }
 }
 

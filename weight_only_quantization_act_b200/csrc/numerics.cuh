@@ -194,15 +194,15 @@ __device__ __forceinline__ GroupParams group_params(float mx, float mn) {
 // below issues no division instructions.
 __device__ __noinline__ float rint_quotient_exact(float wp, float step) { return rintf(__fdiv_rn(wp, step)); }
 
-// rint(RN32(wp / step)) exactly. For |qa| < 64 the product qa = wp * RN32(1/step) is within
-// 1.5 * 2^-23 * 64 < 1.2e-5 of the real quotient, and RN32 moves the quotient by at most 2^-18, so the
-// two round to the same integer whenever qa is farther than 2^-14 from a half-integer. Only the rare
-// remaining cases (about one element in 10^4, and groups with the step at its floor) take the division.
+// rint(RN32(wp / step)) exactly. For |qa| < 128 the product qa = wp * RN32(1/step) is within
+// 1.5 * 2^-23 * 128 < 2.3e-5 of the real quotient, and RN32 moves the quotient by at most 2^-17, so the
+// two round to the same integer whenever qa is farther than 2^-14 (6.1e-5) from a half-integer. Only the
+// rare remaining cases (about one element in 10^4, and groups with the step at its floor) divide.
 __device__ __forceinline__ float rint_quotient(float wp, const GroupParams& g, bool exact) {
   const float qa = __fmul_rn(wp, g.rstep);
   float n = rintf(qa);
   const float d = fabsf(__fsub_rn(qa, n));  // exact: n is within a factor 2 of qa, or n = 0
-  if (exact || !(d < 0.5f - 0x1p-14f && fabsf(qa) < 64.0f)) n = rint_quotient_exact(wp, g.step);
+  if (exact || !(d < 0.5f - 0x1p-14f && fabsf(qa) < 128.0f)) n = rint_quotient_exact(wp, g.step);
   return n;
 }
 
@@ -210,6 +210,20 @@ __device__ __forceinline__ float rint_quotient(float wp, const GroupParams& g, b
 __device__ __forceinline__ float code_of(float wp, const GroupParams& g, bool exact) {
   const float q = __fadd_rn(rint_quotient(wp, g, exact), g.zero);
   return fminf(fmaxf(q, 0.0f), 15.0f);
+}
+
+// INT8 symmetric per-channel code q = min(max(rint(RN32(w'/step)), -127), 127) (g.zero is 0).
+__device__ __forceinline__ float code_of_int8(float wp, const GroupParams& g, bool exact) {
+  return fminf(fmaxf(rint_quotient(wp, g, exact), -127.0f), 127.0f);
+}
+
+// Per-channel INT8 parameters from the row's max |w'|: step = max(RN32(amax / 127), 1e-5), zero 0.
+__device__ __forceinline__ GroupParams int8_params(float amax) {
+  GroupParams g;
+  g.step = fmaxf(__fdiv_rn(amax, 127.0f), AWQ_STEP_FLOOR);
+  g.zero = 0.0f;
+  g.rstep = __frcp_rn(g.step);
+  return g;
 }
 
 // deq = RN32(RN32(q - z) * step)
