@@ -60,3 +60,51 @@ def test_deploy_path_end_to_end():
     mse = float(((Y - ref) ** 2).mean())
     best = float(out["losses"][int(out["best_j"].item())])
     assert 0.5 * best < mse < 1.25 * best, (mse, best)
+
+
+# ------------------------------------------------------------------------------------------------ few tokens
+# M <= 64 runs the decode kernel (weight rows on the MMA's M side, K split over a cluster of up to 8 CTAs,
+# partial sums reduced in distributed shared memory); the shapes cover cluster sizes 2, 4 and 8, CTAs of
+# a cluster left without k-blocks (K = 384, 640), ragged weight-row blocks and every token rounding.
+@pytest.mark.parametrize("M,K,O", [(1, 4096, 4096), (5, 384, 600), (16, 256, 136), (17, 1024, 520),
+                                   (33, 640, 264), (64, 2048, 1024), (64, 128, 8), (65, 512, 256)])
+def test_w4a16_few_tokens_match_oracle(M, K, O):
+    _, _, (words, steps, zeros) = quantized(O, K, 3 * M + K + O)
+    Xp = inputs.random_bf16((M, K), 11 * M + 5, scale=1.0)
+    Y = awq.w4a16_gemm(bf16_to_device(Xp), torch.from_numpy(words.view(np.int32)).cuda(),
+                       torch.from_numpy(steps).cuda(), torch.from_numpy(zeros).cuda())
+    torch.cuda.synchronize()
+    check_against_oracle(Xp, words, steps, zeros, Y)
+
+
+def test_w4a16_few_tokens_deterministic_and_strided():
+    _, _, (words, steps, zeros) = quantized(1024, 2048, 77)
+    wide = inputs.random_bf16((8, 2304), 78, scale=1.0)
+    Xd = bf16_to_device(wide)[:, 128:2176]  # row stride 2304
+    args = (torch.from_numpy(words.view(np.int32)).cuda(), torch.from_numpy(steps).cuda(),
+            torch.from_numpy(zeros).cuda())
+    a = awq.w4a16_gemm(Xd, *args)
+    b = awq.w4a16_gemm(Xd, *args)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b), "the cluster reduction adds the partial sums in a fixed order"
+    check_against_oracle(np.ascontiguousarray(wide[:, 128:2176]), words, steps, zeros, a)
+
+
+@pytest.mark.parametrize("M", [4, 300])
+def test_w4a16_huge_zero_points(M):
+    """Zero points beyond 2^19 (constant groups of large weights at the step floor) take the exact slow
+    dequantization path in both kernels."""
+    O, K = 256, 512
+    _, _, (words, steps, zeros) = quantized(O, K, 91)
+    steps, zeros = steps.copy(), zeros.copy()
+    steps[3, :] = F32(1e-5)
+    zeros[3, :] = F32(-3_000_000.0)
+    steps[40, 1] = F32(2.0 ** -17)
+    zeros[40, 1] = F32(9_999_999.0)
+    zeros[41, 2] = F32(-524_288.0)
+    zeros[42, 0] = F32(524_287.0)
+    Xp = inputs.random_bf16((M, K), 92 + M, scale=1.0)
+    Y = awq.w4a16_gemm(bf16_to_device(Xp), torch.from_numpy(words.view(np.int32)).cuda(),
+                       torch.from_numpy(steps).cuda(), torch.from_numpy(zeros).cuda())
+    torch.cuda.synchronize()
+    check_against_oracle(Xp, words, steps, zeros, Y)

@@ -21,7 +21,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libawq.so")
 SOURCES = ["awq_capi.cu"]
-HEADERS = ["ptx.cuh", "numerics.cuh", "kernels_simple.cuh", "kernel_loss_gemm.cuh", "kernel_w4a16.cuh"]
+HEADERS = ["ptx.cuh", "numerics.cuh", "kernels_simple.cuh", "kernel_loss_gemm.cuh", "kernel_w4a16.cuh",
+           "kernel_w4a16_decode.cuh", "dequant_w4.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

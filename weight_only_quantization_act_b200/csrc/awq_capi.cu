@@ -14,6 +14,7 @@
 #include "awq.h"
 #include "kernel_loss_gemm.cuh"
 #include "kernel_w4a16.cuh"
+#include "kernel_w4a16_decode.cuh"
 #include "kernels_simple.cuh"
 
 namespace {
@@ -90,6 +91,8 @@ awq_status device_info(DeviceInfo** out) {
     cfg.dynamicSmemBytes = awq::dq::SMEM_BYTES;
     AWQ_CUDA(cudaOccupancyMaxActiveClusters(&d.w4_clusters, awq::dq::w4a16_gemm_kernel, &cfg));
     if (d.w4_clusters < 1) return fail(AWQ_ERR_UNSUPPORTED, "the W4A16 GEMM does not fit on this device");
+    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::dec::smem_bytes(awq::dec::MAX_NT)));
     d.gemm_attr_set = true;
   }
   *out = &d;
@@ -656,17 +659,68 @@ extern "C" awq_status awq_scale_rows(const void* A, int64_t R, int64_t C, int64_
 
 namespace {
 struct W4Layout {
-  int64_t O_pad, G;
-  size_t steps_off, zeros_off, bytes;
+  int64_t O_pad, G, n_rb;
+  size_t steps_off, zeros_off, counter_off, partial_off, bytes;
 };
+// status (16 B) and tile counter at 0; group-major steps and zeros (many tokens); per-row-block counters
+// and split-K partial sums (few tokens).
 W4Layout w4_layout(int64_t K, int64_t O) {
   W4Layout l;
   l.O_pad = (O + awq::lg::BN - 1) / awq::lg::BN * awq::lg::BN;
   l.G = K / 128;
+  l.n_rb = (O + awq::dec::ROWS - 1) / awq::dec::ROWS;
   l.steps_off = 512;
   l.zeros_off = align_up(l.steps_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
-  l.bytes = align_up(l.zeros_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
+  l.counter_off = align_up(l.zeros_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
+  l.partial_off = align_up(l.counter_off + static_cast<size_t>(l.n_rb) * 4, 256);
+  l.bytes = align_up(l.partial_off + static_cast<size_t>(l.n_rb) * awq::dec::max_slices(l.n_rb) * awq::dec::MAX_NT *
+                                         awq::dec::ROWS * 4,
+                     256);
   return l;
+}
+
+// Few tokens: weight rows on the MMA's M side, k-blocks split into slices until every SM has a share,
+// slices added by the last CTA of each row block. A memset of the counters and one launch.
+awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const uint32_t* codes, const float* steps,
+                        const float* zeros, int64_t O, void* Y, int64_t ldy, void* workspace, const W4Layout& l,
+                        awq_stream_t stream) {
+  DeviceInfo* d = nullptr;
+  AWQ_TRY(device_info(&d));
+  const int nt = static_cast<int>((M + 15) / 16 * 16);
+  const int num_kb = static_cast<int>(K / awq::dec::BK);
+  int64_t slices = 2 * static_cast<int64_t>(d->sms) / l.n_rb;  // one wave at two CTAs per SM
+  slices = std::max<int64_t>(1, std::min<int64_t>({slices, awq::dec::max_slices(l.n_rb), num_kb}));
+  const int kb_per = static_cast<int>((num_kb + slices - 1) / slices);
+  slices = (num_kb + kb_per - 1) / kb_per;
+  if (l.n_rb * slices >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "O is too large");
+  CUtensorMap tmX, tmC;
+  AWQ_TRY(make_tmap(&tmX, X, M, K, ldx, nt));
+  AWQ_TRY(make_tmap_plain(&tmC, codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, O, K / 8, K / 8, awq::dec::BK / 8,
+                          awq::dec::ROWS));
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  awq::dec::Params p;
+  p.steps = steps;
+  p.zeros = zeros;
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.partial = reinterpret_cast<float*>(ws + l.partial_off);
+  p.counter = reinterpret_cast<unsigned int*>(ws + l.counter_off);
+  p.M = M;
+  p.O = O;
+  p.G = l.G;
+  p.ldy = ldy;
+  p.nt = nt;
+  p.num_kb = num_kb;
+  p.kb_per = kb_per;
+  p.slices = static_cast<int>(slices);
+  p.idesc = awq::idesc_bf16_f32(awq::dec::ROWS, static_cast<uint32_t>(nt));
+  p.status = reinterpret_cast<awq::DeviceStatus*>(ws);
+  p.limit_ns = g_wait_limit_ns.load();
+  AWQ_CUDA(cudaMemsetAsync(p.counter, 0, static_cast<size_t>(l.n_rb) * 4, st));
+  awq::dec::w4a16_decode_kernel<<<static_cast<unsigned>(l.n_rb * slices), awq::dec::THREADS,
+                                  awq::dec::smem_bytes(nt), st>>>(tmX, tmC, p);
+  AWQ_TRY(check_launch("w4a16_decode_kernel"));
+  return ok();
 }
 }  // namespace
 
@@ -688,8 +742,9 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, int64_t M, int64_t K, int64_
   if (workspace == nullptr || ws_bytes < l.bytes)
     return fail(AWQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", l.bytes, workspace ? ws_bytes : 0);
   if (!aligned16(workspace)) return fail(AWQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
-  const int64_t n_tiles_m = (M + awq::lg::BM - 1) / awq::lg::BM;
-  const int64_t n_bands = l.O_pad / awq::lg::BN;
+  if (M <= awq::dec::MAX_NT) return w4a16_decode(X, M, K, ldx, codes, steps, zeros, O, Y, ldy, workspace, l, stream);
+  const int64_t n_tiles_m = (M + awq::dq::TM - 1) / awq::dq::TM;
+  const int64_t n_bands = l.O_pad / awq::dq::BN;
   if (n_tiles_m * n_bands >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "too many tiles");
   DeviceInfo* d = nullptr;
   AWQ_TRY(device_info(&d));

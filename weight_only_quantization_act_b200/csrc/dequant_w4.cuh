@@ -1,0 +1,65 @@
+// dequant_w4.cuh - on-the-fly dequantization of packed 4-bit AWQ codes into a tensor-core operand tile
+// ("GPU 硬件级反量化算子内联融合" on the bjdmk.com.cn AWQ article: unpack with shifts and masks, convert,
+// apply the group's scale and offset). The value of code q in a group with step and zero point z is
+// bf16(RN32(RN32(q - z) * step)), exactly the weight the quantizer's dequantization gives, rounded once
+// to bf16 for the MMA.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace awq {
+
+// NW consecutive code words of one weight row (in-feature 8c+i at bits 4i..4i+3 of word c) -> 8 NW bf16
+// values, packed two per register in in-feature order (o[4c + j] holds in-features 8c+2j, 8c+2j+1).
+//
+// Fast path (|z| < 2^19, every zero point a quantizer produces for sane weights): byte j of a word holds
+// two codes; OR-ing the low nibble into the mantissa of 2^23 gives the float 2^23 + q exactly, OR-ing
+// the high nibble in place gives 2^23 + 16 q. Subtracting 2^23 + z (resp. 2^23 + 16 z), both exact
+// integers below 2^24, leaves q - z (resp. 16 (q - z)) exactly, and multiplying by step (resp. step / 16,
+// an exact power-of-two scaling) rounds the same real product once. One shift per byte instead of one
+// per code. Slow path (huge |z|): RN32(q - z) directly, as the quantizer defines it.
+template <int NW>
+__device__ __forceinline__ void dequant_words(const uint32_t (&w)[NW], float z, float stp, uint32_t (&o)[4 * NW]) {
+  if (fabsf(z) < 524288.0f) {
+    const float zb = __fadd_rn(8388608.0f, z);
+    const float zb16 = __fadd_rn(8388608.0f, __fmul_rn(16.0f, z));
+    const float st16 = __fmul_rn(stp, 0.0625f);
+#pragma unroll
+    for (int c = 0; c < NW; ++c)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t b = w[c] >> (8 * j);
+        const float lo = __uint_as_float((b & 0x0Fu) | 0x4B000000u);
+        const float hi = __uint_as_float((b & 0xF0u) | 0x4B000000u);
+        const __nv_bfloat162 pr =
+            __floats2bfloat162_rn(__fmul_rn(__fsub_rn(lo, zb), stp), __fmul_rn(__fsub_rn(hi, zb16), st16));
+        o[4 * c + j] = *reinterpret_cast<const uint32_t*>(&pr);
+      }
+  } else {
+#pragma unroll
+    for (int c = 0; c < NW; ++c)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float q0 = static_cast<float>((w[c] >> (8 * j)) & 0xFu);
+        const float q1 = static_cast<float>((w[c] >> (8 * j + 4)) & 0xFu);
+        const __nv_bfloat162 pr =
+            __floats2bfloat162_rn(__fmul_rn(__fsub_rn(q0, z), stp), __fmul_rn(__fsub_rn(q1, z), stp));
+        o[4 * c + j] = *reinterpret_cast<const uint32_t*>(&pr);
+      }
+  }
+}
+
+// The values of dequant_words for words c0 .. c0+NW-1 of a row's k-block of 64 in-features, stored into
+// the row's 128-byte line of a K-major tile with 128-byte swizzle: the 16-byte chunk of word c lands at
+// chunk c ^ (row & 7) of the line at `line_addr`.
+template <int NW>
+__device__ __forceinline__ void store_words_sw128(const uint32_t (&o)[4 * NW], uint32_t line_addr, int row, int c0) {
+  const uint32_t sw = static_cast<uint32_t>(row & 7);
+#pragma unroll
+  for (int c = 0; c < NW; ++c)
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(line_addr + ((static_cast<uint32_t>(c + c0) ^ sw) << 4)),
+                 "r"(o[4 * c]), "r"(o[4 * c + 1]), "r"(o[4 * c + 2]), "r"(o[4 * c + 3])
+                 : "memory");
+}
+
+}  // namespace awq

@@ -4,27 +4,31 @@
 // the group scale and offset, then fed to the tensor cores). X' is the layer input already divided by
 // the AWQ scales (folded into the previous operation); deq(W)[o, k] = bf16(RN32(RN32(q - z) * step)).
 //
-// Persistent cooperative kernel, clusters of 2 CTAs, one CTA per SM, 18 warps per CTA; tiles of 256
-// tokens x 256 output rows handed out dynamically through an 8-slot ring (as in the loss kernel):
-//   warp 0      TMA: X' tile [128 x 64] per stage for this CTA (128-byte swizzle; both CTAs' bytes are
-//               counted on the even CTA's barrier), and the stage's code words [128 rows x 8 words]
-//               plus the group steps and zeros of those rows (from a group-major copy) into this CTA's
-//               shared memory, counted on a barrier of this CTA
-//   warp 1      pair-wide tensor memory (two 256-column fp32 accumulators); the even CTA issues the pair
-//               MMAs (tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16)
-//   warps 2-5   epilogue: fp32 accumulator -> bf16, stored to Y (each lane one row, 64-byte pieces)
-//   warps 6-17  dequantizers, two per pipeline stage: warps 6+s and 12+s fill every use of stage s with
-//               the CTA's 128 weight rows x 64 in-features from the staged codes, in the 128-byte swizzled
-//               K-major layout the MMA descriptor expects (64 rows each), then one proxy fence and one
-//               arrive on the even CTA's full barrier. Owning whole stages lets the six stages fill
-//               concurrently and pays the fence once per 8 KB; the warps issue no global loads (the
-//               fence would wait for them too).
+// Persistent cooperative kernel, clusters of 2 CTAs, one CTA per SM. A tile is 512 tokens x 256 output
+// rows: one dequantized weight tile (each CTA stages 128 of the 256 rows) feeds two pair MMAs, one per
+// 256-token half, so every dequantized weight is used by 512 tokens. Tiles are handed out dynamically
+// through an 8-slot ring (as in the loss kernel), published one tile ahead so the code loads can run
+// into the next tile. Warps:
+//   0      TMA: both 256-token halves of X' for this CTA's 128 rows of each (128 x 64 per half and stage,
+//          128-byte swizzle; both CTAs' bytes counted on the even CTA's barrier)
+//   1      pair-wide tensor memory (two 256-column fp32 accumulators, one per token half); the even CTA
+//          issues the pair MMAs (tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16)
+//   2-5    epilogue: both accumulators -> bf16 -> Y (each lane one token row, 64-byte pieces)
+//   6      TMA of the code words [128 rows x 8 words], steps and zero points (from a group-major copy) of
+//          every k-block into a ring of its own, so they are resident before the operand stage frees up
+//   7-14   dequantizers, two per operand stage: warps 7+s and 11+s fill every use of stage s with 64 of the
+//          CTA's 128 weight rows x 64 in-features, in the 128-byte swizzled K-major layout the MMA
+//          descriptor expects, then one proxy fence and one arrive on the even CTA's full barrier. The
+//          values are computed in registers as soon as the codes are in, and only stored once the stage
+//          is free, so the arithmetic stays off the MMA's critical path. They issue no global loads (the
+//          fence would wait for them too).
 // Every wait is bounded.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "dequant_w4.cuh"
 #include "kernel_loss_gemm.cuh"
 #include "ptx.cuh"
 
@@ -32,31 +36,35 @@ namespace awq {
 namespace dq {
 
 using lg::BK;
-using lg::BM;
-using lg::BN;
 using lg::HALF;
-using lg::NUM_ACC;
 using lg::RING;
-using lg::TMEM_COLS;
 using lg::UK;
 
-constexpr int STAGES = 6;
-constexpr int A_BYTES = HALF * BK * 2;            // 16 KB  X' rows
+constexpr int TM = 512;                           // tokens per tile (two pair MMAs of M = 256)
+constexpr int BMH = 256;                          // tokens per MMA
+constexpr int BN = 256;                           // weight rows per tile (MMA N; 128 staged per CTA)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = HALF * BK * 2;            // 16 KB  X' rows of one token half
 constexpr int B_BYTES = HALF * BK * 2;            // 16 KB  dequantized weight rows
+constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
+constexpr int CSTAGES = 6;                        // code ring
 constexpr int C_BYTES = HALF * (BK / 8) * 4;      // 4 KB   code words of those rows
 constexpr int S_BYTES = HALF * 4;                 // 512 B  step of each row (this k-block's group)
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES + 2 * S_BYTES;  // 37 KB per CTA
+constexpr int CSTAGE_BYTES = C_BYTES + 2 * S_BYTES;
 constexpr int DQ_PER_STAGE = 2;                   // dequantizer warps per stage (each half the rows)
 constexpr int DQ_WARPS = STAGES * DQ_PER_STAGE;
-constexpr int THREADS = 192 + 32 * DQ_WARPS;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+constexpr int THREADS = 224 + 32 * DQ_WARPS;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CSTAGES * CSTAGE_BYTES + 1024;
+constexpr uint32_t TMEM_COLS = 512;
 constexpr int BANDS_PER_GROUP = 8;                // raster: 8 weight bands advance together over X'
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+constexpr uint32_t IDESC = idesc_bf16_f32(BMH, BN);
+static_assert(SMEM_BYTES <= 232448, "fits the 227 KB of dynamic shared memory");
+static_assert(STAGE_BYTES % 1024 == 0 && CSTAGE_BYTES % 1024 == 0, "tiles stay 1024-byte aligned");
 
 struct Params {
   __nv_bfloat16* Y;        // [M][ldy]
   int64_t M, O, K, ldy;
-  int n_tiles_m;           // ceil(M / 256)
+  int n_tiles_m;           // ceil(M / 512)
   int n_bands;             // ceil(O / 256)
   int num_kb;              // K / 64
   int num_tiles;
@@ -115,7 +123,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                       const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[3 * STAGES + 2 * NUM_ACC + 1 + RING];
+  __shared__ __align__(8) uint64_t bars[2 * STAGES + 2 * CSTAGES + 3 + RING];
   __shared__ uint32_t tmem_slot;
   __shared__ int tile_ring[RING];
 
@@ -123,32 +131,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const uint32_t bar0 = smem_u32(&bars[0]);
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
-  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + NUM_ACC + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * NUM_ACC);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };                               // even CTA: X' + B ready
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };                   // MMAs done with stage
+  auto cfull_bar = [&](int c) { return bar0 + 8u * (2 * STAGES + c); };               // codes landed
+  auto cempty_bar = [&](int c) { return bar0 + 8u * (2 * STAGES + CSTAGES + c); };    // codes read
+  const uint32_t accf_bar = bar0 + 8u * (2 * STAGES + 2 * CSTAGES);                   // tile accumulated
+  const uint32_t acce_bar = accf_bar + 8u;                                            // accumulators read
+  const uint32_t drain_bar = accf_bar + 16u;
   auto tile_bar = [&](int slot) { return drain_bar + 8u + 8u * slot; };
-  auto cfull_bar = [&](int s) { return drain_bar + 8u + 8u * RING + 8u * s; };
   const uint32_t smem_base = smem_u32(smem);
-  auto a_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s) * STAGE_BYTES; };
-  auto b_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s) * STAGE_BYTES + A_BYTES; };
-  auto c_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s) * STAGE_BYTES + A_BYTES + B_BYTES; };
-  auto s_tile = [&](int s) { return c_tile(s) + C_BYTES; };
-  auto z_tile = [&](int s) { return c_tile(s) + C_BYTES + S_BYTES; };
+  auto a_tile = [&](int s, int h) { return smem_base + static_cast<uint32_t>(s * STAGE_BYTES + h * A_BYTES); };
+  auto b_tile = [&](int s) { return smem_base + static_cast<uint32_t>(s * STAGE_BYTES + 2 * A_BYTES); };
+  auto c_tile = [&](int c) { return smem_base + static_cast<uint32_t>(STAGES * STAGE_BYTES + c * CSTAGE_BYTES); };
+  auto s_tile = [&](int c) { return c_tile(c) + C_BYTES; };
+  auto z_tile = [&](int c) { return c_tile(c) + C_BYTES + S_BYTES; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1 + 2 * DQ_PER_STAGE);  // TMA arm + the stage's dequantizer warps of both CTAs
       mbar_init(empty_bar(s), 1);
     }
-    for (int a = 0; a < NUM_ACC; ++a) {
-      mbar_init(accf_bar(a), 1);
-      mbar_init(acce_bar(a), 8);
+    for (int c = 0; c < CSTAGES; ++c) {
+      mbar_init(cfull_bar(c), 1);                    // this CTA's code loader arms it
+      mbar_init(cempty_bar(c), DQ_PER_STAGE);        // the dequantizer warps that read the slot
     }
+    mbar_init(accf_bar, 1);
+    mbar_init(acce_bar, 8);                          // 4 epilogue warps x 2 CTAs
     mbar_init(drain_bar, 1);
     for (int r = 0; r < RING; ++r) mbar_init(tile_bar(r), 1);
-    for (int st2 = 0; st2 < STAGES; ++st2) mbar_init(cfull_bar(st2), 1);  // this CTA's TMA thread arms it
     fence_barrier_init();
     fence_proxy_async_smem();
   }
@@ -197,16 +207,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       const uint64_t pol_x = policy_evict_normal();
+      // The even CTA publishes tile i + 1 when it starts tile i (tile 0 first), so the code loaders can
+      // run into the next tile; -1 ends the sequence.
+      auto publish = [&](int i) -> int {
+        int t = i == 0 ? pair : n_pairs + static_cast<int>(atomicAdd(p.tile_counter, 1u));
+        if (t >= p.num_tiles) t = -1;
+        const int slot = i % RING;
+        tile_ring[slot] = t;
+        st_shared_cluster_u32(map_to_rank(smem_u32(&tile_ring[slot]), 1), static_cast<uint32_t>(t));
+        mbar_arrive(tile_bar(slot));
+        mbar_arrive_remote(map_to_rank(tile_bar(slot), 1));
+        return t;
+      };
+      int next = rank == 0 ? publish(0) : 0;
       for (int i = 0; ok; ++i) {
         int t;
         if (rank == 0) {
-          t = i == 0 ? pair : n_pairs + static_cast<int>(atomicAdd(p.tile_counter, 1u));
-          if (t >= p.num_tiles) t = -1;
-          const int slot = i % RING;
-          tile_ring[slot] = t;
-          st_shared_cluster_u32(map_to_rank(smem_u32(&tile_ring[slot]), 1), static_cast<uint32_t>(t));
-          mbar_arrive(tile_bar(slot));
-          mbar_arrive_remote(map_to_rank(tile_bar(slot), 1));
+          t = next;
+          if (t >= 0) next = publish(i + 1);
         } else {
           t = ring_wait_thread(i, ok);
           if (!ok) break;
@@ -214,20 +232,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (t < 0) break;
         int band, mt;
         tile_coords(t, p, band, mt);
-        const int32_t a_row = mt * BM + static_cast<int32_t>(rank) * HALF;
-        const int32_t w_row = band * BN + static_cast<int32_t>(rank) * HALF;
+        const int32_t a_row = mt * TM + static_cast<int32_t>(rank) * HALF;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, st, p.limit_ns, kSiteTmaEmpty)) {
             ok = false;
             break;
           }
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
-          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * A_BYTES);
-          tma_load_2d_pair_hint(a_tile(stage), &tmX, kb * BK, a_row, fb, pol_x);
-          mbar_arrive_expect_tx(cfull_bar(stage), C_BYTES + 2 * S_BYTES);
-          tma_load_2d(c_tile(stage), &tmC, kb * (BK / 8), w_row, cfull_bar(stage));
-          tma_load_2d(s_tile(stage), &tmS, w_row, (kb * BK) >> 7, cfull_bar(stage));
-          tma_load_2d(z_tile(stage), &tmZ, w_row, (kb * BK) >> 7, cfull_bar(stage));
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 4 * A_BYTES);
+          tma_load_2d_pair_hint(a_tile(stage, 0), &tmX, kb * BK, a_row, fb, pol_x);
+          tma_load_2d_pair_hint(a_tile(stage, 1), &tmX, kb * BK, a_row + BMH, fb, pol_x);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -245,25 +259,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       for (int i = 0; ok; ++i) {
         const int t = ring_wait_thread(i, ok);
         if (!ok || t < 0) break;
-        const int acc = i & 1;
-        const uint32_t acc_phase = static_cast<uint32_t>(i >> 1) & 1u;
-        if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, st, p.limit_ns, kSiteMmaAccEmpty)) {
+        if (i > 0 && !mbar_wait(acce_bar, static_cast<uint32_t>(i - 1) & 1u, st, p.limit_ns, kSiteMmaAccEmpty)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, st, p.limit_ns, kSiteMmaFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = a_tile(stage), b0 = b_tile(stage);
+          const uint32_t b0 = b_tile(stage);
 #pragma unroll
-          for (int kk = 0; kk < BK / UK; ++kk)
-            umma_bf16_pair(d_tmem, smem_desc_sw128(a0 + kk * UK * 2), smem_desc_sw128(b0 + kk * UK * 2), IDESC,
-                           (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / UK; ++kk) {
+            const uint64_t bd = smem_desc_sw128(b0 + kk * UK * 2);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            umma_bf16_pair(tmem_base, smem_desc_sw128(a_tile(stage, 0) + kk * UK * 2), bd, IDESC, acc);
+            umma_bf16_pair(tmem_base + BN, smem_desc_sw128(a_tile(stage, 1) + kk * UK * 2), bd, IDESC, acc);
+          }
           umma_commit_pair(empty_bar(stage), 0x3);
           if (++stage == STAGES) {
             stage = 0;
@@ -271,7 +285,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
         }
         if (!ok) break;
-        umma_commit_pair(accf_bar(acc), 0x3);
+        umma_commit_pair(accf_bar, 0x3);
       }
       umma_commit_pair(drain_bar, 0x1);
       const uint64_t t0 = global_timer_ns();
@@ -282,14 +296,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
     }
     __syncwarp();
-  } else if (warp >= 6) {
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------------------ TMA (codes)
+    if (elect_one()) {
+      bool ok = true;
+      int slot = 0;
+      uint32_t phase = 0;
+      for (int i = 0; ok; ++i) {
+        const int t = ring_wait_thread(i, ok);
+        if (!ok || t < 0) break;
+        int band, mt;
+        tile_coords(t, p, band, mt);
+        const int32_t w_row = band * BN + static_cast<int32_t>(rank) * HALF;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(cempty_bar(slot), phase ^ 1u, st, p.limit_ns, kSiteTmaProduced)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(cfull_bar(slot), CSTAGE_BYTES);
+          tma_load_2d(c_tile(slot), &tmC, kb * (BK / 8), w_row, cfull_bar(slot));
+          tma_load_2d(s_tile(slot), &tmS, w_row, (kb * BK) >> 7, cfull_bar(slot));
+          tma_load_2d(z_tile(slot), &tmZ, w_row, (kb * BK) >> 7, cfull_bar(slot));
+          if (++slot == CSTAGES) {
+            slot = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 7) {
     // ------------------------------------------------------------------------------ dequantizers
-    // Warp 6+s owns stage s: the pipeline's k-blocks are numbered continuously over this pair's tiles
-    // (tile i, k-block kb -> i * num_kb + kb), and stage s carries the numbers congruent to s mod STAGES.
-    const int s_own = (warp - 6) % STAGES;
-    const int part = (warp - 6) / STAGES;  // which HALF / DQ_PER_STAGE rows of the stage this warp fills
+    // K-blocks are numbered continuously over this pair's tiles (tile i, k-block kb -> g = i * num_kb + kb);
+    // operand stage g % STAGES, code slot g % CSTAGES. Warps 7+s and 11+s own stage s.
+    const int s_own = (warp - 7) % STAGES;
+    const int part = (warp - 7) / STAGES;  // which HALF / DQ_PER_STAGE rows of the stage this warp fills
+    constexpr int RR = HALF / 32 / DQ_PER_STAGE;
     bool ok = true;
-    int known_tile = -1;  // tiles < known_tile + 1 exist (the ring told us)
+    int known_tile = -1;
     for (int64_t g = s_own, use = 0; ok; g += STAGES, ++use) {
       const int i = static_cast<int>(g / p.num_kb);
       if (i > known_tile) {
@@ -297,44 +341,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (!ok || t < 0) break;
         known_tile = i;
       }
-      if (!warp_wait_any(cfull_bar(s_own), static_cast<uint32_t>(use) & 1u, st, p.limit_ns, kSiteTmaEmpty, false)) {
+      const int cs = static_cast<int>(g % CSTAGES);
+      if (!warp_wait_any(cfull_bar(cs), static_cast<uint32_t>(g / CSTAGES) & 1u, st, p.limit_ns, kSiteTmaEmpty,
+                         false)) {
         ok = false;
         break;
       }
-      const uint32_t cbase = c_tile(s_own), bbase = b_tile(s_own);
-#pragma unroll 1
-      for (int rr = 0; rr < HALF / 32 / DQ_PER_STAGE; ++rr) {
-        const int r = lane + 32 * (rr + part * (HALF / 32 / DQ_PER_STAGE));
-        uint32_t w[8];
-        float z, stp;
+      const uint32_t cbase = c_tile(cs), bbase = b_tile(s_own);
+      uint32_t w[RR][8];
+      float z[RR], stp[RR];
+#pragma unroll
+      for (int rr = 0; rr < RR; ++rr) {
+        const int r = lane + 32 * (rr + part * RR);
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "=r"(w[rr][0]), "=r"(w[rr][1]), "=r"(w[rr][2]), "=r"(w[rr][3])
                      : "r"(cbase + static_cast<uint32_t>(r * 32)));
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                     : "=r"(w[rr][4]), "=r"(w[rr][5]), "=r"(w[rr][6]), "=r"(w[rr][7])
                      : "r"(cbase + static_cast<uint32_t>(r * 32 + 16)));
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(stp) : "r"(s_tile(s_own) + static_cast<uint32_t>(r * 4)));
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(z) : "r"(z_tile(s_own) + static_cast<uint32_t>(r * 4)));
-        // (2^23 + q) - (2^23 + z) = q - z exactly; then one fp32 rounding for the step, one for bf16.
-        // Rows past O arrive as zero codes with zero step and zero: they dequantize to 0.
-        const float zb = __fadd_rn(8388608.0f, z);
-        const uint32_t row_base = bbase + static_cast<uint32_t>(r) * 128u;
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(stp[rr]) : "r"(s_tile(cs) + static_cast<uint32_t>(r * 4)));
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(z[rr]) : "r"(z_tile(cs) + static_cast<uint32_t>(r * 4)));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(cempty_bar(cs));  // the code slot may be refilled
+      // Dequantize into registers while the operand stage may still be in use (rows past O arrive as
+      // zero codes with zero step and zero: they dequantize to 0) ...
+      uint32_t v[RR][32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {  // code word c = in-features 8c..8c+7 = 16-byte chunk c of the row
-          uint32_t o4[4];
+      for (int rr = 0; rr < RR; ++rr) dequant_words<8>(w[rr], z[rr], stp[rr], v[rr]);
+      // ... and store once the MMAs of its previous use have completed.
+      if (use > 0 && !warp_wait_any(empty_bar(s_own), static_cast<uint32_t>(use - 1) & 1u, st, p.limit_ns,
+                                    kSiteMmaFull, true)) {
+        ok = false;
+        break;
+      }
 #pragma unroll
-          for (int n = 0; n < 8; n += 2) {
-            const float q0 = __uint_as_float(0x4B000000u | ((w[c] >> (4 * n)) & 0xFu));
-            const float q1 = __uint_as_float(0x4B000000u | ((w[c] >> (4 * n + 4)) & 0xFu));
-            const __nv_bfloat162 pr = __floats2bfloat162_rn(__fmul_rn(__fsub_rn(q0, zb), stp),
-                                                            __fmul_rn(__fsub_rn(q1, zb), stp));
-            o4[n / 2] = *reinterpret_cast<const uint32_t*>(&pr);
-          }
-          const uint32_t chunk = static_cast<uint32_t>(c) ^ static_cast<uint32_t>(r & 7);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row_base + (chunk << 4)), "r"(o4[0]),
-                       "r"(o4[1]), "r"(o4[2]), "r"(o4[3])
-                       : "memory");
-        }
+      for (int rr = 0; rr < RR; ++rr) {
+        const int r = lane + 32 * (rr + part * RR);
+        store_words_sw128<8>(v[rr], bbase + static_cast<uint32_t>(r) * 128u, r, 0);
       }
       fence_proxy_async_smem();  // the tensor cores read these bytes through the async proxy
       __syncwarp();
@@ -347,38 +391,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int i = 0; ok; ++i) {
       const int t = ring_wait_warp(i, ok);
       if (!ok || t < 0) break;
-      const int acc = i & 1;
-      const uint32_t acc_phase = static_cast<uint32_t>(i >> 1) & 1u;
-      if (!warp_wait_any(accf_bar(acc), acc_phase, st, p.limit_ns, kSiteEpiAccFull, false)) break;
+      if (!warp_wait_any(accf_bar, static_cast<uint32_t>(i) & 1u, st, p.limit_ns, kSiteEpiAccFull, false)) break;
       tc_fence_after();
       int band, mt;
       tile_coords(t, p, band, mt);
-      const int64_t row = static_cast<int64_t>(mt) * BM + static_cast<int64_t>(rank) * HALF + quarter * 32 + lane;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
-        const int64_t col0 = static_cast<int64_t>(band) * BN + c * 32;
-        if (row < p.M && col0 < p.O) {
-          uint32_t packed[16];
+      for (int h = 0; h < 2; ++h) {
+        const int64_t row = static_cast<int64_t>(mt) * TM + h * BMH + static_cast<int64_t>(rank) * HALF +
+                            quarter * 32 + lane;
+        const uint32_t taddr =
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(h * BN);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
+          const int64_t col0 = static_cast<int64_t>(band) * BN + c * 32;
+          if (row < p.M && col0 < p.O) {
+            uint32_t packed[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const __nv_bfloat162 pr = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-            packed[k] = *reinterpret_cast<const uint32_t*>(&pr);
+            for (int k = 0; k < 16; ++k) {
+              const __nv_bfloat162 pr = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+              packed[k] = *reinterpret_cast<const uint32_t*>(&pr);
+            }
+            __nv_bfloat16* dst = p.Y + row * p.ldy + col0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (col0 + 8 * q < p.O)  // O % 8 == 0: 16-byte pieces are all in or all out
+                *reinterpret_cast<uint4*>(dst + 8 * q) =
+                    make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
           }
-          __nv_bfloat16* dst = p.Y + row * p.ldy + col0;
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (col0 + 8 * q < p.O)  // O % 8 == 0: 16-byte pieces are all in or all out
-              *reinterpret_cast<uint4*>(dst + 8 * q) =
-                  make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(map_to_rank(acce_bar(acc), 0));
+      if (lane == 0) mbar_arrive_remote(map_to_rank(acce_bar, 0));
     }
   }
 
