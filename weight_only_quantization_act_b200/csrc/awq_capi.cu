@@ -145,6 +145,21 @@ awq_status make_tmap_plain(CUtensorMap* map, const void* base, CUtensorMapDataTy
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Code words [rows][cols] (uint32) in boxes of 32 words x box_rows with 128-byte swizzle.
+awq_status make_tmap_codes_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+  cuuint32_t box[2] = {32u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return AWQ_OK;
+}
+
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ----------------------------------------------------------------------------- workspace layouts
@@ -690,13 +705,13 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   const int num_kb = static_cast<int>(K / awq::dec::BK);
   int64_t slices = 2 * static_cast<int64_t>(d->sms) / l.n_rb;  // one wave at two CTAs per SM
   slices = std::max<int64_t>(1, std::min<int64_t>({slices, awq::dec::max_slices(l.n_rb), num_kb}));
-  const int kb_per = static_cast<int>((num_kb + slices - 1) / slices);
+  const int kb_box = awq::dec::KB_PER_BOX;
+  const int kb_per = static_cast<int>(((num_kb + slices - 1) / slices + kb_box - 1) / kb_box * kb_box);
   slices = (num_kb + kb_per - 1) / kb_per;
   if (l.n_rb * slices >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "O is too large");
   CUtensorMap tmX, tmC;
   AWQ_TRY(make_tmap(&tmX, X, M, K, ldx, nt));
-  AWQ_TRY(make_tmap_plain(&tmC, codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, O, K / 8, K / 8, awq::dec::BK / 8,
-                          awq::dec::ROWS));
+  AWQ_TRY(make_tmap_codes_sw128(&tmC, codes, O, K / 8, awq::dec::ROWS));
   char* ws = static_cast<char*>(workspace);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   awq::dec::Params p;
@@ -713,6 +728,10 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   p.num_kb = num_kb;
   p.kb_per = kb_per;
   p.slices = static_cast<int>(slices);
+  p.sz_pairs = (l.G % 2 == 0 && (reinterpret_cast<uintptr_t>(steps) & 7u) == 0 &&
+                (reinterpret_cast<uintptr_t>(zeros) & 7u) == 0)
+                   ? 1
+                   : 0;
   p.idesc = awq::idesc_bf16_f32(awq::dec::ROWS, static_cast<uint32_t>(nt));
   p.status = reinterpret_cast<awq::DeviceStatus*>(ws);
   p.limit_ns = g_wait_limit_ns.load();

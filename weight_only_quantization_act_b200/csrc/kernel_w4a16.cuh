@@ -47,7 +47,7 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = HALF * BK * 2;            // 16 KB  X' rows of one token half
 constexpr int B_BYTES = HALF * BK * 2;            // 16 KB  dequantized weight rows
 constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
-constexpr int CSTAGES = 6;                        // code ring
+constexpr int CSTAGES = 4;                        // code ring
 constexpr int C_BYTES = HALF * (BK / 8) * 4;      // 4 KB   code words of those rows
 constexpr int S_BYTES = HALF * 4;                 // 512 B  step of each row (this k-block's group)
 constexpr int CSTAGE_BYTES = C_BYTES + 2 * S_BYTES;
@@ -60,6 +60,12 @@ constexpr int BANDS_PER_GROUP = 8;                // raster: 8 weight bands adva
 constexpr uint32_t IDESC = idesc_bf16_f32(BMH, BN);
 static_assert(SMEM_BYTES <= 232448, "fits the 227 KB of dynamic shared memory");
 static_assert(STAGE_BYTES % 1024 == 0 && CSTAGE_BYTES % 1024 == 0, "tiles stay 1024-byte aligned");
+// A parity wait only tells the phase apart from its neighbours: a waiter must see every phase of the
+// barrier it waits on. With CSTAGES a multiple of STAGES, code slot c is always read by the warps of
+// operand stage c % STAGES, so they wait on each of its phases in turn (any other ratio lets a warp wait
+// for fill n+2 of a slot while fill n+1, read by another stage's warps, has not landed yet, and the
+// parity of fill n would pass it).
+static_assert(CSTAGES % STAGES == 0, "each code slot is read by one stage's warps");
 
 struct Params {
   __nv_bfloat16* Y;        // [M][ldy]
@@ -352,23 +358,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       float z[RR], stp[RR];
 #pragma unroll
       for (int rr = 0; rr < RR; ++rr) {
+        // "memory" keeps these loads ahead of the barrier arrive below that hands the slot back.
         const int r = lane + 32 * (rr + part * RR);
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(w[rr][0]), "=r"(w[rr][1]), "=r"(w[rr][2]), "=r"(w[rr][3])
-                     : "r"(cbase + static_cast<uint32_t>(r * 32)));
+                     : "r"(cbase + static_cast<uint32_t>(r * 32))
+                     : "memory");
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(w[rr][4]), "=r"(w[rr][5]), "=r"(w[rr][6]), "=r"(w[rr][7])
-                     : "r"(cbase + static_cast<uint32_t>(r * 32 + 16)));
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(stp[rr]) : "r"(s_tile(cs) + static_cast<uint32_t>(r * 4)));
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(z[rr]) : "r"(z_tile(cs) + static_cast<uint32_t>(r * 4)));
+                     : "r"(cbase + static_cast<uint32_t>(r * 32 + 16))
+                     : "memory");
+        asm volatile("ld.shared.f32 %0, [%1];"
+                     : "=f"(stp[rr])
+                     : "r"(s_tile(cs) + static_cast<uint32_t>(r * 4))
+                     : "memory");
+        asm volatile("ld.shared.f32 %0, [%1];"
+                     : "=f"(z[rr])
+                     : "r"(z_tile(cs) + static_cast<uint32_t>(r * 4))
+                     : "memory");
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(cempty_bar(cs));  // the code slot may be refilled
       // Dequantize into registers while the operand stage may still be in use (rows past O arrive as
-      // zero codes with zero step and zero: they dequantize to 0) ...
+      // zero codes with zero step and zero: they dequantize to 0); the code slot goes back once the
+      // values are computed ...
       uint32_t v[RR][32];
 #pragma unroll
       for (int rr = 0; rr < RR; ++rr) dequant_words<8>(w[rr], z[rr], stp[rr], v[rr]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(cempty_bar(cs));
       // ... and store once the MMAs of its previous use have completed.
       if (use > 0 && !warp_wait_any(empty_bar(s_own), static_cast<uint32_t>(use - 1) & 1u, st, p.limit_ns,
                                     kSiteMmaFull, true)) {

@@ -3,19 +3,22 @@
 // packed weights, so the weight rows take the MMA's M side and the k-blocks are split until every SM has
 // a share:
 //
-//   CTA (b, c) covers weight rows [128 b, 128 b + 128) and k-blocks [c * kb_per, (c + 1) * kb_per);
-//   D[128 rows][nt tokens] accumulates in tensor memory (tcgen05.mma cta_group::1, kind::f16, M = 128,
-//   N = nt = tokens rounded up to 16, K = 16) and is written to the workspace as slice c of row block b;
-//   the last CTA of a row block to finish (a per-block counter) adds the S slices in slice order
-//   (deterministic), converts to bf16 and writes Y.
+//   CTA (b, c) covers weight rows [128 b, 128 b + 128) and k-blocks [c * kb_per, (c + 1) * kb_per)
+//   (kb_per a multiple of 4); D[128 rows][nt tokens] accumulates in tensor memory (tcgen05.mma
+//   cta_group::1, kind::f16, M = 128, N = nt = tokens rounded up to 16, K = 16) and is written to the
+//   workspace as slice c of row block b; the last CTA of a row block to finish (a per-block counter) adds
+//   the S slices in slice order (deterministic), converts to bf16 and writes Y.
 //
-// Warps: 0 loads into an 8-deep input ring (lane 0: TMA of the k-block's code words [128 rows x 8 words]
-// and X' tile [nt x 64], 128-byte swizzle; all lanes: cp.async of the rows' steps and zero points straight
-// from the [O][K/128] arrays), so a CTA's first 8 k-blocks are requested at once; 1 allocates tensor memory
+// The loads are few and large, since scattered small requests are what limits this size: the code words
+// of 4 k-blocks come as one TMA box [128 rows x 32 words] with 128-byte swizzle (128 contiguous bytes per
+// row), with the two groups' steps and zero points of those rows (8-byte cp.async per row and array); X'
+// comes per k-block [nt x 64] (128-byte swizzle) through a ring of its own.
+//
+// Warps: 0 loads (lane 0 the TMA boxes; all lanes the steps and zero points); 1 allocates tensor memory
 // and issues the MMAs; 2-9 dequantize into a 3-deep ring of K-major swizzled operand tiles (warp 2 + q + 4h
-// takes rows 32q..32q+31, in-features 32h..32h+31 of the k-block; then proxy fence, arrive); warps 2-5 then
-// read the accumulator (warp w may read tensor-memory lanes 32 (w % 4) ...). All waits are bounded; a
-// timeout is recorded in the caller's status word.
+// takes rows 32q..32q+31, in-features 32h..32h+31 of the k-block), computing in registers first and
+// storing once the tile is free; warps 2-5 then read the accumulator (warp w may read tensor-memory lanes
+// 32 (w % 4) ...). All waits are bounded; a timeout is recorded in the caller's status word.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -31,22 +34,26 @@ constexpr int ROWS = 128;                     // weight rows per CTA (the MMA's 
 constexpr int BK = 64;                        // in-features per k-block
 constexpr int UK = 16;                        // K of one MMA
 constexpr int MAX_NT = 64;                    // tokens per launch (the MMA's N, a multiple of 16)
-constexpr int IN_STAGES = 8;                  // k-blocks of inputs in flight (codes, X', steps, zeros)
+constexpr int KB_PER_BOX = 4;                 // k-blocks per code box (32 words = 128 bytes per row)
+constexpr int C_STAGES = 2;                   // code boxes in flight
+constexpr int C_BYTES = ROWS * 128;           // 16 KB code words
+constexpr int SZ_BYTES = 2 * 2 * ROWS * 4;    // 2 KB steps and zero points of the box's two groups
+constexpr int C_STAGE_BYTES = C_BYTES + SZ_BYTES;
+constexpr int X_STAGES = 8;                   // X' k-blocks in flight
 constexpr int A_STAGES = 3;                   // dequantized operand tiles
 constexpr int A_BYTES = ROWS * BK * 2;        // 16 KB dequantized weight rows
-constexpr int C_BYTES = ROWS * (BK / 8) * 4;  // 4 KB code words
-constexpr int SZ_BYTES = ROWS * 4;            // 512 B steps (as much again for the zero points)
 constexpr int DQ_WARPS = 8;
 constexpr int THREADS = 64 + 32 * DQ_WARPS;
 constexpr int TMEM_COLS = 64;                 // >= MAX_NT, a power of two >= 32
 constexpr int MAX_SLICES = 16;
 
-// Input stage: X' tile [nt x 64] (128-byte swizzle) first, then code words, steps, zero points.
-__host__ __device__ constexpr int in_stage_bytes(int nt) { return nt * BK * 2 + C_BYTES + 2 * SZ_BYTES; }
+__host__ __device__ constexpr int x_stage_bytes(int nt) { return nt * BK * 2; }
 __host__ __device__ constexpr int smem_bytes(int nt) {
-  return A_STAGES * A_BYTES + IN_STAGES * in_stage_bytes(nt) + 1024;
+  return C_STAGES * C_STAGE_BYTES + A_STAGES * A_BYTES + X_STAGES * x_stage_bytes(nt) + 1024;
 }
-static_assert(in_stage_bytes(16) % 1024 == 0 && in_stage_bytes(MAX_NT) % 1024 == 0, "stages stay 1024-byte aligned");
+static_assert(C_STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0 && x_stage_bytes(16) % 1024 == 0,
+              "swizzled tiles stay 1024-byte aligned");
+static_assert(MAX_NT * ROWS * 4 <= A_STAGES * A_BYTES, "the partial sums fit in the operand tiles' memory");
 
 // Slices of the k-blocks per row block the workspace is sized for: enough for 512 CTAs, at most
 // MAX_SLICES. The workspace holds partial[n_rb][slices][MAX_NT][ROWS] fp32 and one counter per row block.
@@ -70,8 +77,9 @@ struct Params {
   int64_t M, O, G, ldy;
   int nt;                 // MMA N: M rounded up to 16
   int num_kb;             // K / 64
-  int kb_per;             // k-blocks per slice
+  int kb_per;             // k-blocks per slice, a multiple of KB_PER_BOX
   int slices;
+  int sz_pairs;           // G even and steps / zeros 8-byte aligned: one 8-byte copy per row and array
   uint32_t idesc;
   DeviceStatus* status;
   uint64_t limit_ns;
@@ -118,7 +126,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     w4a16_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[2 * IN_STAGES + 2 * A_STAGES + 1];
+  __shared__ __align__(8) uint64_t bars[2 * C_STAGES + 2 * X_STAGES + 2 * A_STAGES + 1];
   __shared__ uint32_t tmem_slot;
   __shared__ int failed;
   __shared__ unsigned int ticket;
@@ -130,26 +138,32 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int64_t row0 = static_cast<int64_t>(rb) * ROWS;
   const int kb0 = slice * p.kb_per;
   const int nkb = max(0, min(p.kb_per, p.num_kb - kb0));
-  const uint32_t ib = static_cast<uint32_t>(in_stage_bytes(p.nt));
-  const uint32_t x_bytes = static_cast<uint32_t>(p.nt * BK * 2);
+  const uint32_t xb = static_cast<uint32_t>(x_stage_bytes(p.nt));
 
   const uint32_t bar0 = smem_u32(&bars[0]);
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };                      // inputs landed
-  auto empty_bar = [&](int s) { return bar0 + 8u * (IN_STAGES + s); };       // MMAs done with X' of the stage
-  auto dq_bar = [&](int a) { return bar0 + 8u * (2 * IN_STAGES + a); };      // operand tile written
-  auto afree_bar = [&](int a) { return bar0 + 8u * (2 * IN_STAGES + A_STAGES + a); };  // MMAs done with it
-  const uint32_t acc_bar = bar0 + 8u * (2 * IN_STAGES + 2 * A_STAGES);
+  auto cfull_bar = [&](int c) { return bar0 + 8u * c; };                                   // codes landed
+  auto cempty_bar = [&](int c) { return bar0 + 8u * (C_STAGES + c); };                     // codes read
+  auto xfull_bar = [&](int x) { return bar0 + 8u * (2 * C_STAGES + x); };                  // X' landed
+  auto xempty_bar = [&](int x) { return bar0 + 8u * (2 * C_STAGES + X_STAGES + x); };      // MMAs done with X'
+  auto dq_bar = [&](int a) { return bar0 + 8u * (2 * C_STAGES + 2 * X_STAGES + a); };      // operand written
+  auto afree_bar = [&](int a) { return bar0 + 8u * (2 * C_STAGES + 2 * X_STAGES + A_STAGES + a); };
+  const uint32_t acc_bar = bar0 + 8u * (2 * C_STAGES + 2 * X_STAGES + 2 * A_STAGES);
   const uint32_t base = smem_u32(smem);
-  auto a_tile = [&](int a) { return base + static_cast<uint32_t>(a) * A_BYTES; };
-  auto x_tile = [&](int s) { return base + A_STAGES * A_BYTES + static_cast<uint32_t>(s) * ib; };
-  auto c_tile = [&](int s) { return x_tile(s) + x_bytes; };
-  auto s_tile = [&](int s) { return c_tile(s) + C_BYTES; };
-  auto z_tile = [&](int s) { return s_tile(s) + SZ_BYTES; };
+  auto c_tile = [&](int c) { return base + static_cast<uint32_t>(c) * C_STAGE_BYTES; };
+  auto sz_tile = [&](int c) { return c_tile(c) + C_BYTES; };  // [array: step, zero][row][group 0, 1]
+  auto a_tile = [&](int a) { return base + C_STAGES * C_STAGE_BYTES + static_cast<uint32_t>(a) * A_BYTES; };
+  auto x_tile = [&](int x) {
+    return base + C_STAGES * C_STAGE_BYTES + A_STAGES * A_BYTES + static_cast<uint32_t>(x) * xb;
+  };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < IN_STAGES; ++s) {
-      mbar_init(full_bar(s), 1 + 32);  // the TMA arm and the 32 loader lanes' cp.async arrivals
-      mbar_init(empty_bar(s), 1);
+    for (int c = 0; c < C_STAGES; ++c) {
+      mbar_init(cfull_bar(c), 1 + 32);  // the TMA arm and the 32 loader lanes' cp.async arrivals
+      mbar_init(cempty_bar(c), DQ_WARPS);
+    }
+    for (int x = 0; x < X_STAGES; ++x) {
+      mbar_init(xfull_bar(x), 1);
+      mbar_init(xempty_bar(x), 1);
     }
     for (int a = 0; a < A_STAGES; ++a) {
       mbar_init(dq_bar(a), DQ_WARPS);
@@ -170,36 +184,61 @@ __global__ void __launch_bounds__(THREADS, 2)
 
   if (warp == 0) {
     // ------------------------------------------------------------------------------ loads
+    // Box j (k-blocks 4j..4j+3 of the slice) is requested before X' of its first k-block.
+    const bool pair_aligned = p.sz_pairs != 0;  // the box's two groups are one aligned 8-byte pair
     for (int i = 0; i < nkb; ++i) {
-      const int s = i % IN_STAGES;
-      const uint32_t use = static_cast<uint32_t>(i / IN_STAGES);
-      if (use > 0 && !wait_warp(empty_bar(s), (use - 1u) & 1u, p, kSiteDecodeEmpty)) {
+      if (i % KB_PER_BOX == 0) {
+        const int j = i / KB_PER_BOX;
+        const int c = j % C_STAGES;
+        const uint32_t use = static_cast<uint32_t>(j / C_STAGES);
+        if (use > 0 && !wait_warp(cempty_bar(c), (use - 1u) & 1u, p, kSiteDecodeEmpty)) {
+          failed = 1;
+          break;
+        }
+        const int kb = kb0 + i;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(cfull_bar(c), C_BYTES);
+          tma_load_2d(c_tile(c), &tmC, kb * (BK / 8), static_cast<int32_t>(row0), cfull_bar(c));
+        }
+        const int64_t g0 = (static_cast<int64_t>(kb) * BK) >> 7;  // even: kb is a multiple of 4
+#pragma unroll
+        for (int jr = 0; jr < ROWS / 32; ++jr) {
+          const int r = lane + 32 * jr;
+          const int64_t o = min(row0 + r, p.O - 1);  // rows past O: any valid address (their codes are 0)
+          const uint32_t ds = sz_tile(c) + 8u * r, dz = sz_tile(c) + 8u * (ROWS + r);
+          if (pair_aligned) {
+            cp_async_8(ds, p.steps + o * p.G + g0);
+            cp_async_8(dz, p.zeros + o * p.G + g0);
+          } else {
+            cp_async_4(ds, p.steps + o * p.G + g0);
+            cp_async_4(dz, p.zeros + o * p.G + g0);
+            if (g0 + 1 < p.G) {
+              cp_async_4(ds + 4u, p.steps + o * p.G + g0 + 1);
+              cp_async_4(dz + 4u, p.zeros + o * p.G + g0 + 1);
+            }
+          }
+        }
+        cp_async_mbar_arrive(cfull_bar(c));
+      }
+      const int x = i % X_STAGES;
+      const uint32_t xuse = static_cast<uint32_t>(i / X_STAGES);
+      if (xuse > 0 && !wait_warp(xempty_bar(x), (xuse - 1u) & 1u, p, kSiteDecodeEmpty)) {
         failed = 1;
         break;
       }
-      const int kb = kb0 + i;
       if (lane == 0) {
-        mbar_arrive_expect_tx(full_bar(s), C_BYTES + x_bytes);
-        tma_load_2d(c_tile(s), &tmC, kb * (BK / 8), static_cast<int32_t>(row0), full_bar(s));
-        tma_load_2d(x_tile(s), &tmX, kb * BK, 0, full_bar(s));
+        mbar_arrive_expect_tx(xfull_bar(x), xb);
+        tma_load_2d(x_tile(x), &tmX, (kb0 + i) * BK, 0, xfull_bar(x));
       }
-      const int64_t g = (static_cast<int64_t>(kb) * BK) >> 7;
-#pragma unroll
-      for (int j = 0; j < ROWS / 32; ++j) {
-        const int r = lane + 32 * j;
-        const int64_t o = min(row0 + r, p.O - 1);  // rows past O: any valid address (their codes are 0)
-        cp_async_4(s_tile(s) + 4u * r, p.steps + o * p.G + g);
-        cp_async_4(z_tile(s) + 4u * r, p.zeros + o * p.G + g);
-      }
-      cp_async_mbar_arrive(full_bar(s));
+      __syncwarp();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------------------ MMA
     if (elect_one()) {
       bool ok = true;
       for (int i = 0; i < nkb; ++i) {
-        const int s = i % IN_STAGES, a = i % A_STAGES;
-        if (!wait_thread(full_bar(s), static_cast<uint32_t>(i / IN_STAGES) & 1u, p, kSiteDecodeFull) ||
+        const int x = i % X_STAGES, a = i % A_STAGES;
+        if (!wait_thread(xfull_bar(x), static_cast<uint32_t>(i / X_STAGES) & 1u, p, kSiteDecodeFull) ||
             !wait_thread(dq_bar(a), static_cast<uint32_t>(i / A_STAGES) & 1u, p, kSiteDecodeDequant)) {
           ok = false;
           failed = 1;
@@ -208,9 +247,9 @@ __global__ void __launch_bounds__(THREADS, 2)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BK / UK; ++kk)
-          umma_bf16(tmem_base, smem_desc_sw128(a_tile(a) + kk * UK * 2), smem_desc_sw128(x_tile(s) + kk * UK * 2),
+          umma_bf16(tmem_base, smem_desc_sw128(a_tile(a) + kk * UK * 2), smem_desc_sw128(x_tile(x) + kk * UK * 2),
                     p.idesc, (i | kk) != 0 ? 1u : 0u);
-        umma_commit(empty_bar(s));
+        umma_commit(xempty_bar(x));
         umma_commit(afree_bar(a));
       }
       if (ok && nkb > 0)
@@ -223,22 +262,36 @@ __global__ void __launch_bounds__(THREADS, 2)
     // ------------------------------------------------------------------------------ dequantize
     const int r = (warp & 3) * 32 + lane;  // warps 2+q and 6+q both take rows 32q ...
     const int half = (warp - 2) >> 2;      // ... and split the k-block's in-features
+    const uint32_t sw = static_cast<uint32_t>(r & 7);
     for (int i = 0; i < nkb; ++i) {
-      const int s = i % IN_STAGES, a = i % A_STAGES;
-      const uint32_t ause = static_cast<uint32_t>(i / A_STAGES);
-      if (!wait_warp(full_bar(s), static_cast<uint32_t>(i / IN_STAGES) & 1u, p, kSiteDecodeFull)) {
+      const int j = i / KB_PER_BOX, sub = i % KB_PER_BOX;
+      const int c = j % C_STAGES, a = i % A_STAGES;
+      if (!wait_warp(cfull_bar(c), static_cast<uint32_t>(j / C_STAGES) & 1u, p, kSiteDecodeFull)) {
         failed = 1;
         break;
       }
+      // Words 8 sub + 4 half .. +3 of row r: 16-byte chunk 2 sub + half of the row's swizzled line.
+      // "memory" keeps these loads ahead of the barrier arrive below that hands the box back.
       uint32_t w[4];
       float z, stp;
       asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                    : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                   : "r"(c_tile(s) + static_cast<uint32_t>(r * 32 + half * 16)));
-      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(stp) : "r"(s_tile(s) + 4u * r));
-      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(z) : "r"(z_tile(s) + 4u * r));
+                   : "r"(c_tile(c) + static_cast<uint32_t>(r) * 128u +
+                         ((static_cast<uint32_t>(2 * sub + half) ^ sw) << 4))
+                   : "memory");
+      asm volatile("ld.shared.f32 %0, [%1];"
+                   : "=f"(stp)
+                   : "r"(sz_tile(c) + 8u * r + 4u * (sub >> 1))
+                   : "memory");
+      asm volatile("ld.shared.f32 %0, [%1];"
+                   : "=f"(z)
+                   : "r"(sz_tile(c) + 8u * (ROWS + r) + 4u * (sub >> 1))
+                   : "memory");
       uint32_t v[16];
       dequant_words<4>(w, z, stp, v);  // in registers while the operand tile may still be in use
+      __syncwarp();
+      if (lane == 0 && (sub == KB_PER_BOX - 1 || i == nkb - 1)) mbar_arrive(cempty_bar(c));
+      const uint32_t ause = static_cast<uint32_t>(i / A_STAGES);
       if (ause > 0 && !wait_warp(afree_bar(a), (ause - 1u) & 1u, p, kSiteDecodeEmpty)) {
         failed = 1;
         break;
@@ -254,16 +307,16 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (!have && nkb > 0) failed = 1;
       tc_fence_after();
       float* mine = p.partial + (static_cast<int64_t>(rb) * p.slices + slice) * p.nt * ROWS + r;
-      for (int c = 0; c < p.nt / 16; ++c) {
+      for (int cc = 0; cc < p.nt / 16; ++cc) {
         float v[16];
         if (have) {
-          tmem_ld16(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + static_cast<uint32_t>(c * 16), v);
+          tmem_ld16(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + static_cast<uint32_t>(cc * 16), v);
         } else {
 #pragma unroll
           for (int k = 0; k < 16; ++k) v[k] = 0.0f;
         }
 #pragma unroll
-        for (int k = 0; k < 16; ++k) __stcg(mine + (c * 16 + k) * ROWS, v[k]);
+        for (int k = 0; k < 16; ++k) __stcg(mine + (cc * 16 + k) * ROWS, v[k]);
       }
       __threadfence();
       epilogue_sync();

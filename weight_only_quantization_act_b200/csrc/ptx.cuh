@@ -332,6 +332,10 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 __device__ __forceinline__ void cp_async_4(uint32_t dst_smem, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst_smem), "l"(src) : "memory");
 }
+// 8-byte asynchronous copy global -> shared (both addresses 8-byte aligned).
+__device__ __forceinline__ void cp_async_8(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst_smem), "l"(src) : "memory");
+}
 // One arrival on `bar` once every cp.async this thread issued so far has landed (the arrival is one of
 // the barrier's expected arrivals: .noinc).
 __device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
