@@ -771,8 +771,9 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, int64_t M, int64_t K, int64_
   char* ws = static_cast<char*>(workspace);
   float* steps_t = reinterpret_cast<float*>(ws + l.steps_off);
   float* zeros_t = reinterpret_cast<float*>(ws + l.zeros_off);
-  CUtensorMap tmX, tmC, tmS, tmZ;
+  CUtensorMap tmX, tmC, tmS, tmZ, tmY;
   AWQ_TRY(make_tmap(&tmX, X, M, K, ldx, awq::lg::HALF));
+  AWQ_TRY(make_tmap_plain(&tmY, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, O, ldy, awq::dq::Y_CHUNK, 32));
   AWQ_TRY(make_tmap_plain(&tmC, codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, O, K / 8, K / 8, awq::lg::BK / 8,
                           awq::lg::HALF));
   AWQ_TRY(make_tmap_plain(&tmS, steps_t, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, l.G, l.O_pad, l.O_pad, awq::lg::HALF, 1));
@@ -804,7 +805,7 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, int64_t M, int64_t K, int64_
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  AWQ_CUDA(cudaLaunchKernelEx(&cfg, awq::dq::w4a16_gemm_kernel, tmX, tmC, tmS, tmZ, p));
+  AWQ_CUDA(cudaLaunchKernelEx(&cfg, awq::dq::w4a16_gemm_kernel, tmX, tmC, tmS, tmZ, tmY, p));
   AWQ_TRY(check_launch("w4a16_gemm_kernel"));
   return ok();
 }

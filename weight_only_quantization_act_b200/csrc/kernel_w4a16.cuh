@@ -13,7 +13,8 @@
 //          128-byte swizzle; both CTAs' bytes counted on the even CTA's barrier)
 //   1      pair-wide tensor memory (two 256-column fp32 accumulators, one per token half); the even CTA
 //          issues the pair MMAs (tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16)
-//   2-5    epilogue: both accumulators -> bf16 -> Y (each lane one token row, 64-byte pieces)
+//   2-5    epilogue: both accumulators -> bf16 -> Y through two 1 KB staging buffers per warp and TMA
+//          stores of 32 rows x 16 columns (clipped at M and O), so the drain between tiles is short
 //   6      TMA of the code words [128 rows x 8 words], steps and zero points (from a group-major copy) of
 //          every k-block into a ring of its own, so they are resident before the operand stage frees up
 //   7-14   dequantizers, two per operand stage: warps 7+s and 11+s fill every use of stage s with 64 of the
@@ -54,7 +55,9 @@ constexpr int CSTAGE_BYTES = C_BYTES + 2 * S_BYTES;
 constexpr int DQ_PER_STAGE = 2;                   // dequantizer warps per stage (each half the rows)
 constexpr int DQ_WARPS = STAGES * DQ_PER_STAGE;
 constexpr int THREADS = 224 + 32 * DQ_WARPS;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CSTAGES * CSTAGE_BYTES + 1024;
+constexpr int Y_CHUNK = 16;                       // output columns per TMA store (32 rows x 32 bytes)
+constexpr int Y_BUF_BYTES = 32 * Y_CHUNK * 2;     // 1 KB; two per epilogue warp
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CSTAGES * CSTAGE_BYTES + 8 * Y_BUF_BYTES + 1024;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int BANDS_PER_GROUP = 8;                // raster: 8 weight bands advance together over X'
 constexpr uint32_t IDESC = idesc_bf16_f32(BMH, BN);
@@ -126,7 +129,8 @@ __global__ void __launch_bounds__(256) transpose_groups_kernel(const float* __re
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
-                      const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ, Params p) {
+                      const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
+                      const __grid_constant__ CUtensorMap tmY, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t bars[2 * STAGES + 2 * CSTAGES + 3 + RING];
@@ -151,6 +155,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   auto c_tile = [&](int c) { return smem_base + static_cast<uint32_t>(STAGES * STAGE_BYTES + c * CSTAGE_BYTES); };
   auto s_tile = [&](int c) { return c_tile(c) + C_BYTES; };
   auto z_tile = [&](int c) { return c_tile(c) + C_BYTES + S_BYTES; };
+  auto y_buf = [&](int q, int b) {
+    return smem_base + static_cast<uint32_t>(STAGES * STAGE_BYTES + CSTAGES * CSTAGE_BYTES + (2 * q + b) * Y_BUF_BYTES);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -174,6 +181,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmC);
     tma_prefetch_desc(&tmS);
     tma_prefetch_desc(&tmZ);
+    tma_prefetch_desc(&tmY);
   }
   tc_fence_before();
   cluster_sync();
@@ -404,6 +412,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     bool ok = true;
+    int stores = 0;  // TMA stores this warp has issued; buffer stores & 1
     for (int i = 0; ok; ++i) {
       const int t = ring_wait_warp(i, ok);
       if (!ok || t < 0) break;
@@ -413,28 +422,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       tile_coords(t, p, band, mt);
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
-        const int64_t row = static_cast<int64_t>(mt) * TM + h * BMH + static_cast<int64_t>(rank) * HALF +
-                            quarter * 32 + lane;
+        const int32_t row = mt * TM + h * BMH + static_cast<int32_t>(rank) * HALF + quarter * 32;
         const uint32_t taddr =
             tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(h * BN);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          tmem_ld32(taddr + static_cast<uint32_t>(c * 32), v);
-          const int64_t col0 = static_cast<int64_t>(band) * BN + c * 32;
-          if (row < p.M && col0 < p.O) {
-            uint32_t packed[16];
+        for (int c = 0; c < BN / Y_CHUNK; ++c, ++stores) {
+          float v[Y_CHUNK];
+          tmem_ld16(taddr + static_cast<uint32_t>(c * Y_CHUNK), v);
+          uint32_t pk[Y_CHUNK / 2];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const __nv_bfloat162 pr = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-              packed[k] = *reinterpret_cast<const uint32_t*>(&pr);
-            }
-            __nv_bfloat16* dst = p.Y + row * p.ldy + col0;
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (col0 + 8 * q < p.O)  // O % 8 == 0: 16-byte pieces are all in or all out
-                *reinterpret_cast<uint4*>(dst + 8 * q) =
-                    make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+          for (int k = 0; k < Y_CHUNK / 2; ++k) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+            pk[k] = *reinterpret_cast<const uint32_t*>(&pr);
+          }
+          const uint32_t buf = y_buf(quarter, stores & 1);
+          if (stores >= 2) {  // the store issued two chunks ago must have read this buffer
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+          }
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(buf + 32u * lane), "r"(pk[0]), "r"(pk[1]),
+                       "r"(pk[2]), "r"(pk[3])
+                       : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(buf + 32u * lane + 16u), "r"(pk[4]),
+                       "r"(pk[5]), "r"(pk[6]), "r"(pk[7])
+                       : "memory");
+          fence_proxy_async_smem();  // the TMA reads the buffer through the async proxy
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, buf, band * BN + c * Y_CHUNK, row);
+            bulk_commit();
           }
         }
       }
@@ -442,6 +458,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(map_to_rank(acce_bar, 0));
     }
+    if (lane == 0) bulk_wait_all();  // the staging buffers are read and Y written before the CTA ends
+    __syncwarp();
   }
 
   if (status_code(st) != 0u) {
