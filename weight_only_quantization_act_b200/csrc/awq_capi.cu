@@ -558,12 +558,32 @@ awq_status awq_quantize_pack_int8(const void* W, int64_t O, int64_t K, int64_t l
   if (flags & ~AWQ_FLAG_EXACT_DIVISION) return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   DeviceInfo* d = nullptr;
   AWQ_TRY(device_info(&d));
-  // one warp per row, grid-stride; 8 warps of a block and up to 8 blocks per SM resident at once
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int exact = (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0;
+  const int64_t pieces = (K + 8 * awq::kRowBlock - 1) / (8 * awq::kRowBlock);  // 16-byte pieces per thread
+  if (pieces <= 16) {
+    // W read once: one CTA per row with the row in registers (grid-stride over rows)
+    const int64_t blocks = std::min<int64_t>(static_cast<int64_t>(d->sms) * 8, O);
+    const unsigned grid = static_cast<unsigned>(blocks);
+    const auto* w16 = static_cast<const uint16_t*>(W);
+    if (pieces <= 1)
+      awq::quantize_pack_int8_rows_kernel<1><<<grid, awq::kRowBlock, 0, st>>>(w16, O, K, ldw, scales, exact, codes, steps);
+    else if (pieces <= 2)
+      awq::quantize_pack_int8_rows_kernel<2><<<grid, awq::kRowBlock, 0, st>>>(w16, O, K, ldw, scales, exact, codes, steps);
+    else if (pieces <= 4)
+      awq::quantize_pack_int8_rows_kernel<4><<<grid, awq::kRowBlock, 0, st>>>(w16, O, K, ldw, scales, exact, codes, steps);
+    else if (pieces <= 8)
+      awq::quantize_pack_int8_rows_kernel<8><<<grid, awq::kRowBlock, 0, st>>>(w16, O, K, ldw, scales, exact, codes, steps);
+    else
+      awq::quantize_pack_int8_rows_kernel<16><<<grid, awq::kRowBlock, 0, st>>>(w16, O, K, ldw, scales, exact, codes, steps);
+    AWQ_TRY(check_launch("quantize_pack_int8_rows_kernel"));
+    return ok();
+  }
+  // very long rows: one warp per row, two passes over it (grid-stride)
   const int64_t rows_per_block = awq::kRowThreads / 32;
   const int64_t blocks = std::min<int64_t>(static_cast<int64_t>(d->sms) * 8, (O + rows_per_block - 1) / rows_per_block);
-  awq::quantize_pack_int8_kernel<<<static_cast<unsigned>(blocks), awq::kRowThreads, 0,
-                                   reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(W), O, K, ldw, scales, (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0, codes, steps);
+  awq::quantize_pack_int8_kernel<<<static_cast<unsigned>(blocks), awq::kRowThreads, 0, st>>>(
+      static_cast<const uint16_t*>(W), O, K, ldw, scales, exact, codes, steps);
   AWQ_TRY(check_launch("quantize_pack_int8_kernel"));
   return ok();
 }

@@ -328,32 +328,56 @@ __global__ void __launch_bounds__(THREADS, 2)
   __syncthreads();
   if (ticket == static_cast<unsigned int>(p.slices - 1)) {
     // Last slice of this row block: every other slice's sums are visible (each CTA fenced before taking
-    // its ticket). The whole CTA adds them in slice order, four rows per item, all slices' loads in flight.
+    // its ticket). The whole CTA adds them in slice order, four rows per item.
     __threadfence();
     const float* blk = p.partial + static_cast<int64_t>(rb) * p.slices * p.nt * ROWS;
     const int items = static_cast<int>(p.M) * (ROWS / 4);
-    for (int it = threadIdx.x; it < items; it += THREADS) {
-      const int t = it / (ROWS / 4);
-      const int r4 = (it - t * (ROWS / 4)) * 4;
-      const int64_t o = row0 + r4;
-      if (o >= p.O) continue;  // O % 8 == 0: four rows are all in or all out
-      float4 v[MAX_SLICES];
+    // Two items per thread per pass and eight slices per round, so up to 16 loads are in flight at once.
+    for (int base_it = static_cast<int>(threadIdx.x); base_it < items; base_it += 2 * THREADS) {
+      int t[2], r4[2];
+      bool live[2];
 #pragma unroll
-      for (int c = 0; c < MAX_SLICES; ++c)
-        v[c] = c < p.slices ? __ldcg(reinterpret_cast<const float4*>(blk + (static_cast<int64_t>(c) * p.nt + t) * ROWS + r4))
-                            : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      float4 acc = v[0];
+      for (int u = 0; u < 2; ++u) {
+        const int it = base_it + u * THREADS;
+        t[u] = it / (ROWS / 4);
+        r4[u] = (it - t[u] * (ROWS / 4)) * 4;
+        live[u] = it < items && row0 + r4[u] < p.O;  // O % 8 == 0: four rows are all in or all out
+      }
+      float4 acc[2] = {make_float4(0.0f, 0.0f, 0.0f, 0.0f), make_float4(0.0f, 0.0f, 0.0f, 0.0f)};
+#pragma unroll 1
+      for (int c0 = 0; c0 < p.slices; c0 += 8) {
+        float4 v[2][8];
 #pragma unroll
-      for (int c = 1; c < MAX_SLICES; ++c)
-        if (c < p.slices) {
-          acc.x = __fadd_rn(acc.x, v[c].x);
-          acc.y = __fadd_rn(acc.y, v[c].y);
-          acc.z = __fadd_rn(acc.z, v[c].z);
-          acc.w = __fadd_rn(acc.w, v[c].w);
-        }
-      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-      *reinterpret_cast<uint2*>(p.Y + t * p.ldy + o) =
-          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            v[u][c] = live[u] && c0 + c < p.slices
+                          ? __ldcg(reinterpret_cast<const float4*>(blk + (static_cast<int64_t>(c0 + c) * p.nt + t[u]) * ROWS +
+                                                                   r4[u]))
+                          : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (c0 + c >= p.slices) continue;
+            if (c0 + c == 0) {
+              acc[u] = v[u][0];  // slice order: ((s0 + s1) + s2) + ...
+            } else {
+              acc[u].x = __fadd_rn(acc[u].x, v[u][c].x);
+              acc[u].y = __fadd_rn(acc[u].y, v[u][c].y);
+              acc[u].z = __fadd_rn(acc[u].z, v[u][c].z);
+              acc[u].w = __fadd_rn(acc[u].w, v[u][c].w);
+            }
+          }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (!live[u]) continue;
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[u].x, acc[u].y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[u].z, acc[u].w);
+        *reinterpret_cast<uint2*>(p.Y + t[u] * p.ldy + row0 + r4[u]) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+      }
     }
   }
   if (failed) {  // let copies still in flight land before the shared memory is given up

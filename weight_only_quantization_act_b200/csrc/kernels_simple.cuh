@@ -630,4 +630,69 @@ __global__ void __launch_bounds__(kRowThreads) quantize_pack_int8_kernel(
   }
 }
 
+// One CTA per row (grid-stride), the row held in registers: every thread keeps NV 16-byte pieces of it
+// (piece v of thread t = in-features 8 (256 v + t) ..), so W is read once. The row's max |w'| is reduced
+// over the CTA, then each thread codes its pieces. K <= 2048 NV.
+constexpr int kRowBlock = 256;
+template <int NV>
+__global__ void __launch_bounds__(kRowBlock) quantize_pack_int8_rows_kernel(
+    const uint16_t* __restrict__ W, int64_t O, int64_t K, int64_t ldw, const float* __restrict__ scales, int exact,
+    int8_t* __restrict__ codes, float* __restrict__ steps) {
+  __shared__ float wmax[kRowBlock / 32];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  for (int64_t o = blockIdx.x; o < O; o += gridDim.x) {
+    uint4 u[NV];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int64_t k0 = (static_cast<int64_t>(v) * kRowBlock + t) * 8;
+      u[v] = k0 < K ? __ldg(reinterpret_cast<const uint4*>(W + o * ldw + k0)) : make_uint4(0, 0, 0, 0);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int64_t k0 = (static_cast<int64_t>(v) * kRowBlock + t) * 8;
+      if (k0 < K) {
+        const float4 s0 = __ldg(reinterpret_cast<const float4*>(scales + k0));
+        const float4 s1 = __ldg(reinterpret_cast<const float4*>(scales + k0) + 1);
+        const uint32_t uu[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
+        const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          amax = fmaxf(amax, fabsf(__fmul_rn(bf16_lo(uu[i]), ss[2 * i])));
+          amax = fmaxf(amax, fabsf(__fmul_rn(bf16_hi(uu[i]), ss[2 * i + 1])));
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) wmax[warp] = amax;
+    __syncthreads();
+    amax = wmax[0];
+#pragma unroll
+    for (int w = 1; w < kRowBlock / 32; ++w) amax = fmaxf(amax, wmax[w]);
+    __syncthreads();  // wmax is rewritten for the next row
+    const GroupParams g = int8_params(amax);
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int64_t k0 = (static_cast<int64_t>(v) * kRowBlock + t) * 8;
+      if (k0 < K) {
+        const float4 s0 = __ldg(reinterpret_cast<const float4*>(scales + k0));
+        const float4 s1 = __ldg(reinterpret_cast<const float4*>(scales + k0) + 1);
+        const uint32_t uu[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
+        const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int q0 = static_cast<int>(code_of_int8(__fmul_rn(bf16_lo(uu[i]), ss[2 * i]), g, exact != 0));
+          const int q1 = static_cast<int>(code_of_int8(__fmul_rn(bf16_hi(uu[i]), ss[2 * i + 1]), g, exact != 0));
+          packed[i / 2] |= (static_cast<uint32_t>(q0) & 0xFFu) << (16 * (i & 1));
+          packed[i / 2] |= (static_cast<uint32_t>(q1) & 0xFFu) << (16 * (i & 1) + 8);
+        }
+        *reinterpret_cast<uint2*>(codes + o * K + k0) = make_uint2(packed[0], packed[1]);
+      }
+    }
+    if (t == 0) steps[o] = g.step;
+  }
+}
+
 }  // namespace awq
