@@ -443,7 +443,7 @@ def measure_w4a16(Xd, Wd, scales):
     codes, steps, zeros = awq.quantize_pack(Wd, scales)
     Xs = awq.scale_columns(Xd, scales, divide=True)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=Xd.device)
-    ws = torch.empty(awq.load_library().awq_w4a16_workspace_size(Xd.shape[1], codes.shape[0]), dtype=torch.uint8,
+    ws = torch.zeros(awq.load_library().awq_w4a16_workspace_size(Xd.shape[1], codes.shape[0]), dtype=torch.uint8,
                      device=Xd.device)
     out = {}
     for name, X in (("prefill_ms", Xs), ("decode_ms", Xs[:16].contiguous())):

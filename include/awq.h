@@ -259,10 +259,15 @@ AWQ_API awq_status awq_scale_rows(const void *A, int64_t R, int64_t C, int64_t l
  *   X       device bf16 [M, K], row stride ldx (multiple of 8)
  *   codes   device uint32 [O, K/8], steps / zeros device float [O, K/128] (contiguous, as packed)
  *   Y       device bf16 [M, O], row stride ldy (multiple of 8)
- *   workspace  device, >= awq_w4a16_workspace_size(K, O) bytes (status word, tile counter and a
- *              group-major copy of steps and zeros, rewritten every call)
- * Requires K % 128 == 0, O % 8 == 0, M >= 1. A device timeout is reported by awq_search_status() on the
- * same workspace.
+ *   workspace  device, >= awq_w4a16_workspace_size(K, O) bytes, ZERO-FILLED BEFORE ITS FIRST USE
+ *              (e.g. cudaMemsetAsync once after allocating it). It holds the status word and a tile
+ *              counter, a fixed 256 KB region of per-block counters (M <= 64 tokens; every call leaves
+ *              them at zero, and nothing else writes there, so one zero fill serves all later calls
+ *              whatever their shapes), a group-major copy of steps and zeros (many tokens) and split-K
+ *              partial sums (few tokens).
+ * Requires K % 128 == 0, O % 8 == 0, M >= 1. M <= 64 runs a few-token kernel (weight rows on the MMA's M
+ * side, K split across CTAs, partial sums added in a fixed order). A device timeout is reported by
+ * awq_search_status() on the same workspace.
  * ------------------------------------------------------------------------------------------------- */
 AWQ_API size_t awq_w4a16_workspace_size(int64_t K, int64_t O);
 AWQ_API awq_status awq_w4a16_gemm(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *codes,

@@ -124,3 +124,20 @@ def test_w4a16_repeated_runs_are_bit_identical(M, K, O):
     check_against_oracle(Xp, words, steps, zeros, first)
     for _ in range(24):
         assert torch.equal(awq.w4a16_gemm(Xd, *args), first)
+
+
+def test_w4a16_shared_workspace_across_calls_and_shapes():
+    """One workspace, zero-filled once, serves every later call: the few-token kernel's per-block
+    counters are handed back at zero by each call, whatever the shape (different slice counts)."""
+    lib = awq.load_library()
+    shapes = [(16, 4096, 1024), (5, 384, 600), (64, 2048, 1024), (16, 4096, 1024), (300, 512, 256), (1, 256, 136)]
+    ws = torch.zeros(max(lib.awq_w4a16_workspace_size(K, O) for _, K, O in shapes), dtype=torch.uint8,
+                     device="cuda")
+    for n, (M, K, O) in enumerate(shapes):
+        _, _, (words, steps, zeros) = quantized(O, K, 17 * n + 1)
+        Xp = inputs.random_bf16((M, K), 19 * n + 2, scale=1.0)
+        for _ in range(3):
+            Y = awq.w4a16_gemm(bf16_to_device(Xp), torch.from_numpy(words.view(np.int32)).cuda(),
+                               torch.from_numpy(steps).cuda(), torch.from_numpy(zeros).cuda(), workspace=ws)
+            torch.cuda.synchronize()
+            check_against_oracle(Xp, words, steps, zeros, Y)

@@ -379,8 +379,8 @@ def w4a16_gemm(X: torch.Tensor, codes: torch.Tensor, steps: torch.Tensor, zeros:
     O = codes.shape[0]
     if out is None:
         out = torch.empty((M, O), dtype=torch.bfloat16, device=X.device)
-    if workspace is None:
-        workspace = torch.empty(lib.awq_w4a16_workspace_size(K, O), dtype=torch.uint8, device=X.device)
+    if workspace is None:  # zero-filled once; the library keeps its counters zero from call to call
+        workspace = torch.zeros(lib.awq_w4a16_workspace_size(K, O), dtype=torch.uint8, device=X.device)
     _check("awq_w4a16_gemm", lib.awq_w4a16_gemm(_ptr(X), M, K, X.stride(0), _ptr(codes), _ptr(steps), _ptr(zeros),
                                                 O, _ptr(out), out.stride(0), _ptr(workspace), workspace.numel(),
                                                 _stream(stream)))

@@ -697,25 +697,30 @@ struct W4Layout {
   int64_t O_pad, G, n_rb;
   size_t steps_off, zeros_off, counter_off, partial_off, bytes;
 };
-// status (16 B) and tile counter at 0; group-major steps and zeros (many tokens); per-row-block counters
-// and split-K partial sums (few tokens).
+constexpr int64_t kW4MaxRowBlocks = 65536;  // few-token counters reserved for O up to 8M rows
+// [0, 512) status word and tile counter (cleared by each many-token call); [512, 512 + 256 KB) the
+// few-token kernel's per-row-block counters, at the same place for every shape and written by nothing
+// else, so they stay zero from one call to the next whatever the shapes; then the group-major steps and
+// zeros (many tokens) and the split-K partial sums (few tokens).
 W4Layout w4_layout(int64_t K, int64_t O) {
   W4Layout l;
   l.O_pad = (O + awq::lg::BN - 1) / awq::lg::BN * awq::lg::BN;
   l.G = K / 128;
   l.n_rb = (O + awq::dec::ROWS - 1) / awq::dec::ROWS;
-  l.steps_off = 512;
+  l.counter_off = 512;
+  l.steps_off = l.counter_off + static_cast<size_t>(kW4MaxRowBlocks) * 4;
   l.zeros_off = align_up(l.steps_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
-  l.counter_off = align_up(l.zeros_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
-  l.partial_off = align_up(l.counter_off + static_cast<size_t>(l.n_rb) * 4, 256);
-  l.bytes = align_up(l.partial_off + static_cast<size_t>(l.n_rb) * awq::dec::max_slices(l.n_rb) * awq::dec::MAX_NT *
+  l.partial_off = align_up(l.zeros_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
+  const int64_t rb = std::min(l.n_rb, kW4MaxRowBlocks);
+  l.bytes = align_up(l.partial_off + static_cast<size_t>(rb) * awq::dec::max_slices(rb) * awq::dec::MAX_NT *
                                          awq::dec::ROWS * 4,
                      256);
   return l;
 }
 
 // Few tokens: weight rows on the MMA's M side, k-blocks split into slices until every SM has a share,
-// slices added by the last CTA of each row block. A memset of the counters and one launch.
+// slices added by the last CTA of each row block. One launch; the per-block counters are zero from the
+// caller's initial zero fill and every call leaves them zero.
 awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const uint32_t* codes, const float* steps,
                         const float* zeros, int64_t O, void* Y, int64_t ldy, void* workspace, const W4Layout& l,
                         awq_stream_t stream) {
@@ -723,7 +728,9 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   AWQ_TRY(device_info(&d));
   const int nt = static_cast<int>((M + 15) / 16 * 16);
   const int num_kb = static_cast<int>(K / awq::dec::BK);
-  int64_t slices = 2 * static_cast<int64_t>(d->sms) / l.n_rb;  // one wave at two CTAs per SM
+  // one wave: two CTAs per SM when their shared memory allows it (up to 32 tokens), else one
+  const int64_t per_sm = awq::dec::smem_bytes(nt) <= 112 * 1024 ? 2 : 1;
+  int64_t slices = per_sm * static_cast<int64_t>(d->sms) / l.n_rb;
   slices = std::max<int64_t>(1, std::min<int64_t>({slices, awq::dec::max_slices(l.n_rb), num_kb}));
   const int kb_box = awq::dec::KB_PER_BOX;
   const int kb_per = static_cast<int>(((num_kb + slices - 1) / slices + kb_box - 1) / kb_box * kb_box);
@@ -755,7 +762,6 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   p.idesc = awq::idesc_bf16_f32(awq::dec::ROWS, static_cast<uint32_t>(nt));
   p.status = reinterpret_cast<awq::DeviceStatus*>(ws);
   p.limit_ns = g_wait_limit_ns.load();
-  AWQ_CUDA(cudaMemsetAsync(p.counter, 0, static_cast<size_t>(l.n_rb) * 4, st));
   awq::dec::w4a16_decode_kernel<<<static_cast<unsigned>(l.n_rb * slices), awq::dec::THREADS,
                                   awq::dec::smem_bytes(nt), st>>>(tmX, tmC, p);
   AWQ_TRY(check_launch("w4a16_decode_kernel"));
@@ -781,7 +787,8 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, int64_t M, int64_t K, int64_
   if (workspace == nullptr || ws_bytes < l.bytes)
     return fail(AWQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", l.bytes, workspace ? ws_bytes : 0);
   if (!aligned16(workspace)) return fail(AWQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
-  if (M <= awq::dec::MAX_NT) return w4a16_decode(X, M, K, ldx, codes, steps, zeros, O, Y, ldy, workspace, l, stream);
+  if (M <= awq::dec::MAX_NT && l.n_rb <= kW4MaxRowBlocks)
+    return w4a16_decode(X, M, K, ldx, codes, steps, zeros, O, Y, ldy, workspace, l, stream);
   const int64_t n_tiles_m = (M + awq::dq::TM - 1) / awq::dq::TM;
   const int64_t n_bands = l.O_pad / awq::dq::BN;
   if (n_tiles_m * n_bands >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "too many tiles");

@@ -6,8 +6,9 @@
 //   CTA (b, c) covers weight rows [128 b, 128 b + 128) and k-blocks [c * kb_per, (c + 1) * kb_per)
 //   (kb_per a multiple of 4); D[128 rows][nt tokens] accumulates in tensor memory (tcgen05.mma
 //   cta_group::1, kind::f16, M = 128, N = nt = tokens rounded up to 16, K = 16) and is written to the
-//   workspace as slice c of row block b; the last CTA of a row block to finish (a per-block counter) adds
-//   the S slices in slice order (deterministic), converts to bf16 and writes Y.
+//   workspace as slice c of row block b; the last CTA of a row block to finish (a per-block counter,
+//   which it resets to zero for the next call) adds the S slices in slice order (deterministic), converts
+//   to bf16 and writes Y. With one slice the accumulator goes straight to Y.
 //
 // The loads are few and large, since scattered small requests are what limits this size: the code words
 // of 4 k-blocks come as one TMA box [128 rows x 32 words] with 128-byte swizzle (128 contiguous bytes per
@@ -73,7 +74,7 @@ struct Params {
   const float* zeros;     // [O][G]
   __nv_bfloat16* Y;       // [M][ldy]
   float* partial;         // [n_rb][slices][nt][ROWS]
-  unsigned int* counter;  // [n_rb], zero at launch
+  unsigned int* counter;  // [n_rb], zero at launch and left zero
   int64_t M, O, G, ldy;
   int nt;                 // MMA N: M rounded up to 16
   int num_kb;             // K / 64
@@ -176,6 +177,63 @@ __global__ void __launch_bounds__(THREADS, 2)
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmC);
   }
+  // Loads of k-block i: its code box when i starts one (the TMA part, then the steps and zero points),
+  // and its X' tile. Warp 0 only, all lanes; false when a wait gave up.
+  const bool pair_aligned = p.sz_pairs != 0;  // the box's two groups are one aligned 8-byte pair
+  auto box_tma = [&](int i) -> bool {           // i a multiple of KB_PER_BOX
+    const int j = i / KB_PER_BOX;
+    const int c = j % C_STAGES;
+    const uint32_t use = static_cast<uint32_t>(j / C_STAGES);
+    if (use > 0 && !wait_warp(cempty_bar(c), (use - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(cfull_bar(c), C_BYTES);
+      tma_load_2d(c_tile(c), &tmC, (kb0 + i) * (BK / 8), static_cast<int32_t>(row0), cfull_bar(c));
+    }
+    return true;
+  };
+  auto box_sz = [&](int i) {  // after box_tma(i)
+    const int c = (i / KB_PER_BOX) % C_STAGES;
+    const int64_t g0 = (static_cast<int64_t>(kb0 + i) * BK) >> 7;  // even: kb0 + i is a multiple of 4
+#pragma unroll
+    for (int jr = 0; jr < ROWS / 32; ++jr) {
+      const int r = lane + 32 * jr;
+      const int64_t o = min(row0 + r, p.O - 1);  // rows past O: any valid address (their codes are 0)
+      const uint32_t ds = sz_tile(c) + 8u * r, dz = sz_tile(c) + 8u * (ROWS + r);
+      if (pair_aligned) {
+        cp_async_8(ds, p.steps + o * p.G + g0);
+        cp_async_8(dz, p.zeros + o * p.G + g0);
+      } else {
+        cp_async_4(ds, p.steps + o * p.G + g0);
+        cp_async_4(dz, p.zeros + o * p.G + g0);
+        if (g0 + 1 < p.G) {
+          cp_async_4(ds + 4u, p.steps + o * p.G + g0 + 1);
+          cp_async_4(dz + 4u, p.zeros + o * p.G + g0 + 1);
+        }
+      }
+    }
+    cp_async_mbar_arrive(cfull_bar(c));
+  };
+  auto x_tma = [&](int i) -> bool {
+    const int x = i % X_STAGES;
+    const uint32_t xuse = static_cast<uint32_t>(i / X_STAGES);
+    if (xuse > 0 && !wait_warp(xempty_bar(x), (xuse - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(xfull_bar(x), xb);
+      tma_load_2d(x_tile(x), &tmX, (kb0 + i) * BK, 0, xfull_bar(x));
+    }
+    __syncwarp();
+    return true;
+  };
+  // The first k-blocks need no free slots: warp 0 requests them right after initialising the barriers
+  // (every TMA first, then the steps and zero points), so the first memory round trip overlaps the
+  // tensor-memory allocation and the CTA barrier.
+  const int pre = min(nkb, min(C_STAGES * KB_PER_BOX, X_STAGES));
+  if (warp == 0) {
+    __syncwarp();  // the barriers thread 0 initialised are visible to the whole warp
+    for (int i = 0; i < pre; i += KB_PER_BOX) box_tma(i);
+    for (int i = 0; i < pre; ++i) x_tma(i);
+    for (int i = 0; i < pre; i += KB_PER_BOX) box_sz(i);
+  }
   if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -185,52 +243,18 @@ __global__ void __launch_bounds__(THREADS, 2)
   if (warp == 0) {
     // ------------------------------------------------------------------------------ loads
     // Box j (k-blocks 4j..4j+3 of the slice) is requested before X' of its first k-block.
-    const bool pair_aligned = p.sz_pairs != 0;  // the box's two groups are one aligned 8-byte pair
-    for (int i = 0; i < nkb; ++i) {
+    for (int i = pre; i < nkb; ++i) {
       if (i % KB_PER_BOX == 0) {
-        const int j = i / KB_PER_BOX;
-        const int c = j % C_STAGES;
-        const uint32_t use = static_cast<uint32_t>(j / C_STAGES);
-        if (use > 0 && !wait_warp(cempty_bar(c), (use - 1u) & 1u, p, kSiteDecodeEmpty)) {
+        if (!box_tma(i)) {
           failed = 1;
           break;
         }
-        const int kb = kb0 + i;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(cfull_bar(c), C_BYTES);
-          tma_load_2d(c_tile(c), &tmC, kb * (BK / 8), static_cast<int32_t>(row0), cfull_bar(c));
-        }
-        const int64_t g0 = (static_cast<int64_t>(kb) * BK) >> 7;  // even: kb is a multiple of 4
-#pragma unroll
-        for (int jr = 0; jr < ROWS / 32; ++jr) {
-          const int r = lane + 32 * jr;
-          const int64_t o = min(row0 + r, p.O - 1);  // rows past O: any valid address (their codes are 0)
-          const uint32_t ds = sz_tile(c) + 8u * r, dz = sz_tile(c) + 8u * (ROWS + r);
-          if (pair_aligned) {
-            cp_async_8(ds, p.steps + o * p.G + g0);
-            cp_async_8(dz, p.zeros + o * p.G + g0);
-          } else {
-            cp_async_4(ds, p.steps + o * p.G + g0);
-            cp_async_4(dz, p.zeros + o * p.G + g0);
-            if (g0 + 1 < p.G) {
-              cp_async_4(ds + 4u, p.steps + o * p.G + g0 + 1);
-              cp_async_4(dz + 4u, p.zeros + o * p.G + g0 + 1);
-            }
-          }
-        }
-        cp_async_mbar_arrive(cfull_bar(c));
+        box_sz(i);
       }
-      const int x = i % X_STAGES;
-      const uint32_t xuse = static_cast<uint32_t>(i / X_STAGES);
-      if (xuse > 0 && !wait_warp(xempty_bar(x), (xuse - 1u) & 1u, p, kSiteDecodeEmpty)) {
+      if (!x_tma(i)) {
         failed = 1;
         break;
       }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(xfull_bar(x), xb);
-        tma_load_2d(x_tile(x), &tmX, (kb0 + i) * BK, 0, xfull_bar(x));
-      }
-      __syncwarp();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------------------ MMA
@@ -302,31 +326,57 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (lane == 0) mbar_arrive(dq_bar(a));
     }
     if (warp < 6) {
-      // -------------------------------------------------------------------- accumulator -> workspace
+      // -------------------------------------------------------------------- accumulator out
       const bool have = wait_warp(acc_bar, 0u, p, kSiteDecodeAcc) && nkb > 0;
       if (!have && nkb > 0) failed = 1;
       tc_fence_after();
-      float* mine = p.partial + (static_cast<int64_t>(rb) * p.slices + slice) * p.nt * ROWS + r;
-      for (int cc = 0; cc < p.nt / 16; ++cc) {
-        float v[16];
-        if (have) {
-          tmem_ld16(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + static_cast<uint32_t>(cc * 16), v);
-        } else {
+      const uint32_t tlane = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+      if (p.slices == 1) {
+        // One slice: the accumulator is the result; each lane writes its weight row of Y.
+        const int64_t o = row0 + r;
+        for (int cc = 0; cc < p.nt / 16; ++cc) {
+          float v[16];
+          if (have) {
+            tmem_ld16(tlane + static_cast<uint32_t>(cc * 16), v);
+          } else {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) v[k] = 0.0f;
+            for (int k = 0; k < 16; ++k) v[k] = 0.0f;
+          }
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int t = cc * 16 + k;
+            if (t < p.M && o < p.O) p.Y[t * p.ldy + o] = __float2bfloat16_rn(v[k]);
+          }
         }
+      } else {
+        // Slice `slice` of the row block's partial sums, then a ticket.
+        float* mine = p.partial + (static_cast<int64_t>(rb) * p.slices + slice) * p.nt * ROWS + r;
+        for (int cc = 0; cc < p.nt / 16; ++cc) {
+          float v[16];
+          if (have) {
+            tmem_ld16(tlane + static_cast<uint32_t>(cc * 16), v);
+          } else {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) __stcg(mine + (cc * 16 + k) * ROWS, v[k]);
+            for (int k = 0; k < 16; ++k) v[k] = 0.0f;
+          }
+#pragma unroll
+          for (int k = 0; k < 16; ++k) __stcg(mine + (cc * 16 + k) * ROWS, v[k]);
+        }
+        __threadfence();
+        epilogue_sync();
+        if (warp == 2 && lane == 0) {
+          // Every CTA takes a ticket, even after a timeout, and the last one hands the counter back at
+          // zero, so the next call needs no clearing.
+          ticket = atomicAdd(p.counter + rb, 1u);
+          if (ticket == static_cast<unsigned int>(p.slices - 1)) p.counter[rb] = 0u;
+        }
       }
-      __threadfence();
-      epilogue_sync();
-      if (warp == 2 && lane == 0) ticket = atomicAdd(p.counter + rb, 1u);
     }
   }
 
   __syncwarp();
   __syncthreads();
-  if (ticket == static_cast<unsigned int>(p.slices - 1)) {
+  if (p.slices > 1 && ticket == static_cast<unsigned int>(p.slices - 1)) {
     // Last slice of this row block: every other slice's sums are visible (each CTA fenced before taking
     // its ticket). The whole CTA adds them in slice order, four rows per item.
     __threadfence();
