@@ -435,7 +435,8 @@ def measure_int8_pack(Wd, scales):
 
 def measure_w4a16(Xd, Wd, scales):
     """The deployment GEMM on the quantized layer: a prefill of all N calibration tokens and a 16-token
-    decode step, each timed alone (L2 flushed before every launch)."""
+    decode step. Each is timed cold: 40 launches, each after a 512 MiB L2 flush, between two events,
+    minus 40 flushes alone (single launches would be read off an event clock that ticks in ~2 us steps)."""
     import torch
 
     from weight_only_quantization_act_b200 import awq
@@ -445,20 +446,26 @@ def measure_w4a16(Xd, Wd, scales):
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=Xd.device)
     ws = torch.zeros(awq.load_library().awq_w4a16_workspace_size(Xd.shape[1], codes.shape[0]), dtype=torch.uint8,
                      device=Xd.device)
+
+    def batch(fn, n=40):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            flush.zero_()
+            if fn is not None:
+                fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
     out = {}
     for name, X in (("prefill_ms", Xs), ("decode_ms", Xs[:16].contiguous())):
         Y = torch.empty((X.shape[0], codes.shape[0]), dtype=torch.bfloat16, device=Xd.device)
-        times = []
-        for i in range(6):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            awq.w4a16_gemm(X, codes, steps, zeros, out=Y, workspace=ws)
-            e1.record()
-            torch.cuda.synchronize()
-            if i >= 2:
-                times.append(e0.elapsed_time(e1))
-        out[name] = float(np.mean(times))
+        fn = lambda X=X, Y=Y: awq.w4a16_gemm(X, codes, steps, zeros, out=Y, workspace=ws)
+        batch(fn, 4)
+        batch(None, 4)
+        base = float(np.median([batch(None) for _ in range(3)]))
+        out[name] = float(np.median([batch(fn) for _ in range(3)])) - base
     return out
 
 
