@@ -12,7 +12,7 @@ Plain, slow, step-by-step restatement of the method, one operation at a time:
 * sums that define the activation statistic are fp64, in a fixed order;
 * the reconstruction loss is evaluated in fp64 (the weight error ``w - w_hat`` is exact in fp64).
 
-Sources (five web pages about AWQ, cited by title and section):
+Sources (web pages about AWQ and weight quantization, cited by title and section):
 
 [P1] "AWQ 离群激活平滑实操逐通道等价缩放与 4-bit 精度无损转换" (gsyq.cn): section 一 (the equivalence
      ``Y = (X diag(s)^-1)(diag(s) W)``), section 二 (the asymmetric group-128 INT4 pseudo-quantizer and the
@@ -24,6 +24,9 @@ Sources (five web pages about AWQ, cited by title and section):
      .clamp(min=1e-4)``, ``scales = scales / sqrt(scales.max() * scales.min())``, ratio in [0, 1) with step
      1/n_grid, n_grid = 20), section 缩放因子搜索流程 (scale, quantize, unscale, MSE, keep the minimum),
      section NormLinearSubgraph (several linears on one input share one scale; outputs concatenated).
+[P5] "大模型量化中的离群值：成因、解法与部署实战" (hncyxsy.com): section 1.1 (outlier channels sit at nearly
+     fixed positions), sections 2.1-2.2 (symmetric per-channel INT8, ``s = max|x| / 127``, codes clamped to
+     [-127, 127], and the worked figures of one outlier wiping out small values), used by the INT8 option.
 
 Readings where the pages are silent or disagree (each is listed with its reason in the design notes):
 the mean statistic (P2/P4) rather than P1's max formula; P4's clamp-then-normalise with the geometric
