@@ -17,23 +17,41 @@ namespace awq {
 // the high nibble in place gives 2^23 + 16 q. Subtracting 2^23 + z (resp. 2^23 + 16 z), both exact
 // integers below 2^24, leaves q - z (resp. 16 (q - z)) exactly, and multiplying by step (resp. step / 16,
 // an exact power-of-two scaling) rounds the same real product once. One shift per byte instead of one
-// per code. Slow path (huge |z|): RN32(q - z) directly, as the quantizer defines it.
+// per code, and the two codes of a byte go through one paired subtract and one paired multiply. Slow path (huge |z|): RN32(q - z) directly, as the quantizer defines it.
+// Two fp32 lanes in one 64-bit register for the paired fp32 instructions of sm_100 (each lane is an
+// ordinary IEEE operation rounded to nearest, so a pair gives exactly what two scalar operations give).
+__device__ __forceinline__ uint64_t f32x2_pack(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_sub_mul(uint64_t a, uint64_t b, uint64_t c) {  // (a - b) * c
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;\n\tmul.rn.f32x2 %0, %0, %3;" : "=&l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(uint64_t v) {  // low lane -> low half, rounded to nearest
+  uint32_t lo, hi, r;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "r"(hi), "r"(lo));
+  return r;
+}
+
 template <int NW>
 __device__ __forceinline__ void dequant_words(const uint32_t (&w)[NW], float z, float stp, uint32_t (&o)[4 * NW]) {
   if (fabsf(z) < 524288.0f) {
     const float zb = __fadd_rn(8388608.0f, z);
     const float zb16 = __fadd_rn(8388608.0f, __fmul_rn(16.0f, z));
     const float st16 = __fmul_rn(stp, 0.0625f);
+    const uint64_t zz = f32x2_pack(__float_as_uint(zb), __float_as_uint(zb16));
+    const uint64_t ss = f32x2_pack(__float_as_uint(stp), __float_as_uint(st16));
 #pragma unroll
     for (int c = 0; c < NW; ++c)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint32_t b = w[c] >> (8 * j);
-        const float lo = __uint_as_float((b & 0x0Fu) | 0x4B000000u);
-        const float hi = __uint_as_float((b & 0xF0u) | 0x4B000000u);
-        const __nv_bfloat162 pr =
-            __floats2bfloat162_rn(__fmul_rn(__fsub_rn(lo, zb), stp), __fmul_rn(__fsub_rn(hi, zb16), st16));
-        o[4 * c + j] = *reinterpret_cast<const uint32_t*>(&pr);
+        const uint64_t v = f32x2_pack((b & 0x0Fu) | 0x4B000000u, (b & 0xF0u) | 0x4B000000u);
+        o[4 * c + j] = f32x2_to_bf16x2(f32x2_sub_mul(v, zz, ss));
       }
   } else {
 #pragma unroll

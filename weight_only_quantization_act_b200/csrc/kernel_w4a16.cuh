@@ -14,7 +14,9 @@
 //   1      pair-wide tensor memory (two 256-column fp32 accumulators, one per token half); the even CTA
 //          issues the pair MMAs (tcgen05.mma.cta_group::2 kind::f16, M = 256, N = 256, K = 16)
 //   2-5    epilogue: both accumulators -> bf16 -> Y through two 1 KB staging buffers per warp and TMA
-//          stores of 32 rows x 16 columns (clipped at M and O), so the drain between tiles is short
+//          stores of 32 rows x 16 columns (clipped at M and O), each chunk's TMEM load issued one chunk
+//          ahead and the accumulators released once the last chunk is read, so the drain between tiles
+//          is short
 //   6      TMA of the code words [128 rows x 8 words], steps and zero points (from a group-major copy) of
 //          every k-block into a ring of its own, so they are resident before the operand stage frees up
 //   7-14   dequantizers, two per operand stage: warps 7+s and 11+s fill every use of stage s with 64 of the
@@ -92,8 +94,30 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& band, i
 }
 
 // Warp-uniform bounded wait (all lanes poll), with cluster-scope acquire when `cluster` is set.
+// tcgen05.ld of 16 accumulator columns (32 lanes x 32 bit) without the wait, so the next chunk's load
+// runs while the previous one is converted and stored. The registers hold the values only after
+// tmem_wait_ld16 on them; passing them through that asm as read-write operands keeps every use below it.
+__device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])
+               :
+               : "memory");
+}
+
 __device__ __forceinline__ bool warp_wait_any(uint32_t bar, uint32_t parity, DeviceStatus* st, uint64_t limit,
                                               unsigned where, bool cluster) {
+  // the phase has usually completed already: one poll before the timer is read
+  if (__all_sync(0xffffffffu, cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity))) return true;
   uint64_t t0 = 0;
   const int lane = threadIdx.x & 31;
   if (lane == 0) t0 = global_timer_ns();
@@ -420,43 +444,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       tc_fence_after();
       int band, mt;
       tile_coords(t, p, band, mt);
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
+      // 32 chunks of 16 columns: both token halves' accumulators, each chunk's TMEM load issued while the
+      // previous chunk is converted and stored; the accumulators go back to the MMA warp as soon as the
+      // last chunk is in registers.
+      constexpr int CHUNKS = 2 * BN / Y_CHUNK;
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+      auto chunk_addr = [&](int cc) {
+        return tq + static_cast<uint32_t>((cc / (BN / Y_CHUNK)) * BN + (cc % (BN / Y_CHUNK)) * Y_CHUNK);
+      };
+      auto emit = [&](const uint32_t (&r)[16], int cc) {
+        const int h = cc / (BN / Y_CHUNK), c = cc % (BN / Y_CHUNK);
         const int32_t row = mt * TM + h * BMH + static_cast<int32_t>(rank) * HALF + quarter * 32;
-        const uint32_t taddr =
-            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(h * BN);
-#pragma unroll 1
-        for (int c = 0; c < BN / Y_CHUNK; ++c, ++stores) {
-          float v[Y_CHUNK];
-          tmem_ld16(taddr + static_cast<uint32_t>(c * Y_CHUNK), v);
-          uint32_t pk[Y_CHUNK / 2];
+        uint32_t pk[Y_CHUNK / 2];
 #pragma unroll
-          for (int k = 0; k < Y_CHUNK / 2; ++k) {
-            const __nv_bfloat162 pr = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-            pk[k] = *reinterpret_cast<const uint32_t*>(&pr);
-          }
-          const uint32_t buf = y_buf(quarter, stores & 1);
-          if (stores >= 2) {  // the store issued two chunks ago must have read this buffer
-            if (lane == 0) bulk_wait_read<1>();
-            __syncwarp();
-          }
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(buf + 32u * lane), "r"(pk[0]), "r"(pk[1]),
-                       "r"(pk[2]), "r"(pk[3])
-                       : "memory");
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(buf + 32u * lane + 16u), "r"(pk[4]),
-                       "r"(pk[5]), "r"(pk[6]), "r"(pk[7])
-                       : "memory");
-          fence_proxy_async_smem();  // the TMA reads the buffer through the async proxy
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmY, buf, band * BN + c * Y_CHUNK, row);
-            bulk_commit();
-          }
+        for (int k = 0; k < Y_CHUNK / 2; ++k) {
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+          pk[k] = *reinterpret_cast<const uint32_t*>(&pr);
         }
+        const uint32_t buf = y_buf(quarter, stores & 1);
+        if (stores >= 2) {  // the store issued two chunks ago must have read this buffer
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+        }
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(buf + 32u * lane), "r"(pk[0]), "r"(pk[1]),
+                     "r"(pk[2]), "r"(pk[3])
+                     : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(buf + 32u * lane + 16u), "r"(pk[4]),
+                     "r"(pk[5]), "r"(pk[6]), "r"(pk[7])
+                     : "memory");
+        fence_proxy_async_smem();  // the TMA reads the buffer through the async proxy
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmY, buf, band * BN + c * Y_CHUNK, row);
+          bulk_commit();
+        }
+        ++stores;
+      };
+      uint32_t ra[16], rb[16];
+      tmem_ld16_issue(chunk_addr(0), ra);
+#pragma unroll 1
+      for (int cc = 0; cc < CHUNKS; cc += 2) {
+        tmem_wait_ld16(ra);
+        tmem_ld16_issue(chunk_addr(cc + 1), rb);
+        emit(ra, cc);
+        tmem_wait_ld16(rb);
+        if (cc + 2 < CHUNKS) {
+          tmem_ld16_issue(chunk_addr(cc + 2), ra);
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(map_to_rank(acce_bar, 0));
+        }
+        emit(rb, cc + 1);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(map_to_rank(acce_bar, 0));
     }
     if (lane == 0) bulk_wait_all();  // the staging buffers are read and Y written before the CTA ends
     __syncwarp();

@@ -104,6 +104,8 @@ __device__ __forceinline__ bool wait_thread(uint32_t bar, uint32_t parity, const
 
 // Warp-uniform bounded wait: every lane polls, the warp leaves together.
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const Params& p, unsigned int where) {
+  // the phase has usually completed already: one poll before the timer is read
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   const int lane = threadIdx.x & 31;
   uint64_t t0 = 0;
   if (lane == 0) t0 = global_timer_ns();
