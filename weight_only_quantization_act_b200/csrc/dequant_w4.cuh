@@ -9,15 +9,6 @@
 
 namespace awq {
 
-// NW consecutive code words of one weight row (in-feature 8c+i at bits 4i..4i+3 of word c) -> 8 NW bf16
-// values, packed two per register in in-feature order (o[4c + j] holds in-features 8c+2j, 8c+2j+1).
-//
-// Fast path (|z| < 2^19, every zero point a quantizer produces for sane weights): byte j of a word holds
-// two codes; OR-ing the low nibble into the mantissa of 2^23 gives the float 2^23 + q exactly, OR-ing
-// the high nibble in place gives 2^23 + 16 q. Subtracting 2^23 + z (resp. 2^23 + 16 z), both exact
-// integers below 2^24, leaves q - z (resp. 16 (q - z)) exactly, and multiplying by step (resp. step / 16,
-// an exact power-of-two scaling) rounds the same real product once. One shift per byte instead of one
-// per code, and the two codes of a byte go through one paired subtract and one paired multiply. Slow path (huge |z|): RN32(q - z) directly, as the quantizer defines it.
 // Two fp32 lanes in one 64-bit register for the paired fp32 instructions of sm_100 (each lane is an
 // ordinary IEEE operation rounded to nearest, so a pair gives exactly what two scalar operations give).
 __device__ __forceinline__ uint64_t f32x2_pack(uint32_t lo, uint32_t hi) {
@@ -37,6 +28,17 @@ __device__ __forceinline__ uint32_t f32x2_to_bf16x2(uint64_t v) {  // low lane -
   return r;
 }
 
+// NW consecutive code words of one weight row (in-feature 8c+i at bits 4i..4i+3 of word c) -> 8 NW bf16
+// values, packed two per register in in-feature order (o[4c + j] holds in-features 8c+2j, 8c+2j+1).
+//
+// Fast path (|z| < 2^19, every zero point a quantizer produces for sane weights): byte j of a word holds
+// two codes; one byte permute puts the byte under the exponent bits of 2^23 (0x4B0000bb), and masking
+// keeps the low nibble (the float 2^23 + q) or the high nibble in place (2^23 + 16 q). Subtracting
+// 2^23 + z (resp. 2^23 + 16 z), both exact integers below 2^24, leaves q - z (resp. 16 (q - z)) exactly,
+// and multiplying by step (resp. step / 16, an exact power-of-two scaling) rounds the same real product
+// once. The two codes of a byte go through one paired subtract and one paired multiply. (Measured: the
+// permute costs fewer ALU-pipe instructions per code than a shift per byte, and the ALU pipe is what
+// bounds the dequantization.) Slow path (huge |z|): RN32(q - z) directly, as the quantizer defines it.
 template <int NW>
 __device__ __forceinline__ void dequant_words(const uint32_t (&w)[NW], float z, float stp, uint32_t (&o)[4 * NW]) {
   if (fabsf(z) < 524288.0f) {
@@ -49,8 +51,9 @@ __device__ __forceinline__ void dequant_words(const uint32_t (&w)[NW], float z, 
     for (int c = 0; c < NW; ++c)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint32_t b = w[c] >> (8 * j);
-        const uint64_t v = f32x2_pack((b & 0x0Fu) | 0x4B000000u, (b & 0xF0u) | 0x4B000000u);
+        uint32_t t;  // 2^23 + byte j: byte j of the word under the exponent bits of 2^23
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(w[c]), "r"(0x4B000000u), "r"(0x7650u | j));
+        const uint64_t v = f32x2_pack(t & 0x4B00000Fu, t & 0x4B0000F0u);
         o[4 * c + j] = f32x2_to_bf16x2(f32x2_sub_mul(v, zz, ss));
       }
   } else {
