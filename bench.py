@@ -436,7 +436,8 @@ def measure_int8_pack(Wd, scales):
 def measure_w4a16(Xd, Wd, scales):
     """The deployment GEMM on the quantized layer: a prefill of all N calibration tokens and a 16-token
     decode step. Each is timed cold: 40 launches, each after a 512 MiB L2 flush, between two events,
-    minus 40 flushes alone (single launches would be read off an event clock that ticks in ~2 us steps)."""
+    minus 40 flushes alone timed just before (single launches would be read off an event clock that ticks
+    in ~2 us steps); the median over seven such pairs."""
     import torch
 
     from weight_only_quantization_act_b200 import awq
@@ -464,8 +465,13 @@ def measure_w4a16(Xd, Wd, scales):
         fn = lambda X=X, Y=Y: awq.w4a16_gemm(X, codes, steps, zeros, out=Y, workspace=ws)
         batch(fn, 4)
         batch(None, 4)
-        base = float(np.median([batch(None) for _ in range(3)]))
-        out[name] = float(np.median([batch(fn) for _ in range(3)])) - base
+        # flush-only and flush+kernel batches alternate, so a drift of the flush time cancels in each
+        # pair; the median of the pairs' differences is the kernel time
+        diffs = []
+        for _ in range(7):
+            base = batch(None)
+            diffs.append(batch(fn) - base)
+        out[name] = float(np.median(diffs))
     return out
 
 
