@@ -16,9 +16,10 @@
 // comes per k-block [nt x 64] (128-byte swizzle) through a ring of its own.
 //
 // Warps: 0 loads (lane 0 the TMA boxes; all lanes the steps and zero points); 1 allocates tensor memory
-// and issues the MMAs; 2-9 dequantize into a 3-deep ring of K-major swizzled operand tiles (warp 2 + q + 4h
-// takes rows 32q..32q+31, in-features 32h..32h+31 of the k-block), computing in registers first and
-// storing once the tile is free; warps 2-5 then read the accumulator (warp w may read tensor-memory lanes
+// and issues the MMAs; 2-9 dequantize into a 3-deep ring of K-major swizzled operand tiles in two groups
+// that take alternate k-blocks (warp 2 + q + 4g takes rows 32q..32q+31, all 64 in-features, of the
+// k-blocks i with i % 2 == g, so each warp synchronises once per 64 weights of a row), computing in
+// registers first and storing once the tile is free; warps 2-5 then read the accumulator (warp w may read tensor-memory lanes
 // 32 (w % 4) ...). All waits are bounded; a timeout is recorded in the caller's status word.
 #pragma once
 #include <cstdint>
@@ -169,7 +170,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       mbar_init(xempty_bar(x), 1);
     }
     for (int a = 0; a < A_STAGES; ++a) {
-      mbar_init(dq_bar(a), DQ_WARPS);
+      mbar_init(dq_bar(a), DQ_WARPS / 2);  // the four warps of the group that writes the tile
       mbar_init(afree_bar(a), 1);
     }
     mbar_init(acc_bar, 1);
@@ -287,23 +288,27 @@ __global__ void __launch_bounds__(THREADS, 2)
   } else {
     // ------------------------------------------------------------------------------ dequantize
     const int r = (warp & 3) * 32 + lane;  // warps 2+q and 6+q both take rows 32q ...
-    const int half = (warp - 2) >> 2;      // ... and split the k-block's in-features
+    const int group = (warp - 2) >> 2;     // ... of the k-blocks i with i % 2 == group, all 8 words
     const uint32_t sw = static_cast<uint32_t>(r & 7);
-    for (int i = 0; i < nkb; ++i) {
+    for (int i = group; i < nkb; i += 2) {
       const int j = i / KB_PER_BOX, sub = i % KB_PER_BOX;
       const int c = j % C_STAGES, a = i % A_STAGES;
       if (!wait_warp(cfull_bar(c), static_cast<uint32_t>(j / C_STAGES) & 1u, p, kSiteDecodeFull)) {
         failed = 1;
         break;
       }
-      // Words 8 sub + 4 half .. +3 of row r: 16-byte chunk 2 sub + half of the row's swizzled line.
+      // Words 8 sub .. 8 sub + 7 of row r: 16-byte chunks 2 sub and 2 sub + 1 of the row's swizzled line.
       // "memory" keeps these loads ahead of the barrier arrive below that hands the box back.
-      uint32_t w[4];
+      uint32_t w[8];
       float z, stp;
       asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                    : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                   : "r"(c_tile(c) + static_cast<uint32_t>(r) * 128u + ((static_cast<uint32_t>(2 * sub) ^ sw) << 4))
+                   : "memory");
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
                    : "r"(c_tile(c) + static_cast<uint32_t>(r) * 128u +
-                         ((static_cast<uint32_t>(2 * sub + half) ^ sw) << 4))
+                         ((static_cast<uint32_t>(2 * sub + 1) ^ sw) << 4))
                    : "memory");
       asm volatile("ld.shared.f32 %0, [%1];"
                    : "=f"(stp)
@@ -313,16 +318,17 @@ __global__ void __launch_bounds__(THREADS, 2)
                    : "=f"(z)
                    : "r"(sz_tile(c) + 8u * (ROWS + r) + 4u * (sub >> 1))
                    : "memory");
-      uint32_t v[16];
-      dequant_words<4>(w, z, stp, v);  // in registers while the operand tile may still be in use
+      uint32_t v[32];
+      dequant_words<8>(w, z, stp, v);  // in registers while the operand tile may still be in use
       __syncwarp();
-      if (lane == 0 && (sub == KB_PER_BOX - 1 || i == nkb - 1)) mbar_arrive(cempty_bar(c));
+      // this warp's last k-block of the box (nkb is even, so each group has one in every box)
+      if (lane == 0 && (sub + 2 >= KB_PER_BOX || i + 2 >= nkb)) mbar_arrive(cempty_bar(c));
       const uint32_t ause = static_cast<uint32_t>(i / A_STAGES);
       if (ause > 0 && !wait_warp(afree_bar(a), (ause - 1u) & 1u, p, kSiteDecodeEmpty)) {
         failed = 1;
         break;
       }
-      store_words_sw128<4>(v, a_tile(a) + static_cast<uint32_t>(r) * 128u, r, 4 * half);
+      store_words_sw128<8>(v, a_tile(a) + static_cast<uint32_t>(r) * 128u, r, 0);
       fence_proxy_async_smem();  // the tensor cores read the tile through the async proxy
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_bar(a));
