@@ -19,8 +19,9 @@
 // and issues the MMAs; 2-9 dequantize into a 3-deep ring of K-major swizzled operand tiles in two groups
 // that take alternate k-blocks (warp 2 + q + 4g takes rows 32q..32q+31, all 64 in-features, of the
 // k-blocks i with i % 2 == g, so each warp synchronises once per 64 weights of a row), computing in
-// registers first and storing once the tile is free; warps 2-5 then read the accumulator (warp w may read tensor-memory lanes
-// 32 (w % 4) ...). All waits are bounded; a timeout is recorded in the caller's status word.
+// registers first and storing once the tile is free; warps 2-5 then read the accumulator (warp w may
+// read tensor-memory lanes 32 (w % 4) ...). All waits are bounded; a timeout is recorded in the caller's
+// status word.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
