@@ -121,3 +121,41 @@ def test_binding_fails_loudly_without_library(tmp_path):
             awq.load_library(str(tmp_path / "missing.so"))
     finally:
         awq._lib = saved
+
+
+def test_next_row_entry_points_reject_bad_arguments(lib):
+    bad8 = ctypes.c_void_p((1 << 20) + 4)  # 4-byte aligned only
+    # INT8 pack: W, K % 8, null outputs, codes alignment, flags
+    assert lib.awq_quantize_pack_int8(None, 4, 256, 256, FAKE, 0, FAKE, FAKE, None) == 1
+    assert lib.awq_quantize_pack_int8(FAKE, 4, 252, 256, FAKE, 0, FAKE, FAKE, None) == 1
+    assert lib.awq_quantize_pack_int8(FAKE, 4, 256, 256, None, 0, FAKE, FAKE, None) == 1
+    assert lib.awq_quantize_pack_int8(FAKE, 4, 256, 256, FAKE, 0, bad8, FAKE, None) == 1
+    assert lib.awq_quantize_pack_int8(FAKE, 4, 256, 256, FAKE, 0x40, FAKE, FAKE, None) == 1
+    # scale folding: operands, C % 8, s, op, in place with different strides
+    for fn in (lib.awq_scale_columns, lib.awq_scale_rows):
+        assert fn(None, 4, 256, 256, FAKE, 0, FAKE, 256, None) == 1
+        assert fn(FAKE, 4, 252, 256, FAKE, 0, FAKE, 256, None) == 1
+        assert fn(FAKE, 4, 256, 256, None, 0, FAKE, 256, None) == 1
+        assert fn(FAKE, 4, 256, 256, FAKE, 2, FAKE, 256, None) == 1
+        assert fn(FAKE, 4, 256, 256, FAKE, 1, FAKE, 264, None) == 1
+    # W4A16: shapes, codes, workspace
+    ws = lib.awq_w4a16_workspace_size(256, 256)
+    assert ws > 256 * 1024 and lib.awq_w4a16_workspace_size(64, 256) == 0
+
+    def w4(X=FAKE, M=16, K=256, ldx=256, codes=FAKE, steps=FAKE, zeros=FAKE, O=256, Y=FAKE, ldy=256, wsp=FAKE,
+           wsb=ws):
+        return lib.awq_w4a16_gemm(X, M, K, ldx, codes, steps, zeros, O, Y, ldy, wsp, wsb, None)
+
+    assert w4(X=None) == 1 and w4(Y=None) == 1
+    assert w4(M=0) == 1
+    assert w4(K=192, ldx=192) == 1          # K % 128
+    assert w4(O=252, ldy=256) == 1          # O % 8
+    assert w4(codes=None) == 1 and w4(codes=bad8) == 1 and w4(zeros=None) == 1
+    assert w4(wsp=None) == 3 and w4(wsb=ws - 1) == 3
+    rc, msg = status_and_message(lib, w4(wsb=16))
+    assert rc == 3 and "workspace" in msg
+    assert w4(wsp=bad8) == 1
+    # the allocation-free statistic: operands, and a shape beyond its fixed scratch array
+    assert lib.awq_act_stats_noalloc(None, 16, 256, 256, FAKE, None) == 1
+    assert lib.awq_act_stats_noalloc(FAKE, 16, 256, 256, None, None) == 1
+    assert lib.awq_act_stats_noalloc(FAKE, 1 << 20, 1 << 20, 1 << 20, FAKE, None) == 1
