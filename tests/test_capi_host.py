@@ -159,3 +159,15 @@ def test_next_row_entry_points_reject_bad_arguments(lib):
     assert lib.awq_act_stats_noalloc(None, 16, 256, 256, FAKE, None) == 1
     assert lib.awq_act_stats_noalloc(FAKE, 16, 256, 256, None, None) == 1
     assert lib.awq_act_stats_noalloc(FAKE, 1 << 20, 1 << 20, 1 << 20, FAKE, None) == 1
+
+
+def test_w4a16_workspace_covers_its_regions(lib):
+    # header (512 B) + the fixed few-token counter region (65536 x 4 B) + group-major steps and zeros
+    # (K/128 x O rounded up to 256, fp32, each) + split-K partial sums
+    fixed = 512 + 65536 * 4
+    for K, O in [(128, 8), (256, 256), (4096, 4096), (14336, 4096), (28672, 8192), (4096, 28672)]:
+        ws = lib.awq_w4a16_workspace_size(K, O)
+        o_pad = (O + 255) // 256 * 256
+        assert ws >= fixed + 2 * (K // 128) * o_pad * 4, (K, O, ws)
+        assert ws % 256 == 0
+    assert lib.awq_w4a16_workspace_size(127, 8) == 0 and lib.awq_w4a16_workspace_size(128, 0) == 0
