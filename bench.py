@@ -1,6 +1,6 @@
 """Benchmark of the AWQ scale search on B200: one JSON line on rank 0.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 5] [--impl ours|reference]
 
 A step is one pass of the whole path over one layer: the activation statistic, the search (scale table,
 weight-error producer, tensor-core loss GEMM, argmin) and the packed INT4 artefact at the best scales.
@@ -10,9 +10,11 @@ around its launch inside the library) for the roofline. ``e2e`` repeats the meas
 public Python API with pinned host buffers: H2D of X and W, the path, D2H of codes/steps/zeros/scales/
 losses/best_j, all inside the timed region.
 
+The default workload is 5, the largest single-GPU configuration (X 16384 x 28672, W 8192 x 28672).
+
 With N > 1 (torchrun) every rank quantizes its own layer (independent replicas, no data exchange); the
 time is the max over ranks and ``value`` counts every rank's candidates. ``--impl reference`` times the
-CPU oracle on a bounded sample of the same workload (rank 0 only).
+CPU oracle on a bounded sample of the same workload (rank 0 only), the same sample as ``cpu_baseline``.
 """
 from __future__ import annotations
 
@@ -41,7 +43,7 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--workload", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -65,22 +67,23 @@ def gemm_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "loss_gemm_traffic.json")
+
+
 def profiled_traffic(workload: int):
-    """Per-launch DRAM bytes of the loss GEMM from the committed ncu summary, if it was taken on the
-    current kernel source (same hash); otherwise None."""
-    path = os.path.join(ROOT, "profiles", f"loss_gemm_workload{workload}.md")
-    if not os.path.exists(path):
-        return None
-    src_hash, traffic = None, None
-    with open(path) as f:
-        for line in f:
-            if line.startswith("kernel_source_sha256_16:"):
-                src_hash = line.split(":", 1)[1].strip()
-            if line.startswith("dram_bytes_per_launch:"):
-                traffic = float(line.split(":", 1)[1].strip())
-    if src_hash != gemm_source_hash():
-        return None
-    return traffic
+    """Per-launch DRAM bytes (read + write) of the loss GEMM from the committed ncu summary
+    (profiles/loss_gemm_traffic.json), if it was taken on the current kernel source (same hash) for this
+    workload; otherwise (None, why)."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no ncu traffic record"
+    with open(TRAFFIC_FILE) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_sha256_16") != gemm_source_hash():
+        return None, "the loss kernel changed since its DRAM counters were taken"
+    w = rec.get("workloads", {}).get(str(workload))
+    if w is None:
+        return None, f"no ncu DRAM capture for workload {workload}"
+    return float(w["dram_bytes_per_launch"]), w.get("how", "")
 
 
 class ClockSampler:
@@ -142,45 +145,82 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------ oracle arm
-def oracle_sample(wl, X, W, j_list=None, tokens=1024):
-    """Time the oracle on a bounded sample of the workload and extrapolate to candidates/s.
+SAMPLE_TOKENS = 512   # the loss GEMM is timed on the first 512 tokens and scaled by N / 512
+SAMPLE_BLOCKS = 8     # the quantizer and the loss are timed in 8 blocks of output rows
 
-    Sample: the statistic over all N tokens; for each sampled ratio j (every other one by default) one
-    scale-table row (correctly rounded powers over K), the quantizer over the full W, and the fp64 loss
-    GEMM on the first `tokens` tokens, whose time is scaled by N / tokens (the loss GEMM is linear in N)."""
-    from oracle import awq_oracle as orc
 
-    if j_list is None:
-        j_list = range(0, wl.n_grid, 2)
-    tokens = min(tokens, wl.N)
-    t0 = time.perf_counter()
-    act = orc.act_mean(X)
-    t_act = time.perf_counter() - t0
-    t_scale = t_quant = t_loss = 0.0
-    for j in j_list:
+def _blocks(O):
+    step = -(-O // SAMPLE_BLOCKS)
+    return [(r0, min(O, r0 + step)) for r0 in range(0, O, step)]
+
+
+class OracleSample:
+    """The one bounded sample of the oracle that both ``cpu_baseline`` and ``--impl reference`` time.
+
+    For one candidate (ratio j = n_grid // 2): its scale-table row (correctly rounded powers over K), then,
+    block by block over 8 blocks of output rows, the quantizer (scale, group-quantize, dequantize,
+    unscale) on the block's rows of the full W and the fp64 loss GEMM of the first 512 tokens against the
+    block. The quantizer is thus timed in full; the loss time is scaled by N / 512 (the loss GEMM is
+    linear in N). The statistic over all N tokens is timed once. One layer of n_grid candidates is then
+    t_statistic + n_grid * (t_scale_row + sum over blocks of (t_quant + t_loss * N / 512))."""
+
+    def __init__(self, wl, X, W):
+        from oracle import awq_oracle as orc
+
+        self.orc, self.wl, self.X, self.W = orc, wl, X, W
+        self.tokens = min(SAMPLE_TOKENS, wl.N)
+        self.scale = wl.N / self.tokens
+        self.j = wl.n_grid // 2
+        self.blocks = _blocks(W.shape[0])
         t0 = time.perf_counter()
-        s = orc.scale_candidates(act, orc.ratio(j, wl.n_grid))
+        self.act = orc.act_mean(X)
+        self.t_act = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        self.s = orc.scale_candidates(self.act, orc.ratio(self.j, wl.n_grid))
+        self.t_scale = time.perf_counter() - t0
+        self.wall = self.t_act + self.t_scale
+
+    def block(self, b):
+        """Quantizer and loss for block b; returns its extrapolated seconds (loss scaled by N / tokens)."""
+        r0, r1 = self.blocks[b]
+        Wb = self.W[r0:r1]
+        t0 = time.perf_counter()
+        w_hat, _, _, _ = self.orc.pseudo_quantize(Wb, self.s)
         t1 = time.perf_counter()
-        w_hat, _, _, _ = orc.pseudo_quantize(W, s)
+        self.orc.loss_of(self.X[:self.tokens], Wb, w_hat)
         t2 = time.perf_counter()
-        orc.loss_of(X[:tokens], W, w_hat)
-        t3 = time.perf_counter()
-        t_scale += t1 - t0
-        t_quant += t2 - t1
-        t_loss += t3 - t2
-    n = len(j_list)
-    per_cand = (t_scale + t_quant + t_loss * (wl.N / tokens)) / n
-    per_layer = t_act + wl.n_grid * per_cand
-    wall = t_act + t_scale + t_quant + t_loss
+        self.wall += t2 - t0
+        return (t1 - t0) + (t2 - t1) * self.scale
+
+    def per_layer_s(self, block_times):
+        """Extrapolated seconds of one layer from the mean extrapolated block time."""
+        per_cand = self.t_scale + len(self.blocks) * float(np.mean(block_times))
+        return self.t_act + self.wl.n_grid * per_cand
+
+    def describe(self, n_block_runs):
+        wl = self.wl
+        return (f"workload {wl.number}: statistic over all {wl.N} tokens; candidate j={self.j} of {wl.n_grid}: "
+                f"scale row, then in {len(self.blocks)} blocks of output rows the quantizer over the full W "
+                f"and the fp64 loss GEMM on the first {self.tokens} tokens ({n_block_runs} block runs); loss "
+                f"time scaled by N/{self.tokens} = {self.scale:g}; extrapolated to one layer of {wl.n_grid} "
+                f"candidates")
+
+
+def oracle_sample(wl, X, W):
+    """cpu_baseline: the sample once (every block of one candidate), extrapolated to candidates/s."""
+    smp = OracleSample(wl, X, W)
+    smp.block(0)  # one untimed block first (page faults of numpy's first large temporaries)
+    times = [smp.block(b) for b in range(len(smp.blocks))]
+    per_layer = smp.per_layer_s(times)
     return {
         "value": wl.n_grid / per_layer,
         "unit": UNIT,
         "cores": int(os.cpu_count() or 1),
         "kind": "oracle",
-        "sample": (f"workload {wl.number}: statistic over all {wl.N} tokens; {n} of {wl.n_grid} ratios "
-                   f"(scale row + quantizer over full W + fp64 loss GEMM on the first {tokens} tokens, "
-                   f"loss time scaled by {wl.N}/{tokens}); extrapolated to one layer of {wl.n_grid} candidates; "
-                   f"sample wall {wall:.1f} s"),
+        "sample": smp.describe(len(times)) + " (after one untimed warm-up block)",
+        "extrapolated": True,
+        "sample_wall_s": smp.wall,
+        "loss_scale_factor": smp.scale,
         "threads": _blas_threads(),
     }
 
@@ -195,29 +235,34 @@ def _blas_threads():
 
 
 def run_reference(args, rank, world):
+    """The oracle as the reference arm: the same sample as cpu_baseline, one block of output rows per step
+    (blocks in turn), so a step is a bounded piece of one candidate's work."""
     from weight_only_quantization_act_b200 import inputs
 
     if rank != 0:
         return
     wl = inputs.workload(args.workload)
     X, W, _ = inputs.make_inputs(wl)
-    for _ in range(args.warmup):
-        oracle_sample(wl, X, W, j_list=(0,), tokens=256)
-    vals, t_total = [], 0.0
-    res = None
-    for k in range(args.steps):
-        t0 = time.perf_counter()
-        res = oracle_sample(wl, X, W, j_list=((5 * k) % wl.n_grid,), tokens=256)
-        t_total += time.perf_counter() - t0
-        vals.append(res["value"])
-    value = float(np.mean(vals))
+    smp = OracleSample(wl, X, W)
+    nb = len(smp.blocks)
+    for k in range(args.warmup):
+        smp.block(k % nb)
+    wall0 = smp.wall
+    times = [smp.block((args.warmup + k) % nb) for k in range(args.steps)]
+    per_layer = smp.per_layer_s(times)
+    value = wl.n_grid / per_layer
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.n_grid / value,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * (smp.wall - wall0) / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(wl, args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": res["cores"], "kind": "oracle",
-                         "sample": res["sample"]},
+        "extrapolated": True,
+        "ms_per_step_is": "measured wall time of one sample step (one block of output rows of one candidate)",
+        "layer_ms_extrapolated": 1e3 * per_layer,
+        "sample_wall_s": smp.wall - wall0,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(os.cpu_count() or 1), "kind": "oracle",
+                         "sample": smp.describe(len(times)), "extrapolated": True,
+                         "sample_wall_s": smp.wall, "loss_scale_factor": smp.scale},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -323,7 +368,7 @@ def run_ours(args, rank, world, local_rank):
     flops = J * 2.0 * N * O * K
     gemm_avg_s = float(np.mean(gemm_ms)) / 1e3
     achieved_tflops = flops / gemm_avg_s / 1e12
-    traffic = profiled_traffic(wl.number)
+    traffic, traffic_how = profiled_traffic(wl.number)
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         cpu = oracle_sample(wl, X, W)
@@ -342,7 +387,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac_of_sustained": achieved_tflops / peaks["bf16_tflops_sustained"],
                      "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)" if peaks_src == "measured"
                      else "fallback 1.59 PFLOP/s",
-                     "traffic": traffic, "algorithmic_flops_per_launch": flops},
+                     "traffic": traffic, "traffic_source": traffic_how, "algorithmic_flops_per_launch": flops},
         "hbm": {"act_stats_gbs": (2.0 * N * K + 4.0 * K) / (np.mean(act_ms) / 1e3) / 1e9,
                 "quantize_pack_gbs": (2.0 * O * K + 4.0 * K + O * K / 2.0 + 8.0 * O * K / 128)
                 / (np.mean(pack_ms) / 1e3) / 1e9,
@@ -350,11 +395,7 @@ def run_ours(args, rank, world, local_rank):
                 "int8_pack_gbs": (2.0 * O * K + 4.0 * K + 1.0 * O * K + 4.0 * O) / (int8_pack_ms / 1e3) / 1e9,
                 "peak_gbs": peaks.get("hbm_gbs")},
         "search_ms_by_rule": rules_ms,
-        "w4a16": {"prefill_tokens": N, "prefill_ms": w4["prefill_ms"],
-                  "prefill_tflops": 2.0 * N * O * K / (w4["prefill_ms"] / 1e3) / 1e12,
-                  "prefill_frac_of_peak": 2.0 * N * O * K / (w4["prefill_ms"] / 1e3) / 1e12 / peaks["bf16_tflops"],
-                  "decode_tokens": 16, "decode_ms": w4["decode_ms"],
-                  "decode_weight_gbs": (0.5 * O * K + 8.0 * O * K / 128) / (w4["decode_ms"] / 1e3) / 1e9},
+        "w4a16": w4a16_summary(w4, peaks),
         "gpu_launches": launches_per_step(J) * args.steps,
         "clocks": clocks,
         "best_j": best,
@@ -398,8 +439,10 @@ def measure_rules(Xd, Wd, act, J):
     from weight_only_quantization_act_b200 import awq
 
     out = {}
+    N, K = Xd.shape
+    ws = awq._workspace(awq.search_workspace_size(N, K, Wd.shape[0], J), Xd.device, None)  # shared by all rules
     for rule, n, quant in (("p4", J, "int4"), ("weight_aware", J, "int4"), ("rms", 11, "int4"), ("p4", J, "int8")):
-        res = awq.search(Xd, Wd, act, n_grid=n, rule=rule, quant=quant)
+        res = awq.search(Xd, Wd, act, n_grid=n, rule=rule, quant=quant, workspace=ws)
         times = []
         for i in range(4):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -434,21 +477,21 @@ def measure_int8_pack(Wd, scales):
 
 
 def measure_w4a16(Xd, Wd, scales):
-    """The deployment GEMM on the quantized layer: a prefill of all N calibration tokens and a 16-token
-    decode step. Each is timed cold: 40 launches, each after a 512 MiB L2 flush, between two events,
-    minus 40 flushes alone timed just before (single launches would be read off an event clock that ticks
-    in ~2 us steps); the median over seven such pairs."""
+    """The deployment GEMM on the quantized layer, and a dense bf16 GEMM (torch.matmul) of the same shapes
+    on the same harness as a comparator (measurement only): a prefill of all N calibration tokens, a
+    16-token decode on the whole layer, and a 16-token decode on its first 4096 rows and in-features.
+    Each is timed cold: a batch of launches, each after a 512 MiB L2 flush, between two events, minus a
+    batch of flushes alone timed just before (single launches of a few microseconds would be read off an
+    event clock that ticks in ~2 us steps); the median over seven such pairs. Batches hold 40 launches,
+    fewer for launches longer than 0.1 ms."""
     import torch
 
     from weight_only_quantization_act_b200 import awq
 
-    codes, steps, zeros = awq.quantize_pack(Wd, scales)
-    Xs = awq.scale_columns(Xd, scales, divide=True)
+    lib = awq.load_library()
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=Xd.device)
-    ws = torch.zeros(awq.load_library().awq_w4a16_workspace_size(Xd.shape[1], codes.shape[0]), dtype=torch.uint8,
-                     device=Xd.device)
 
-    def batch(fn, n=40):
+    def batch(fn, n):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(n):
@@ -459,19 +502,57 @@ def measure_w4a16(Xd, Wd, scales):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n
 
-    out = {}
-    for name, X in (("prefill_ms", Xs), ("decode_ms", Xs[:16].contiguous())):
-        Y = torch.empty((X.shape[0], codes.shape[0]), dtype=torch.bfloat16, device=Xd.device)
-        fn = lambda X=X, Y=Y: awq.w4a16_gemm(X, codes, steps, zeros, out=Y, workspace=ws)
-        batch(fn, 4)
-        batch(None, 4)
+    def cold_ms(fn):
+        n = 4
+        est = batch(fn, n) - batch(None, n)
+        n = int(max(3, min(40, 4.0 / max(est, 1e-3))))  # ~4 ms of kernel time per batch
         # flush-only and flush+kernel batches alternate, so a drift of the flush time cancels in each
         # pair; the median of the pairs' differences is the kernel time
         diffs = []
         for _ in range(7):
-            base = batch(None)
-            diffs.append(batch(fn) - base)
-        out[name] = float(np.median(diffs))
+            base = batch(None, n)
+            diffs.append(batch(fn, n) - base)
+        return float(np.median(diffs))
+
+    out = {}
+    layers = [("", Xd, Wd, scales)]
+    if Xd.shape[1] > 4096 or Wd.shape[0] > 4096:
+        Ks, Os = min(4096, Xd.shape[1]), min(4096, Wd.shape[0])
+        layers.append(("small_", Xd[:, :Ks].contiguous(), Wd[:Os, :Ks].contiguous(), scales[:Ks].contiguous()))
+    for prefix, X, W, s in layers:
+        codes, steps, zeros = awq.quantize_pack(W, s)
+        Xs = awq.scale_columns(X, s, divide=True)
+        ws = torch.zeros(lib.awq_w4a16_workspace_size(X.shape[1], codes.shape[0]), dtype=torch.uint8,
+                         device=X.device)
+        cases = (("decode", Xs[:16].contiguous()),) if prefix else (("prefill", Xs), ("decode", Xs[:16].contiguous()))
+        for name, A in cases:
+            Y = torch.empty((A.shape[0], codes.shape[0]), dtype=torch.bfloat16, device=X.device)
+            fn = lambda A=A, Y=Y: awq.w4a16_gemm(A, codes, steps, zeros, out=Y, workspace=ws)
+            ref = lambda A=A, Y=Y, W=W: torch.matmul(A, W.t(), out=Y)
+            out[f"{prefix}{name}_ms"] = cold_ms(fn)
+            out[f"{prefix}{name}_bf16_ms"] = cold_ms(ref)
+            out[f"{prefix}{name}_shape"] = [int(A.shape[0]), int(X.shape[1]), int(codes.shape[0])]
+    return out
+
+
+def w4a16_summary(w4, peaks):
+    """Rates of the W4A16 launches: prefill in TFLOP/s, decodes in HBM GB/s of their algorithmic bytes
+    (codes O*K/2, steps and zeros 8*O*K/128, X' 2*M*K, Y 2*M*O), each beside the bf16 comparator."""
+    out = {"comparator": "torch.matmul bf16 on the same shapes and harness (measurement only)"}
+    M, K, O = w4["prefill_shape"]
+    out.update({"prefill_shape_MKO": [M, K, O], "prefill_ms": w4["prefill_ms"], "prefill_bf16_ms": w4["prefill_bf16_ms"],
+                "prefill_tflops": 2.0 * M * O * K / (w4["prefill_ms"] / 1e3) / 1e12})
+    out["prefill_frac_of_peak"] = out["prefill_tflops"] / peaks["bf16_tflops"]
+    for prefix in ("", "small_"):
+        if f"{prefix}decode_ms" not in w4:
+            continue
+        M, K, O = w4[f"{prefix}decode_shape"]
+        nbytes = 0.5 * O * K + 8.0 * O * K / 128 + 2.0 * M * K + 2.0 * M * O
+        ms = w4[f"{prefix}decode_ms"]
+        out.update({f"{prefix}decode_shape_MKO": [M, K, O], f"{prefix}decode_ms": ms,
+                    f"{prefix}decode_bf16_ms": w4[f"{prefix}decode_bf16_ms"],
+                    f"{prefix}decode_gbs": nbytes / (ms / 1e3) / 1e9,
+                    f"{prefix}decode_frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]})
     return out
 
 

@@ -68,7 +68,8 @@ typedef enum awq_status {
 } awq_status;
 
 /* Flags for the *_ex entry points (0 = the production behaviour of the plain entry points). */
-#define AWQ_FLAG_EXACT_DIVISION 0x1u /* every w'/step quotient by IEEE division, no reciprocal fast path */
+#define AWQ_FLAG_EXACT_DIVISION 0x1u /* every w'/step quotient by IEEE division, no reciprocal fast path;
+                                        in the search also the unscale w_hat = RN32(deq / s) */
 #define AWQ_FLAG_EXACT_POW 0x2u      /* every act_mean^ratio by the double-double path, no fp64 pow */
 #define AWQ_FLAG_INJECT_STALL 0x100u /* test hook: the loss GEMM waits on a barrier nobody signals */
 /* Candidate-scale rule of the search (default: 原理 on the msModelSlim page, see (2) below). */
@@ -96,7 +97,8 @@ AWQ_API void awq_set_wait_limit_ns(uint64_t ns);
  *   X         device, bf16 [N, K], row stride ldx (elements)
  *   workspace device, >= awq_act_stats_workspace_size(N, K) bytes, contents need not be initialised
  *   act_mean  device, float [K] (output)
- * Requires N >= 1, K >= 1, K % 2 == 0.
+ * Requires N >= 1, K >= 1, K % 2 == 0 and ceil(N / 256) <= 65535 (N <= 16,776,960), else
+ * AWQ_ERR_INVALID_ARG before any launch.
  * ------------------------------------------------------------------------------------------------- */
 AWQ_API size_t awq_act_stats_workspace_size(int64_t N, int64_t K);
 AWQ_API awq_status awq_act_stats(const void *X, int64_t N, int64_t K, int64_t ldx, void *workspace,
@@ -115,6 +117,9 @@ AWQ_API awq_status awq_act_stats(const void *X, int64_t N, int64_t K, int64_t ld
  *   (e.g. N = 16384 with K <= 32768, or N = 4096 with K <= 131072).
  *   The first call on each device looks up the array's device address (cudaGetSymbolAddress, which may
  *   load the library's device code on that device); make that first call before any stream capture.
+ *   The address is kept per device and CUDA context: after cudaDeviceReset (a new primary context, in
+ *   which the library's device code and the array are loaded afresh) the next call looks it up again,
+ *   so that call too belongs before any capture.
  *   All calls share the one array, which keeps the last call's contents (every value a call reads is
  *   first written by that call, so nothing needs clearing): calls that overlap on the GPU, e.g. on two
  *   streams, race and give wrong results. Serialise them.

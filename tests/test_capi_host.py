@@ -102,6 +102,15 @@ def test_other_entry_points_reject_bad_arguments(lib):
     assert lib.awq_act_stats(FAKE, 10, 255, 256, FAKE, 1 << 20, FAKE, None) == 1
     assert lib.awq_act_stats(FAKE, 10, 256, 256, FAKE, 8, FAKE, None) == 3
     assert lib.awq_act_stats(FAKE, 0, 256, 256, FAKE, 1 << 20, FAKE, None) == 1
+    # more than 65535 chunks of 256 rows (the chunk-sum grid's y extent): rejected before any launch
+    rows = 65535 * 256 + 1
+    assert lib.awq_act_stats(FAKE, rows, 2, 8, FAKE, 1 << 30, FAKE, None) == 1
+    assert "65535 chunks" in lib.awq_last_error().decode()
+    assert lib.awq_act_stats_noalloc(FAKE, rows, 2, 8, FAKE, None) == 1
+    assert "65535 chunks" in lib.awq_last_error().decode()
+    assert lib.awq_search_ex(FAKE, 512, 256, 256, FAKE, rows, 256, FAKE, 128, 20, 0x10, FAKE, 1 << 40, FAKE, FAKE,
+                             FAKE, None) == 1
+    assert "65535 chunks" in lib.awq_last_error().decode()
     assert lib.awq_quantize_pack(FAKE, 4, 256, 256, FAKE, 32, FAKE, FAKE, FAKE, None) == 2
     assert lib.awq_quantize_pack(FAKE, 4, 192, 192, FAKE, 128, FAKE, FAKE, FAKE, None) == 1
     assert lib.awq_quantize_pack(FAKE, 4, 256, 256, None, 128, FAKE, FAKE, FAKE, None) == 1

@@ -182,15 +182,30 @@ def test_search_on_grid_weight_zero_loss_at_ratio_zero():
 
 
 def test_search_flags_do_not_change_results():
+    """The exact paths (IEEE division for every quotient and for the unscale w_hat = deq / s, the
+    double-double power for every scale) give the same scales, argmin, codes, steps and zeros; the losses
+    move by at most the bf16 rounding of a weight error that changed by one fp32 ulp, and stay within the
+    tolerance of the oracle, whose unscale is the IEEE division."""
     X = inputs.random_bf16((384, 512), seed=51, outliers=3, factor=40)
     W = inputs.random_bf16((512, 512), seed=52, scale=0.02)
     Xd, Wd = bf16_to_device(X), bf16_to_device(W)
     act = awq.act_stats(Xd)
+    ref = orc.search(X, W, n_grid=20)
     a = awq.search(Xd, Wd, act)
     b = awq.search(Xd, Wd, act, flags=awq.FLAG_EXACT_DIVISION | awq.FLAG_EXACT_POW)
     c = awq.search(Xd, Wd, act)
-    assert torch.equal(a.losses, b.losses) and torch.equal(a.losses, c.losses), "search must be deterministic"
+    d = awq.search(Xd, Wd, act, flags=awq.FLAG_EXACT_DIVISION | awq.FLAG_EXACT_POW)
+    assert torch.equal(a.losses, c.losses) and torch.equal(b.losses, d.losses), "search must be deterministic"
     assert torch.equal(a.scales, b.scales) and int(a.best_j.item()) == int(b.best_j.item())
+    for res in (a, b):
+        err = loss_rel_err(res.losses.cpu().numpy(), ref["losses"])
+        assert np.all(err <= LOSS_RTOL), err.max()
+        check_argmin_rule(int(res.best_j.item()), ref["losses"])
+    assert np.all(loss_rel_err(b.losses.cpu().numpy(), a.losses.cpu().numpy()) <= 1e-3)
+    pa = awq.quantize_pack(Wd, a.scales)
+    pb = awq.quantize_pack(Wd, b.scales, flags=awq.FLAG_EXACT_DIVISION)
+    for x, y in zip(pa, pb):
+        assert torch.equal(x, y)
 
 
 def test_tile_partials_match_oracle():

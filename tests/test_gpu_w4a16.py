@@ -47,6 +47,21 @@ def test_w4a16_matches_oracle(M, K, O):
     check_against_oracle(Xp, words, steps, zeros, Y)
 
 
+# Many tokens at the tile counts the prefill kernel really runs: tiles of 512 tokens x 256 weight rows
+# handed out dynamically over the device's CTA pairs (74 on B200), so most pairs run a second and a
+# third tile. This is where the one-tile-ahead index publishing, the code ring across tiles and the
+# accumulator handover after the epilogue are exercised: 4096^3 is 128 tiles, 4096 x 1024 x 4096 the same
+# tile count with a short K loop, and 2600 x 512 x 4104 (ragged in tokens and rows) 102 tiles.
+@pytest.mark.parametrize("M,K,O", [(4096, 4096, 4096), (4096, 1024, 4096), (2600, 512, 4104)])
+def test_w4a16_prefill_many_tiles_per_pair(M, K, O):
+    _, _, (words, steps, zeros) = quantized(O, K, M + 2 * K + O)
+    Xp = inputs.random_bf16((M, K), 5 * M + 9, scale=1.0)
+    Y = awq.w4a16_gemm(bf16_to_device(Xp), torch.from_numpy(words.view(np.int32)).cuda(),
+                       torch.from_numpy(steps).cuda(), torch.from_numpy(zeros).cuda())
+    torch.cuda.synchronize()
+    check_against_oracle(Xp, words, steps, zeros, Y)
+
+
 def test_deploy_path_end_to_end():
     """search -> pack -> fold the scales out of X -> W4A16 GEMM reproduces X W^T up to the quantization
     error the search measured (mean squared output error within 25% of the search's best loss)."""
@@ -63,9 +78,10 @@ def test_deploy_path_end_to_end():
 
 
 # ------------------------------------------------------------------------------------------------ few tokens
-# M <= 64 runs the decode kernel (weight rows on the MMA's M side, K split over a cluster of up to 8 CTAs,
-# partial sums reduced in distributed shared memory); the shapes cover cluster sizes 2, 4 and 8, CTAs of
-# a cluster left without k-blocks (K = 384, 640), ragged weight-row blocks and every token rounding.
+# M <= 64 runs the decode kernel (weight rows on the MMA's M side, k-blocks split into slices over
+# independent CTAs whose fp32 partial sums go to the workspace, where the last CTA of a row block adds
+# them in slice order); the shapes cover several slice counts, slices left without k-blocks (K = 384,
+# 640), ragged weight-row blocks and every token rounding.
 @pytest.mark.parametrize("M,K,O", [(1, 4096, 4096), (5, 384, 600), (16, 256, 136), (17, 1024, 520),
                                    (33, 640, 264), (64, 2048, 1024), (64, 128, 8), (65, 512, 256)])
 def test_w4a16_few_tokens_match_oracle(M, K, O):
@@ -86,7 +102,7 @@ def test_w4a16_few_tokens_deterministic_and_strided():
     a = awq.w4a16_gemm(Xd, *args)
     b = awq.w4a16_gemm(Xd, *args)
     torch.cuda.synchronize()
-    assert torch.equal(a, b), "the cluster reduction adds the partial sums in a fixed order"
+    assert torch.equal(a, b), "the split-K reduction adds the slices' partial sums in a fixed order"
     check_against_oracle(np.ascontiguousarray(wide[:, 128:2176]), words, steps, zeros, a)
 
 
@@ -110,10 +126,11 @@ def test_w4a16_huge_zero_points(M):
     check_against_oracle(Xp, words, steps, zeros, Y)
 
 
-@pytest.mark.parametrize("M,K,O", [(513, 4096, 1032), (1024, 2048, 768), (16, 4096, 1024)])
+@pytest.mark.parametrize("M,K,O", [(513, 4096, 1032), (1024, 2048, 768), (16, 4096, 1024), (4096, 4096, 4096)])
 def test_w4a16_repeated_runs_are_bit_identical(M, K, O):
     """Both kernels add in a fixed order, so any run-to-run difference is a race (a buffer handed back
-    or reused too early); many k-blocks per tile and repeated launches give one room to show."""
+    or reused too early); many k-blocks per tile and repeated launches give one room to show. 4096^3 runs
+    128 tiles on the CTA pairs, so pairs hand tiles over to their next tile many times."""
     _, _, (words, steps, zeros) = quantized(O, K, 5 * M + K + O)
     Xp = inputs.random_bf16((M, K), 13 * M + 3, scale=1.0)
     Xd = bf16_to_device(Xp)

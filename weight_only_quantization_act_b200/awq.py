@@ -11,6 +11,7 @@ Tensors: X is a CUDA bfloat16 [N, K] matrix (tokens x in-features), W a CUDA bfl
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 from dataclasses import dataclass
 from typing import Sequence
@@ -116,6 +117,32 @@ def _bf16_matrix(name: str, t: torch.Tensor) -> torch.Tensor:
     return t
 
 
+def _float_vector_out(name: str, out: torch.Tensor, n: int, device) -> torch.Tensor:
+    """A caller-given float32 output of at least n elements, contiguous, on `device`: the kernels write n
+    floats from its first element."""
+    if (not isinstance(out, torch.Tensor) or out.dtype != torch.float32 or not out.is_cuda
+            or out.device != device or out.numel() < n or not out.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA float32 tensor of at least {n} elements on {device}")
+    return out
+
+
+def _on_device(fn):
+    """Run an entry point with its first tensor argument's device current, so that the library launches
+    there and the stream passed is that device's current stream."""
+
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        first = args[0] if args else next(iter(kwargs.values()))
+        if isinstance(first, (list, tuple)):
+            first = first[0]
+        if isinstance(first, torch.Tensor) and first.is_cuda:
+            with torch.cuda.device(first.device):
+                return fn(*args, **kwargs)
+        return fn(*args, **kwargs)
+
+    return wrapper
+
+
 def _workspace(nbytes: int, device, workspace: torch.Tensor | None) -> torch.Tensor:
     if workspace is not None:
         if workspace.numel() * workspace.element_size() < nbytes:
@@ -152,6 +179,7 @@ def act_stats_workspace_size(N: int, K: int) -> int:
     return load_library().awq_act_stats_workspace_size(N, K)
 
 
+@_on_device
 def act_stats(X: torch.Tensor, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
               stream=None) -> torch.Tensor:
     """act_mean[k] = mean_i |X[i,k]| (fixed-order fp64 sum, rounded to fp32)."""
@@ -160,25 +188,33 @@ def act_stats(X: torch.Tensor, out: torch.Tensor | None = None, workspace: torch
     N, K = X.shape
     if out is None:
         out = torch.empty(K, dtype=torch.float32, device=X.device)
+    _float_vector_out("out", out, K, X.device)
     ws = _workspace(lib.awq_act_stats_workspace_size(N, K), X.device, workspace)
     _check("awq_act_stats", lib.awq_act_stats(_ptr(X), N, K, X.stride(0), _ptr(ws), ws.numel(), _ptr(out),
                                               _stream(stream)))
     return out
 
 
+@_on_device
 def act_stats_noalloc(X: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
     """Same statistic with no workspace, for callers that cannot allocate device memory at call time
     (the scratch is a fixed 16 MiB array inside the library; ceil(N/256)*K <= 2**21). ``out`` must be
-    preallocated; calls that overlap on the GPU race on the shared scratch."""
+    preallocated; calls that overlap on the GPU race on the shared scratch. Nothing is allocated here
+    either: X must already have unit column stride (no contiguous copy is made)."""
     lib = load_library()
-    X = _bf16_matrix("X", X)
+    if not isinstance(X, torch.Tensor) or X.dtype != torch.bfloat16 or not X.is_cuda or X.dim() != 2:
+        raise TypeError("X must be a CUDA bfloat16 matrix")
+    if X.stride(1) != 1:
+        raise ValueError("X must have unit column stride (this entry point makes no copy)")
     N, K = X.shape
+    _float_vector_out("out", out, K, X.device)
     _check("awq_act_stats_noalloc", lib.awq_act_stats_noalloc(_ptr(X), N, K, X.stride(0), _ptr(out),
                                                               _stream(stream)))
     return out
 
 
 # --------------------------------------------------------------------------------------------- (2)
+@_on_device
 def scale_table(act_mean: torch.Tensor, n_grid: int = 20, exact_pow: bool = False, rule: str = "p4",
                 weight_mean: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """float32 [n_grid, K] table of candidate scales; rule "p4" (default), "weight_aware" (needs
@@ -228,6 +264,7 @@ def search_layout(N: int, K: int, O: int, n_grid: int = 20, group: int = 128) ->
     return lay
 
 
+@_on_device
 def search(X: torch.Tensor, W, act_mean: torch.Tensor, n_grid: int = 20, group: int = 128, flags: int = 0,
            workspace: torch.Tensor | None = None, out: SearchResult | None = None, rule: str = "p4",
            quant: str = "int4", stream=None) -> SearchResult:
@@ -274,6 +311,7 @@ def tile_partials(result: SearchResult, N: int, K: int, O: int, n_grid: int = 20
 
 
 # --------------------------------------------------------------------------------------------- (5)
+@_on_device
 def quantize_pack(W: torch.Tensor, scales: torch.Tensor, group: int = 128, flags: int = 0, stream=None):
     """(codes uint32 [O, K/8] as int32 storage, steps float32 [O, K/g], zeros float32 [O, K/g])."""
     lib = load_library()
@@ -288,6 +326,7 @@ def quantize_pack(W: torch.Tensor, scales: torch.Tensor, group: int = 128, flags
     return codes, steps, zeros
 
 
+@_on_device
 def quantize_pack_int8(W: torch.Tensor, scales: torch.Tensor, flags: int = 0, stream=None):
     """(codes int8 [O, K], steps float32 [O]): symmetric INT8, one step per output channel."""
     lib = load_library()
@@ -300,6 +339,7 @@ def quantize_pack_int8(W: torch.Tensor, scales: torch.Tensor, flags: int = 0, st
     return codes, steps
 
 
+@_on_device
 def quantize_layer(X: torch.Tensor, W, n_grid: int = 20, group: int = 128, stream=None):
     """The whole path for one layer: statistic, search, and the packed artefact at the best scales."""
     act = act_stats(X, stream=stream)
@@ -320,6 +360,7 @@ def _as_matrix(t: torch.Tensor) -> torch.Tensor:
     return t.view(1, -1) if t.dim() == 1 else t
 
 
+@_on_device
 def scale_columns(A: torch.Tensor, s: torch.Tensor, divide: bool = False, out: torch.Tensor | None = None,
                   stream=None) -> torch.Tensor:
     """out[r, c] = bf16(A[r, c] * s[c]) (or / s[c]); a 1-D tensor is one row. ``out=A`` works in place."""
@@ -335,6 +376,7 @@ def scale_columns(A: torch.Tensor, s: torch.Tensor, divide: bool = False, out: t
     return out
 
 
+@_on_device
 def scale_rows(A: torch.Tensor, s: torch.Tensor, divide: bool = False, out: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
     """out[r, c] = bf16(A[r, c] * s[r]) (or / s[r]); a 1-D tensor is scaled element-wise."""
@@ -370,6 +412,7 @@ def fold_linear_linear(w1: torch.Tensor, b1: torch.Tensor | None, w2: torch.Tens
 
 
 # --------------------------------------------------------------------------------------------- (7)
+@_on_device
 def w4a16_gemm(X: torch.Tensor, codes: torch.Tensor, steps: torch.Tensor, zeros: torch.Tensor,
                out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Y = X' deq(W)^T (bf16 [M, O]) from packed codes [O, K/8], steps and zeros [O, K/128]."""

@@ -44,6 +44,7 @@ awq_status ok() {
   } while (0)
 
 struct DeviceInfo {
+  unsigned long long ctx_id = 0;  // CUDA context the cached state below belongs to
   int sms = 0;
   int cc_major = 0;
   bool gemm_attr_set = false;
@@ -55,13 +56,56 @@ constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
+using PFN_ctx_get_current = CUresult (*)(CUcontext*);
+using PFN_ctx_get_id = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<F>(p);
+}
+
+// The current device and the unique id of its current CUDA context. Per-device state cached by this
+// file (function attributes, the no-alloc scratch address) belongs to one context: after cudaDeviceReset
+// the primary context is created anew, the library's device code is loaded into it again, and the
+// cached state must be rebuilt. cudaSetDevice on the current device makes its primary context current
+// (creating it if needed) without allocating anything.
+awq_status current_context(int* dev, unsigned long long* ctx_id) {
+  static PFN_ctx_get_current get_current = nullptr;
+  static PFN_ctx_get_id get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    get_current = driver_fn<PFN_ctx_get_current>("cuCtxGetCurrent");
+    get_id = driver_fn<PFN_ctx_get_id>("cuCtxGetId");
+  });
+  AWQ_CUDA(cudaGetDevice(dev));
+  if (*dev < 0 || *dev >= kMaxDevices) return fail(AWQ_ERR_UNSUPPORTED, "device index %d out of range", *dev);
+  AWQ_CUDA(cudaSetDevice(*dev));
+  if (get_current == nullptr || get_id == nullptr)
+    return fail(AWQ_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId not available from the driver");
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+    return fail(AWQ_ERR_CUDA, "no current CUDA context on device %d", *dev);
+  if (get_id(ctx, ctx_id) != CUDA_SUCCESS) return fail(AWQ_ERR_CUDA, "cuCtxGetId failed on device %d", *dev);
+  return AWQ_OK;
+}
+
 awq_status device_info(DeviceInfo** out) {
   int dev = 0;
-  AWQ_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return fail(AWQ_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  unsigned long long ctx_id = 0;
+  {
+    awq_status s = current_context(&dev, &ctx_id);
+    if (s != AWQ_OK) return s;
+  }
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DeviceInfo& d = g_dev[dev];
+  if (d.ctx_id != ctx_id) d = DeviceInfo{};  // a new context: attributes are set again
   if (d.sms == 0) {
+    d.ctx_id = ctx_id;
     AWQ_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
     AWQ_CUDA(cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev));
   }
@@ -246,6 +290,15 @@ awq_status check_matrix(const char* name, const void* p, int64_t rows, int64_t K
   return AWQ_OK;
 }
 
+// The chunk-sum kernel runs one grid row per 256-row chunk; a grid's y extent is at most 65535.
+awq_status check_act_chunks(const char* name, int64_t rows) {
+  const int64_t n_chunks = (rows + awq::kActChunk - 1) / awq::kActChunk;
+  if (n_chunks > 65535)
+    return fail(AWQ_ERR_INVALID_ARG, "%s has %lld rows: at most 65535 chunks of %d (%lld rows) are supported", name,
+                static_cast<long long>(rows), awq::kActChunk, 65535ll * awq::kActChunk);
+  return AWQ_OK;
+}
+
 awq_status check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(AWQ_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
@@ -300,6 +353,7 @@ awq_status awq_act_stats(const void* X, int64_t N, int64_t K, int64_t ldx, void*
   AWQ_TRY(check_matrix("X", X, N, K, ldx));
   if (K % 2 != 0) return fail(AWQ_ERR_INVALID_ARG, "K must be even");
   if (act_mean == nullptr) return fail(AWQ_ERR_INVALID_ARG, "act_mean is null");
+  AWQ_TRY(check_act_chunks("X", N));
   const ActLayout l = act_layout(N, K);
   if (workspace == nullptr || ws_bytes < l.bytes)
     return fail(AWQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", l.bytes, workspace ? ws_bytes : 0);
@@ -390,6 +444,7 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
     return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if ((flags & AWQ_FLAG_SCALES_WEIGHT_AWARE) && (flags & AWQ_FLAG_SCALES_RMS))
     return fail(AWQ_ERR_INVALID_ARG, "choose one candidate-scale rule");
+  if (flags & AWQ_FLAG_SCALES_WEIGHT_AWARE) AWQ_TRY(check_act_chunks("W", O));  // mean |W| per column
   const SearchLayout l = search_layout(N, K, O, n_grid);
   if (static_cast<int64_t>(n_grid) * l.O_pad >= (1ll << 31))
     return fail(AWQ_ERR_INVALID_ARG, "n_grid * O is too large");
@@ -603,24 +658,28 @@ namespace {
 
 struct ScratchSlot {
   bool ready = false;
+  unsigned long long ctx_id = 0;  // the context the address belongs to
   double* ptr = nullptr;
 };
 ScratchSlot g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
 
+// The array's device address in the current device's current context, looked up on the first call in
+// that context (the device is current here, as cudaGetSymbolAddress requires).
 awq_status act_scratch_address(double** out) {
   int dev = 0;
-  AWQ_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return fail(AWQ_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  unsigned long long ctx_id = 0;
+  AWQ_TRY(current_context(&dev, &ctx_id));
   std::lock_guard<std::mutex> lk(g_scratch_mu);
   ScratchSlot& slot = g_scratch[dev];
-  if (!slot.ready) {
+  if (!slot.ready || slot.ctx_id != ctx_id) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, awq_act_scratch);
     if (e != cudaSuccess || p == nullptr)
       return fail(AWQ_ERR_CUDA, "cudaGetSymbolAddress of the no-alloc scratch failed on device %d: %s", dev,
                   cudaGetErrorString(e));
     slot.ptr = static_cast<double*>(p);
+    slot.ctx_id = ctx_id;
     slot.ready = true;
   }
   *out = slot.ptr;
@@ -634,6 +693,7 @@ extern "C" awq_status awq_act_stats_noalloc(const void* X, int64_t N, int64_t K,
   AWQ_TRY(check_matrix("X", X, N, K, ldx));
   if (K % 2 != 0) return fail(AWQ_ERR_INVALID_ARG, "K must be even");
   if (act_mean == nullptr) return fail(AWQ_ERR_INVALID_ARG, "act_mean is null");
+  AWQ_TRY(check_act_chunks("X", N));
   const ActLayout l = act_layout(N, K);
   const uint64_t need = static_cast<uint64_t>(l.n_chunks) * static_cast<uint64_t>(K);
   if (need > AWQ_NOALLOC_SCRATCH_DOUBLES)

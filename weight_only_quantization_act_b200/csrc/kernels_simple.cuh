@@ -224,7 +224,8 @@ __global__ void __launch_bounds__(kScaleThreads) scale_normalize_kernel(float* _
 // GEMM (row j * O_pad + o, K contiguous); rows o >= O are written as zeros. A work item is 512
 // consecutive in-features (a segment) of one row, done by one warp: each lane owns 16 in-features
 // (8 lanes per group of 128). The producer warps of the loss-GEMM kernel call produce_rows.
-// w_hat = deq * RN32(1/s) here (within one fp32 rounding of deq / s; it only feeds the loss).
+// w_hat = deq * RN32(1/s) by default (within one fp32 rounding of deq / s; it only feeds the loss);
+// with AWQ_FLAG_EXACT_DIVISION it is the IEEE quotient RN32(deq / s) of the method's unscale step.
 // ===================================================================================================
 constexpr int kProdCols = 16;
 constexpr int kProdWarpCols = 32 * kProdCols;  // 512
@@ -239,6 +240,11 @@ struct ProducerArgs {
   int keep_w;                      // W is re-read once per candidate: ask L2 to keep it (evict_last)
   const float* rowstep;            // INT8 per-channel quantizer: [n_grid][O_pad] steps, else null
 };
+
+// w_hat from the dequantized value: deq * RN32(1/s), or the IEEE quotient deq / s when exact.
+__device__ __forceinline__ float unscale(float deq, float s, float rs, bool exact) {
+  return exact ? __fdiv_rn(deq, s) : __fmul_rn(deq, rs);
+}
 
 // Weight errors of one row of one 512-in-feature segment for candidate j, from the row's raw bf16 words.
 __device__ __forceinline__ void produce_row(const ProducerArgs& a, const uint4 (&u)[2], const float (&s)[kProdCols],
@@ -271,8 +277,8 @@ __device__ __forceinline__ void produce_row(const ProducerArgs& a, const uint4 (
 #pragma unroll
     for (int i = 0; i < kProdCols; i += 2) {
       const float q0 = code_of_int8(wp[i], g, a.exact != 0), q1 = code_of_int8(wp[i + 1], g, a.exact != 0);
-      const float h0 = __fmul_rn(__fmul_rn(q0, g.step), rs[i]);
-      const float h1 = __fmul_rn(__fmul_rn(q1, g.step), rs[i + 1]);
+      const float h0 = unscale(__fmul_rn(q0, g.step), s[i], rs[i], a.exact != 0);
+      const float h1 = unscale(__fmul_rn(q1, g.step), s[i + 1], rs[i + 1], a.exact != 0);
       const __nv_bfloat162 pr = __floats2bfloat162_rn(__fsub_rn(w[i], h0), __fsub_rn(w[i + 1], h1));
       outw[i / 2] = *reinterpret_cast<const uint32_t*>(&pr);
     }
@@ -287,8 +293,8 @@ __device__ __forceinline__ void produce_row(const ProducerArgs& a, const uint4 (
 #pragma unroll
   for (int i = 0; i < kProdCols; i += 2) {
     const float q0 = code_of(wp[i], g, a.exact != 0), q1 = code_of(wp[i + 1], g, a.exact != 0);
-    const float h0 = __fmul_rn(dequant(q0, g), rs[i]);
-    const float h1 = __fmul_rn(dequant(q1, g), rs[i + 1]);
+    const float h0 = unscale(dequant(q0, g), s[i], rs[i], a.exact != 0);
+    const float h1 = unscale(dequant(q1, g), s[i + 1], rs[i + 1], a.exact != 0);
     const __nv_bfloat162 pr = __floats2bfloat162_rn(__fsub_rn(w[i], h0), __fsub_rn(w[i + 1], h1));
     outw[i / 2] = *reinterpret_cast<const uint32_t*>(&pr);
   }

@@ -1,6 +1,8 @@
-// ptx.cuh - thin inline-PTX wrappers for the sm_100a features the loss GEMM uses: mbarriers with
-// bounded waits, TMA tile loads (no multicast), tensor-memory allocation, tcgen05.mma (kind::f16,
-// one CTA) with its commit, and tcgen05.ld of the fp32 accumulator.
+// ptx.cuh - thin inline-PTX wrappers for the sm_100a features the tensor-core kernels use: mbarriers
+// with bounded waits (local and cluster-scope), TMA tile loads (no multicast) and stores,
+// tensor-memory allocation for one CTA or a CTA pair, tcgen05.mma kind::f16 issued for one CTA
+// (cta_group::1) or a CTA pair (cta_group::2) with its commits, and tcgen05.ld of the fp32
+// accumulator.
 #pragma once
 #include <cstdint>
 #include <cuda.h>

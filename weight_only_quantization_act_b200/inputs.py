@@ -21,8 +21,10 @@ Matrices are returned as ``numpy.uint16`` arrays holding bfloat16 bit patterns (
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import hashlib
+import os
 
 import numpy as np
 
@@ -67,16 +69,21 @@ WORKLOADS = {
 }
 
 
+_GEN_THREADS = max(1, min(8, os.cpu_count() or 1))
+
+
 def workload(number: int) -> Workload:
     return WORKLOADS[int(number)]
 
 
 def f32_to_bf16_bits(x) -> np.ndarray:
-    """Round float32 values to bfloat16 (nearest, ties to even); return the 16-bit patterns."""
+    """Round float32 values to bfloat16 (nearest, ties to even); return the 16-bit patterns.
+
+    In 32-bit integer arithmetic: for every finite or infinite value the bit pattern plus 0x7FFF plus the
+    kept lowest bit stays below 2^32 (the largest, -inf, is 0xFF800000); NaNs are replaced afterwards."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    u = x.view(np.uint32)
+    r = ((u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))) >> np.uint32(16)).astype(np.uint16)
     nan = np.isnan(x)
     if nan.any():
         r[nan] = 0x7FC0
@@ -107,15 +114,28 @@ def make_inputs(wl: Workload, rows: int | None = None, chunk_rows: int = 2048):
     mult[outliers] = wl.factor
     keep = N if rows is None else min(int(rows), N)
     X = np.empty((keep, K), np.uint16)
-    for r0 in range(0, keep, chunk_rows):
-        r1 = min(keep, r0 + chunk_rows)
-        if wl.gated:
+
+    def transform(r0, a, b):  # element-wise, so row pieces can run on worker threads
+        v = _silu_times(a, b) * mult if wl.gated else a.astype(np.float64) * mult
+        X[r0:r0 + a.shape[0]] = f32_to_bf16_bits(v.astype(np.float32))
+
+    # The draws stay in one sequential stream (chunk by chunk, a then b); their element-wise transforms
+    # run on a few threads (numpy releases the GIL), at most two chunks in flight.
+    pending = []
+    with concurrent.futures.ThreadPoolExecutor(max_workers=_GEN_THREADS) as pool:
+        for r0 in range(0, keep, chunk_rows):
+            r1 = min(keep, r0 + chunk_rows)
             a = rng.standard_normal((r1 - r0, K), dtype=np.float32)
-            b = rng.standard_normal((r1 - r0, K), dtype=np.float32)
-            v = _silu_times(a, b) * mult
-        else:
-            v = rng.standard_normal((r1 - r0, K), dtype=np.float32).astype(np.float64) * mult
-        X[r0:r1] = f32_to_bf16_bits(v.astype(np.float32))
+            b = rng.standard_normal((r1 - r0, K), dtype=np.float32) if wl.gated else None
+            if len(pending) >= 2:
+                for f in pending.pop(0):
+                    f.result()
+            step = max(1, -(-(r1 - r0) // _GEN_THREADS))
+            pending.append([pool.submit(transform, r0 + i, a[i:i + step], None if b is None else b[i:i + step])
+                            for i in range(0, r1 - r0, step)])
+        for fs in pending:
+            for f in fs:
+                f.result()
     Ws = []
     for o in wl.out_rows:
         Ws.append(f32_to_bf16_bits(
