@@ -262,12 +262,9 @@ __device__ __forceinline__ void produce_row(const ProducerArgs& a, const uint4 (
   for (int i = 0; i < 8; ++i) {
     w[2 * i] = bf16_lo(raw[i]);
     w[2 * i + 1] = bf16_hi(raw[i]);
-  }
-#pragma unroll
-  for (int i = 0; i < kProdCols; ++i) {
-    wp[i] = __fmul_rn(w[i], s[i]);
-    mx = fmaxf(mx, wp[i]);
-    mn = fminf(mn, wp[i]);
+    fx2_split(fx2_mul(fx2(w[2 * i], w[2 * i + 1]), fx2(s[2 * i], s[2 * i + 1])), wp[2 * i], wp[2 * i + 1]);
+    mx = max3f(mx, wp[2 * i], wp[2 * i + 1]);
+    mn = min3f(mn, wp[2 * i], wp[2 * i + 1]);
   }
   if (a.rowstep != nullptr) {  // INT8 per-channel: the row's step comes from the pre-pass
     GroupParams g;
@@ -290,6 +287,27 @@ __device__ __forceinline__ void produce_row(const ProducerArgs& a, const uint4 (
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
   }
   const GroupParams g = group_params(mx, mn);
+  float C = 0.0f;
+  if (a.exact == 0 && fast_group(g, mx, mn, C)) {
+    // Fast path (see fast_group): r = rint(w' / step) from t = RN(RN(w' * rstep) + C), deq = RN(r * step),
+    // w_hat = RN(deq * RN(1/s)), dW = bf16(RN(w - w_hat)), two elements per paired instruction.
+    const uint64_t rs2 = fx2(g.rstep, g.rstep), C2 = fx2(C, C), st2 = fx2(g.step, g.step);
+    float dmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kProdCols; i += 2) {
+      const uint64_t qa = fx2_mul(fx2(wp[i], wp[i + 1]), rs2);
+      const uint64_t r = fx2_sub(fx2_add(qa, C2), C2);
+      float d0, d1;
+      fx2_split(fx2_sub(qa, r), d0, d1);
+      dmax = max3f(dmax, fabsf(d0), fabsf(d1));
+      const uint64_t w_hat = fx2_mul(fx2_mul(r, st2), fx2(rs[i], rs[i + 1]));
+      float e0, e1;
+      fx2_split(fx2_sub(fx2(w[i], w[i + 1]), w_hat), e0, e1);
+      const __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
+      outw[i / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+    }
+    if (dmax < kTieMargin) return;  // else: a quotient near a half-integer, redo the lane exactly
+  }
 #pragma unroll
   for (int i = 0; i < kProdCols; i += 2) {
     const float q0 = code_of(wp[i], g, a.exact != 0), q1 = code_of(wp[i + 1], g, a.exact != 0);
@@ -426,7 +444,7 @@ constexpr int kPackWarpCols = 32 * kPackCols;    // 1024 in-features (one segmen
 // Warp v owns segment v % segs and rows v / segs, v / segs + wps, ... (wps = warps per segment): the
 // segment's scales stay in registers and the next row's weights are loaded while the current row is
 // quantized. With fewer warps than segments a warp walks several whole segments.
-__global__ void __launch_bounds__(kPackThreads) quantize_pack_kernel(
+__global__ void __launch_bounds__(kPackThreads, 2) quantize_pack_kernel(
     const uint16_t* __restrict__ W, int64_t O, int64_t K, int64_t ldw, const float* __restrict__ scales,
     int exact, uint32_t* __restrict__ codes, float* __restrict__ steps, float* __restrict__ zeros) {
   const int64_t segs = (K + kPackWarpCols - 1) / kPackWarpCols;
@@ -476,21 +494,21 @@ __global__ void __launch_bounds__(kPackThreads) quantize_pack_kernel(
 #pragma unroll
         for (int i = 0; i < 4; ++i) nxt[i] = __ldcs(src + i);
       }
-      float wp[kPackCols];
+      // w' = RN(w * s) in pairs (elements 2i, 2i+1 of the lane's 32 in-features)
+      uint64_t wp2[kPackCols / 2];
       float mx = -__int_as_float(0x7f800000), mn = __int_as_float(0x7f800000);
 #pragma unroll
       for (int v4 = 0; v4 < 4; ++v4) {
         const uint32_t uu[4] = {cur[v4].x, cur[v4].y, cur[v4].z, cur[v4].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          wp[8 * v4 + 2 * i] = __fmul_rn(bf16_lo(uu[i]), s[8 * v4 + 2 * i]);
-          wp[8 * v4 + 2 * i + 1] = __fmul_rn(bf16_hi(uu[i]), s[8 * v4 + 2 * i + 1]);
+          const int e = 8 * v4 + 2 * i;
+          wp2[e / 2] = fx2_mul(fx2(bf16_lo(uu[i]), bf16_hi(uu[i])), fx2(s[e], s[e + 1]));
+          float a, b;
+          fx2_split(wp2[e / 2], a, b);
+          mx = max3f(mx, a, b);
+          mn = min3f(mn, a, b);
         }
-      }
-#pragma unroll
-      for (int i = 0; i < kPackCols; ++i) {
-        mx = fmaxf(mx, wp[i]);
-        mn = fminf(mn, wp[i]);
       }
 #pragma unroll
       for (int off = 1; off < 4; off <<= 1) {
@@ -500,12 +518,44 @@ __global__ void __launch_bounds__(kPackThreads) quantize_pack_kernel(
       if (!active) continue;
       const GroupParams g = group_params(mx, mn);
       uint32_t word[4];
+      float C = 0.0f;
+      bool fast = exact == 0 && fast_group(g, mx, mn, C);
+      if (fast) {
+        // t = RN(RN(w' * rstep) + C); its low byte is the code; pairs of codes are joined by one
+        // integer multiply-add (t1 * 16 + t0: the low byte is c0 + 16 c1, no carry out of it), two
+        // pairs by another (p23 * 256 + p01), and the two halves of a word by a byte permute.
+        const uint64_t rs2 = fx2(g.rstep, g.rstep), C2 = fx2(C, C);
+        float dmax = 0.0f;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        word[w] = 0u;
+        for (int w = 0; w < 4; ++w) {
+          uint32_t p[4];  // p[i]: low byte = codes of elements 8w + 2i and 8w + 2i + 1
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          word[w] |= static_cast<uint32_t>(code_of(wp[8 * w + i], g, exact != 0)) << (4 * i);
+          for (int i = 0; i < 4; ++i) {
+            const uint64_t qa = fx2_mul(wp2[4 * w + i], rs2);
+            const uint64_t t = fx2_add(qa, C2);
+            const uint64_t d = fx2_sub(qa, fx2_sub(t, C2));
+            float d0, d1, t0, t1;
+            fx2_split(d, d0, d1);
+            fx2_split(t, t0, t1);
+            dmax = max3f(dmax, fabsf(d0), fabsf(d1));
+            p[i] = __float_as_uint(t1) * 16u + __float_as_uint(t0);
+          }
+          word[w] = __byte_perm(p[1] * 256u + p[0], p[3] * 256u + p[2], 0x5410);
+        }
+        fast = dmax < kTieMargin;
+      }
+      if (!fast) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          word[w] = 0u;
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            float a, b;
+            fx2_split(wp2[(8 * w + i) / 2], a, b);
+            word[w] |= static_cast<uint32_t>(code_of(a, g, exact != 0)) << (4 * i);
+            word[w] |= static_cast<uint32_t>(code_of(b, g, exact != 0)) << (4 * i + 4);
+          }
+        }
       }
       __stcs(reinterpret_cast<uint4*>(codes + o * (K / 8) + k0 / 8), make_uint4(word[0], word[1], word[2], word[3]));
       if ((lane & 3) == 0) {

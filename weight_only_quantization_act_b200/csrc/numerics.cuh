@@ -231,6 +231,74 @@ __device__ __forceinline__ float dequant(float q, const GroupParams& g) {
   return __fmul_rn(__fsub_rn(q, g.zero), g.step);
 }
 
+// ===================================================================================================
+// Paired fp32 arithmetic of sm_100 (add/sub/mul .rn.f32x2): two fp32 values in one 64-bit register,
+// each lane an ordinary IEEE operation rounded to nearest (the same bits as two scalar __f*_rn
+// operations, never contracted), issued as one instruction. Three-input min/max of sm_100.
+// ===================================================================================================
+__device__ __forceinline__ uint64_t fx2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void fx2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fx2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fx2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fx2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// ===================================================================================================
+// Fast path of the group quantizer, bit-identical to code_of / dequant where it applies.
+//
+// With C = M + z, M = 1.5 * 2^23, every float in [2^23, 2^24) is an integer, so
+//   t = RN(qa + C), qa = RN(w' * RN(1/step)),
+// is C + rint(qa) whenever qa is not a tie (z is an integer, |z| < 2^21), r = t - C = rint(qa) exactly,
+// and d = qa - r is exact (r is 0 or within a factor 2 of qa). By the argument of rint_quotient,
+// |d| < 0.5 - 2^-14 and |qa| < 128 make r = rint(RN(w' / step)); then the unclamped code is r + z and
+// t = M + code. The group-level conditions (fast_group):
+//   |z| < 2^21;  RN(max(|max|, |min|) * rstep) < 128 (bounds every |qa| by monotonicity of rounding);
+//   the t of the group's min and max elements lie in [M, M + 15] (t is monotone in w', so every code
+//   of the group lies in [0, 15] and the clamp is the identity).
+// The element-level condition |d| < 0.5 - 2^-14 is checked as the max over a lane's elements; a lane
+// that fails it (a quotient within 2^-14 of a half-integer, about one element in 10^4) redoes its
+// elements with code_of. In the fast path the low byte of t's bit pattern is the code (M = 0x4B400000),
+// and RN32(q - z) = r, so the dequantized value is RN(r * step).
+// ===================================================================================================
+constexpr float kQuantMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr float kTieMargin = 0.5f - 0x1p-14f;
+
+__device__ __forceinline__ bool fast_group(const GroupParams& g, float mx, float mn, float& C) {
+  if (!(fabsf(g.zero) < 2097152.0f)) return false;
+  if (!(__fmul_rn(fmaxf(fabsf(mx), fabsf(mn)), g.rstep) < 128.0f)) return false;
+  C = __fadd_rn(kQuantMagic, g.zero);
+  const float t_mx = __fadd_rn(__fmul_rn(mx, g.rstep), C);
+  const float t_mn = __fadd_rn(__fmul_rn(mn, g.rstep), C);
+  return t_mn >= kQuantMagic && t_mx <= kQuantMagic + 15.0f;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
