@@ -116,6 +116,8 @@ awq_status device_info(DeviceInfo** out) {
                                   awq::lg::SMEM_BYTES));
     AWQ_CUDA(cudaFuncSetAttribute(awq::act_chunk_sums_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   awq::kActSmemBytes));
+    AWQ_CUDA(cudaFuncSetAttribute(awq::quantize_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::kPackSmemBytes));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(d.sms & ~1));
     cfg.blockDim = dim3(awq::lg::THREADS);
@@ -322,6 +324,17 @@ awq_status launch_scale_table(const float* act, const float* wmean, int64_t K, i
   return check_launch("scale_normalize_kernel");
 }
 
+// Tile raster of the loss GEMM: a group of dW bands advances together over the token blocks, so each
+// X tile is read from DRAM once per group while the group's bands (256 rows x K each) are re-read by
+// every token block. In flight, the pairs sit at spread-out points of their K loops, so the bands stay
+// in L2 only if the whole group (bands x 512 K bytes) fits in about half of it; beyond that they are
+// fetched again and again (measured on B200 at K = 28672: 4 bands 1.08 GHz under the power cap, 8
+// bands 1.02 GHz, 16 bands 0.88 GHz). Fewer bands mean more X reads, so take as many as fit, at most 8.
+int loss_bands_per_group(int64_t K) {
+  const int64_t band_bytes = static_cast<int64_t>(awq::lg::BN) * K * 2;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(8, (60ll << 20) / band_bytes)));
+}
+
 int scale_mode_of(unsigned flags) {
   if (flags & AWQ_FLAG_SCALES_WEIGHT_AWARE) return awq::kScalesWeightAware;
   if (flags & AWQ_FLAG_SCALES_RMS) return awq::kScalesRms;
@@ -502,6 +515,7 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   p.n_bands = static_cast<int>(static_cast<int64_t>(n_grid) * l.tiles_o);
   p.num_kb = static_cast<int>(K / awq::lg::BK);
   p.num_tiles = p.n_tiles_n * p.n_bands;
+  p.bands_per_group = loss_bands_per_group(K);
   p.partials = partials;
   p.status = status;
   p.limit_ns = g_wait_limit_ns.load();
@@ -590,7 +604,7 @@ awq_status awq_quantize_pack_ex(const void* W, int64_t O, int64_t K, int64_t ldw
   const int64_t items = O * segs;
   const int64_t max_blocks = static_cast<int64_t>(d->sms) * 2;  // 2 blocks of 256 threads fit per SM
   const int64_t blocks = std::min<int64_t>(max_blocks, (items * 32 + awq::kPackThreads - 1) / awq::kPackThreads);
-  awq::quantize_pack_kernel<<<static_cast<unsigned>(blocks), awq::kPackThreads, 0,
+  awq::quantize_pack_kernel<<<static_cast<unsigned>(blocks), awq::kPackThreads, awq::kPackSmemBytes,
                               reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint16_t*>(W), O, K, ldw, scales, (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0, codes, steps,
       zeros);

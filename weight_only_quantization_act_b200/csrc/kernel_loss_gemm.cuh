@@ -44,7 +44,6 @@ constexpr int NUM_ACC = 2;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int PROD_WARPS = 8;
 constexpr int THREADS = 192 + 32 * PROD_WARPS;
-constexpr int BANDS_PER_GROUP = 8;               // tile raster: 8 dW bands advance together over X
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
 constexpr int PARTIALS_PER_TILE = 8;             // 2 CTAs x 4 lane quarters, 32 token rows each
 constexpr int RING = 8;                          // tile-index slots; producers run <= 4 tiles ahead
@@ -56,6 +55,7 @@ struct Params {
   int n_bands;        // bands this launch covers
   int num_kb;         // K / BK
   int num_tiles;      // n_tiles_n * n_bands
+  int bands_per_group;  // tile raster: this many dW bands advance together over the token blocks
   double* partials;   // [all bands][n_tiles_n][PARTIALS_PER_TILE]
   DeviceStatus* status;
   uint64_t limit_ns;
@@ -70,11 +70,11 @@ struct Params {
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& band, int& nt) {
-  const int per_group = BANDS_PER_GROUP * p.n_tiles_n;
+  const int per_group = p.bands_per_group * p.n_tiles_n;
   const int g = t / per_group;
   const int local = t - g * per_group;
-  const int bands_in_g = min(BANDS_PER_GROUP, p.n_bands - g * BANDS_PER_GROUP);
-  band = p.band_begin + g * BANDS_PER_GROUP + local % bands_in_g;
+  const int bands_in_g = min(p.bands_per_group, p.n_bands - g * p.bands_per_group);
+  band = p.band_begin + g * p.bands_per_group + local % bands_in_g;
   nt = local / bands_in_g;
 }
 

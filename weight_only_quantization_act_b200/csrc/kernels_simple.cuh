@@ -434,23 +434,33 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(const double* __r
 }
 
 // ===================================================================================================
-// (5) pack: codes, steps and zeros of W at scales s. One thread owns 8 in-features (one code word);
-// 16 lanes per group; one warp covers 256 in-features of one row.
+// (5) pack: codes, steps and zeros of W at scales s. One warp covers 1024 in-features (a segment) of one
+// row; each lane owns 32 consecutive in-features (4 lanes per group of 128, four code words).
 // ===================================================================================================
 constexpr int kPackThreads = 256;
 constexpr int kPackCols = 32;                    // in-features per lane (4 lanes per group of 128)
 constexpr int kPackWarpCols = 32 * kPackCols;    // 1024 in-features (one segment) per warp
+constexpr int kPackStages = 6;                   // rows in flight per warp (cp.async ring)
+constexpr int kPackStageBytes = kPackWarpCols * 2;                                   // 2 KB
+constexpr int kPackSmemBytes = kPackStages * (kPackThreads / 32) * kPackStageBytes;  // 96 KB
 
 // Warp v owns segment v % segs and rows v / segs, v / segs + wps, ... (wps = warps per segment): the
-// segment's scales stay in registers and the next row's weights are loaded while the current row is
-// quantized. With fewer warps than segments a warp walks several whole segments.
+// segment's scales stay in registers. Each lane streams its own 64 bytes of the next rows through a
+// ring in shared memory with cp.async (up to kPackStages - 1 rows in flight per warp, no registers
+// held); a lane only reads back what it copied itself, so the ring is laid out for conflict-free
+// access (16-byte piece j of lane l at slot offset 16 (32 j + l)) and needs no warp synchronisation.
+// With fewer warps than segments a warp walks several whole segments.
 __global__ void __launch_bounds__(kPackThreads, 2) quantize_pack_kernel(
     const uint16_t* __restrict__ W, int64_t O, int64_t K, int64_t ldw, const float* __restrict__ scales,
     int exact, uint32_t* __restrict__ codes, float* __restrict__ steps, float* __restrict__ zeros) {
+  extern __shared__ __align__(16) uint8_t pack_ring[];
   const int64_t segs = (K + kPackWarpCols - 1) / kPackWarpCols;
   const int64_t v = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
   const int64_t total = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(pack_ring)) +
+                        static_cast<uint32_t>((threadIdx.x >> 5) * kPackStages * kPackStageBytes) +
+                        static_cast<uint32_t>(lane) * 16u;
   int64_t seg_first, seg_step, row_first, row_step;
   if (total >= segs) {
     const int64_t wps = total / segs;
@@ -480,20 +490,32 @@ __global__ void __launch_bounds__(kPackThreads, 2) quantize_pack_kernel(
 #pragma unroll
       for (int i = 0; i < kPackCols; ++i) s[i] = 1.0f;
     }
-    uint4 nxt[4] = {};
-    if (row_first < O && active) {
-      const uint4* src = reinterpret_cast<const uint4*>(W + row_first * ldw + k0);
+    // row i of this warp is o = row_first + i * row_step, staged in slot i % kPackStages
+    auto issue = [&](int64_t i) {
+      const int64_t o = row_first + i * row_step;
+      if (o < O && active) {
+        const uint16_t* src = W + o * ldw + k0;
+        const uint32_t dst = ring + static_cast<uint32_t>((i % kPackStages) * kPackStageBytes);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) nxt[i] = __ldcs(src + i);
-    }
-    for (int64_t o = row_first; o < O; o += row_step) {
-      const uint4 cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
-      const int64_t on = o + row_step;
-      if (on < O && active) {
-        const uint4* src = reinterpret_cast<const uint4*>(W + on * ldw + k0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) nxt[i] = __ldcs(src + i);
+        for (int j = 0; j < 4; ++j) cp_async_16(dst + static_cast<uint32_t>(j * 512), src + 8 * j, 16u);
       }
+      cp_async_commit();  // an empty group keeps the wait arithmetic uniform
+    };
+#pragma unroll 1
+    for (int64_t i = 0; i < kPackStages - 1; ++i) issue(i);
+#pragma unroll 1
+    for (int64_t i = 0; row_first + i * row_step < O; ++i) {
+      const int64_t o = row_first + i * row_step;
+      issue(i + kPackStages - 1);  // into the slot read in the previous iteration
+      cp_async_wait<kPackStages - 1>();
+      uint4 cur[4];
+      const uint32_t src = ring + static_cast<uint32_t>((i % kPackStages) * kPackStageBytes);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(cur[j].x), "=r"(cur[j].y), "=r"(cur[j].z), "=r"(cur[j].w)
+                     : "r"(src + static_cast<uint32_t>(j * 512))
+                     : "memory");
       // w' = RN(w * s) in pairs (elements 2i, 2i+1 of the lane's 32 in-features)
       uint64_t wp2[kPackCols / 2];
       float mx = -__int_as_float(0x7f800000), mn = __int_as_float(0x7f800000);
@@ -501,9 +523,9 @@ __global__ void __launch_bounds__(kPackThreads, 2) quantize_pack_kernel(
       for (int v4 = 0; v4 < 4; ++v4) {
         const uint32_t uu[4] = {cur[v4].x, cur[v4].y, cur[v4].z, cur[v4].w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int e = 8 * v4 + 2 * i;
-          wp2[e / 2] = fx2_mul(fx2(bf16_lo(uu[i]), bf16_hi(uu[i])), fx2(s[e], s[e + 1]));
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const int e = 8 * v4 + 2 * e2;
+          wp2[e / 2] = fx2_mul(fx2(bf16_lo(uu[e2]), bf16_hi(uu[e2])), fx2(s[e], s[e + 1]));
           float a, b;
           fx2_split(wp2[e / 2], a, b);
           mx = max3f(mx, a, b);
@@ -528,17 +550,17 @@ __global__ void __launch_bounds__(kPackThreads, 2) quantize_pack_kernel(
         float dmax = 0.0f;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          uint32_t p[4];  // p[i]: low byte = codes of elements 8w + 2i and 8w + 2i + 1
+          uint32_t p[4];  // p[e2]: low byte = codes of elements 8w + 2e2 and 8w + 2e2 + 1
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint64_t qa = fx2_mul(wp2[4 * w + i], rs2);
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const uint64_t qa = fx2_mul(wp2[4 * w + e2], rs2);
             const uint64_t t = fx2_add(qa, C2);
             const uint64_t d = fx2_sub(qa, fx2_sub(t, C2));
             float d0, d1, t0, t1;
             fx2_split(d, d0, d1);
             fx2_split(t, t0, t1);
             dmax = max3f(dmax, fabsf(d0), fabsf(d1));
-            p[i] = __float_as_uint(t1) * 16u + __float_as_uint(t0);
+            p[e2] = __float_as_uint(t1) * 16u + __float_as_uint(t0);
           }
           word[w] = __byte_perm(p[1] * 256u + p[0], p[3] * 256u + p[2], 0x5410);
         }
@@ -549,11 +571,11 @@ __global__ void __launch_bounds__(kPackThreads, 2) quantize_pack_kernel(
         for (int w = 0; w < 4; ++w) {
           word[w] = 0u;
 #pragma unroll
-          for (int i = 0; i < 8; i += 2) {
+          for (int e = 0; e < 8; e += 2) {
             float a, b;
-            fx2_split(wp2[(8 * w + i) / 2], a, b);
-            word[w] |= static_cast<uint32_t>(code_of(a, g, exact != 0)) << (4 * i);
-            word[w] |= static_cast<uint32_t>(code_of(b, g, exact != 0)) << (4 * i + 4);
+            fx2_split(wp2[(8 * w + e) / 2], a, b);
+            word[w] |= static_cast<uint32_t>(code_of(a, g, exact != 0)) << (4 * e);
+            word[w] |= static_cast<uint32_t>(code_of(b, g, exact != 0)) << (4 * e + 4);
           }
         }
       }
@@ -564,6 +586,7 @@ __global__ void __launch_bounds__(kPackThreads, 2) quantize_pack_kernel(
         zeros[gi] = g.zero;
       }
     }
+    cp_async_wait<0>();  // nothing of this segment's ring is still being written
   }
 }
 
