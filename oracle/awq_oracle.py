@@ -336,11 +336,18 @@ def dequant_w4(words, steps, zeros, group: int = GROUP) -> np.ndarray:
     return ((q - z) * st).astype(F32)
 
 
-def w4a16_matmul(x_bits, words, steps, zeros, group: int = GROUP) -> np.ndarray:
-    """fp64 [M, O] = X' @ bf16(deq(W))^T, with the bf16 weight operand the GPU feeds its tensor cores."""
-    deq16 = widen_bf16(round_f32_to_bf16(dequant_w4(words, steps, zeros, group))).astype(F64)
+def w4a16_matmul(x_bits, words, steps, zeros, group: int = GROUP, weights: str = "bf16") -> np.ndarray:
+    """fp64 [M, O] = X' @ deq(W)^T with the weights restored to bfloat16 (weights="bf16": the 16-bit
+    operand of a kernel that dequantizes into its tensor-core tiles) or kept at their fp32 dequantized
+    value RN32((q - z) * step) (weights="fp32": a kernel that applies the step and zero point after the
+    products of each group)."""
+    deq = dequant_w4(words, steps, zeros, group)
+    if weights == "bf16":
+        deq = widen_bf16(round_f32_to_bf16(deq))
+    elif weights != "fp32":
+        raise ValueError("weights must be 'bf16' or 'fp32'")
     x = widen_bf16(x_bits).astype(F64)
-    return x @ deq16.T
+    return x @ deq.astype(F64).T
 
 
 # ---------------------------------------------------------------------------------------------------

@@ -18,14 +18,34 @@ def _lib():
     awq.load_library()
 
 
+DECODE_MAX_TOKENS = 64   # up to this many tokens the library runs the few-token kernel
+
+
 def check_against_oracle(Xp, words, steps, zeros, Y):
-    """|Y - ref| <= 2^-8 |ref| + (K/16 + 16) 2^-23 sum_k |x w|: bf16 output rounding plus fp32 accumulation."""
-    K = Xp.shape[1]
-    ref = orc.w4a16_matmul(Xp, words, steps, zeros)
-    deq16 = inputs.bf16_bits_to_f32(orc.round_f32_to_bf16(orc.dequant_w4(words, steps, zeros))).astype(np.float64)
-    mag = np.abs(inputs.bf16_bits_to_f32(Xp).astype(np.float64)) @ np.abs(deq16).T
+    """Many tokens (bf16 weight operand): |Y - ref| <= 2^-8 |ref| + (K/16 + 16) 2^-23 sum_k |x w|, the bf16
+    output rounding plus fp32 accumulation.
+
+    Few tokens (the weights enter at their fp32 dequantized value; per group g the tensor cores sum
+    x (128 + q) exactly-rounded in fp32, and y += step (S_g - (128 + z) Sx_g) in fp32): |Y - ref| <= 2^-8 |ref|
+    + 2^-24 sum_g step_g A_g (128 * 143 + 130 (128 + |z_g|) + (G + 18) (15 + |z_g|)) + 2^-23 sum_k |x w|, where
+    A_g = sum over the group of |x|: the first term of the bracket bounds the accumulation of S_g (128
+    additions of terms up to 143 |x|), the second that of Sx_g and the zero-point product, the third the
+    running sums over groups and slices (at most 16); the last term covers the weight's own fp32 rounding."""
+    M, K = Xp.shape
+    x64 = inputs.bf16_bits_to_f32(Xp).astype(np.float64)
     got = Y.float().cpu().numpy().astype(np.float64)
-    tol = 2.0 ** -8 * np.abs(ref) + (K / 16 + 16) * 2.0 ** -23 * mag
+    if M > DECODE_MAX_TOKENS:
+        ref = orc.w4a16_matmul(Xp, words, steps, zeros)
+        deq16 = inputs.bf16_bits_to_f32(orc.round_f32_to_bf16(orc.dequant_w4(words, steps, zeros))).astype(np.float64)
+        tol = 2.0 ** -8 * np.abs(ref) + (K / 16 + 16) * 2.0 ** -23 * (np.abs(x64) @ np.abs(deq16).T)
+    else:
+        ref = orc.w4a16_matmul(Xp, words, steps, zeros, weights="fp32")
+        deq = orc.dequant_w4(words, steps, zeros).astype(np.float64)
+        G = K // 128
+        A = np.abs(x64).reshape(M, G, 128).sum(axis=2)                     # [M, G]
+        z = np.abs(np.asarray(zeros, np.float64))
+        coef = np.asarray(steps, np.float64) * (128 * 143 + 130 * (128 + z) + (G + 18) * (15 + z))  # [O, G]
+        tol = 2.0 ** -8 * np.abs(ref) + 2.0 ** -24 * (A @ coef.T) + 2.0 ** -23 * (np.abs(x64) @ np.abs(deq).T)
     bad = np.abs(got - ref) > tol
     assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], ref[bad][:5])
 
@@ -91,6 +111,28 @@ def test_w4a16_few_tokens_match_oracle(M, K, O):
                        torch.from_numpy(steps).cuda(), torch.from_numpy(zeros).cuda())
     torch.cuda.synchronize()
     check_against_oracle(Xp, words, steps, zeros, Y)
+
+
+@pytest.mark.parametrize("M,K,O", [(64, 256, 136), (16, 384, 256), (48, 1024, 520), (33, 4096, 128)])
+def test_w4a16_few_tokens_one_hot_columns_exact(M, K, O):
+    """Token m of X' is one-hot at in-feature k_m with a power-of-two value: its row of Y is then exactly
+    bf16(x * RN32((q - z) * step)) of column k_m (the group sums reduce to one exact product, the zero-point
+    term cancels exactly, and the other groups add zeros), so every nibble, the operand permutation, the
+    swizzles, the group's step and zero and the split-K reduction are checked bit for bit."""
+    rng = np.random.default_rng(M + K + O)
+    _, _, (words, steps, zeros) = quantized(O, K, 7 * M + K + O)
+    ks = rng.choice(K, size=M, replace=M > K)
+    ks[:min(M, 8)] = np.arange(min(M, 8))  # the eight nibbles of the first word
+    vals = np.array([0x3F80, 0x4000, 0x3E80, 0xBF00, 0x4100], np.uint16)  # 1, 2, 0.25, -0.5, 8
+    Xp = np.zeros((M, K), np.uint16)
+    Xp[np.arange(M), ks] = vals[np.arange(M) % vals.size]
+    Y = awq.w4a16_gemm(bf16_to_device(Xp), torch.from_numpy(words.view(np.int32)).cuda(),
+                       torch.from_numpy(steps).cuda(), torch.from_numpy(zeros).cuda())
+    torch.cuda.synchronize()
+    want = orc.round_f32_to_bf16(orc.w4a16_matmul(Xp, words, steps, zeros, weights="fp32").astype(np.float32))
+    got = Y.cpu().view(torch.int16).numpy().view(np.uint16)
+    bad = np.argwhere(got != want)
+    assert bad.size == 0, (bad[:5], got[tuple(bad[0])], want[tuple(bad[0])])
 
 
 def test_w4a16_few_tokens_deterministic_and_strided():

@@ -491,6 +491,30 @@ def test_w4a16_hand_examples():
     q = rng.integers(0, 16, (O, K)).astype(np.uint8)
     y = orc.w4a16_matmul(x, orc.pack_codes(q), np.ones((O, 1), F32), np.zeros((O, 1), F32))
     assert np.array_equal(y, inputs.bf16_bits_to_f32(x).astype(np.float64) @ q.T.astype(np.float64))
+    for weights in ("bf16", "fp32"):
+        y = orc.w4a16_matmul(x, orc.pack_codes(q), np.ones((O, 1), F32), np.zeros((O, 1), F32), weights=weights)
+        assert np.array_equal(y, inputs.bf16_bits_to_f32(x).astype(np.float64) @ q.T.astype(np.float64))
+
+
+def test_w4a16_fp32_weights_one_hot_columns():
+    """With X' one-hot at in-feature k (value 1), row m of the fp32-weight product is column k of the
+    dequantized weight exactly, q - z times step rounded once; the bf16-weight product is its bf16 rounding."""
+    O, K = 16, 256
+    rng = np.random.default_rng(115)
+    q = rng.integers(0, 16, (O, K)).astype(np.uint8)
+    steps = (rng.random((O, K // 128)) * 0.01 + 1e-3).astype(F32)
+    zeros = rng.integers(-3, 19, (O, K // 128)).astype(F32)
+    ks = np.array([0, 1, 4, 7, 8, 127, 128, 200, 255])
+    x = np.zeros((ks.size, K), np.uint16)
+    x[np.arange(ks.size), ks] = 0x3F80  # bf16 1.0
+    words = orc.pack_codes(q)
+    y32 = orc.w4a16_matmul(x, words, steps, zeros, weights="fp32")
+    y16 = orc.w4a16_matmul(x, words, steps, zeros, weights="bf16")
+    for i, k in enumerate(ks):
+        g = k // 128
+        want = np.array([np.float32(np.float32(float(q[o, k]) - zeros[o, g]) * steps[o, g]) for o in range(O)])
+        assert np.array_equal(y32[i], want.astype(np.float64))
+        assert np.array_equal(y16[i], inputs.bf16_bits_to_f32(orc.round_f32_to_bf16(want)).astype(np.float64))
 
 
 # ------------------------------------------------------------------------------------------ scale rules

@@ -137,8 +137,14 @@ awq_status device_info(DeviceInfo** out) {
     cfg.dynamicSmemBytes = awq::dq::SMEM_BYTES;
     AWQ_CUDA(cudaOccupancyMaxActiveClusters(&d.w4_clusters, awq::dq::w4a16_gemm_kernel, &cfg));
     if (d.w4_clusters < 1) return fail(AWQ_ERR_UNSUPPORTED, "the W4A16 GEMM does not fit on this device");
-    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  awq::dec::smem_bytes(awq::dec::MAX_NT)));
+    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::dec::Shape<16>::SMEM));
+    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::dec::Shape<32>::SMEM));
+    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<48>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::dec::Shape<48>::SMEM));
+    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::dec::Shape<64>::SMEM));
     d.gemm_attr_set = true;
   }
   *out = &d;
@@ -792,7 +798,7 @@ W4Layout w4_layout(int64_t K, int64_t O) {
   return l;
 }
 
-// Few tokens: weight rows on the MMA's M side, k-blocks split into slices until every SM has a share,
+// Few tokens: weight rows on the MMA's M side, groups split into slices until every SM has a share,
 // slices added by the last CTA of each row block. One launch; the per-block counters are zero from the
 // caller's initial zero fill and every call leaves them zero.
 awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const uint32_t* codes, const float* steps,
@@ -801,14 +807,12 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   DeviceInfo* d = nullptr;
   AWQ_TRY(device_info(&d));
   const int nt = static_cast<int>((M + 15) / 16 * 16);
-  const int num_kb = static_cast<int>(K / awq::dec::BK);
-  // one wave: two CTAs per SM when their shared memory allows it (up to 32 tokens), else one
-  const int64_t per_sm = awq::dec::smem_bytes(nt) <= 112 * 1024 ? 2 : 1;
-  int64_t slices = per_sm * static_cast<int64_t>(d->sms) / l.n_rb;
-  slices = std::max<int64_t>(1, std::min<int64_t>({slices, awq::dec::max_slices(l.n_rb), num_kb}));
-  const int kb_box = awq::dec::KB_PER_BOX;
-  const int kb_per = static_cast<int>(((num_kb + slices - 1) / slices + kb_box - 1) / kb_box * kb_box);
-  slices = (num_kb + kb_per - 1) / kb_per;
+  const int num_groups = static_cast<int>(K / 128);
+  // one wave of CTAs; a slice holds an even number of groups (one code box covers two)
+  int64_t slices = awq::dec::ctas_per_sm(nt) * static_cast<int64_t>(d->sms) / l.n_rb;
+  slices = std::max<int64_t>(1, std::min<int64_t>({slices, awq::dec::max_slices(l.n_rb), (num_groups + 1) / 2}));
+  const int g_per = static_cast<int>(((num_groups + slices - 1) / slices + 1) / 2 * 2);
+  slices = (num_groups + g_per - 1) / g_per;
   if (l.n_rb * slices >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "O is too large");
   CUtensorMap tmX, tmC;
   AWQ_TRY(make_tmap(&tmX, X, M, K, ldx, nt));
@@ -825,19 +829,21 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   p.O = O;
   p.G = l.G;
   p.ldy = ldy;
-  p.nt = nt;
-  p.num_kb = num_kb;
-  p.kb_per = kb_per;
+  p.num_groups = num_groups;
+  p.g_per = g_per;
   p.slices = static_cast<int>(slices);
-  p.sz_pairs = (l.G % 2 == 0 && (reinterpret_cast<uintptr_t>(steps) & 7u) == 0 &&
-                (reinterpret_cast<uintptr_t>(zeros) & 7u) == 0)
-                   ? 1
-                   : 0;
   p.idesc = awq::idesc_bf16_f32(awq::dec::ROWS, static_cast<uint32_t>(nt));
   p.status = reinterpret_cast<awq::DeviceStatus*>(ws);
   p.limit_ns = g_wait_limit_ns.load();
-  awq::dec::w4a16_decode_kernel<<<static_cast<unsigned>(l.n_rb * slices), awq::dec::THREADS,
-                                  awq::dec::smem_bytes(nt), st>>>(tmX, tmC, p);
+  const dim3 grid(static_cast<unsigned>(l.n_rb * slices));
+  if (nt == 16)
+    awq::dec::w4a16_decode_kernel<16><<<grid, awq::dec::THREADS, awq::dec::Shape<16>::SMEM, st>>>(tmX, tmC, p);
+  else if (nt == 32)
+    awq::dec::w4a16_decode_kernel<32><<<grid, awq::dec::THREADS, awq::dec::Shape<32>::SMEM, st>>>(tmX, tmC, p);
+  else if (nt == 48)
+    awq::dec::w4a16_decode_kernel<48><<<grid, awq::dec::THREADS, awq::dec::Shape<48>::SMEM, st>>>(tmX, tmC, p);
+  else
+    awq::dec::w4a16_decode_kernel<64><<<grid, awq::dec::THREADS, awq::dec::Shape<64>::SMEM, st>>>(tmX, tmC, p);
   AWQ_TRY(check_launch("w4a16_decode_kernel"));
   return ok();
 }
