@@ -1,35 +1,32 @@
 // kernel_w4a16_decode.cuh - the deployment GEMM of an AWQ-quantized linear for few tokens (decode, small
 // batches): Y = X' deq(W)^T with M <= 64 tokens. At this size the work is reading and unpacking the packed
-// weights, so the weight rows take the MMA's M side, the k-blocks are split until every SM has a share,
-// and the per-weight arithmetic is moved off the CUDA cores:
+// weights, so the weight rows take the MMA's M side, the groups are split into slices until every SM has
+// a share, and the per-weight arithmetic is moved off the CUDA cores:
 //
 //   deq(W)[o, k] = (q - z_g) * step_g for the group g of 128 in-features holding k, so
 //   Y[m, o] = sum_g step_g * ( S_g[o, m] - (128 + z_g) * Sx_g[m] ),
 //   S_g[o, m] = sum_{k in g} (128 + q[o, k]) * x'[m, k],   Sx_g[m] = sum_{k in g} x'[m, k].
 //
-// The tensor cores compute S_g exactly from bf16 operands (128 + q is the bf16 pattern 0x4300 | q, an
-// OR with the code nibble, and every product of two bf16 values is exact in the fp32 accumulator), one
-// group per accumulator; the CUDA cores then apply the group's step and zero point once per output
-// element and group instead of once per weight. The weights thus enter with their exact dequantized
-// value (q - z) * step ("GPU 硬件级反量化算子内联融合" on the bjdmk.com.cn AWQ article: unpack with shifts and
+// The tensor cores compute S_g from bf16 operands (128 + q is the bf16 pattern 0x4300 | q, an OR with the
+// code nibble, and every product of two bf16 values is exact in the fp32 accumulator), one group per
+// accumulator; the CUDA cores then apply the group's step and zero point once per output element and
+// group instead of once per weight. The weights thus enter with their exact dequantized value
+// (q - z) * step ("GPU 硬件级反量化算子内联融合" on the bjdmk.com.cn AWQ article: unpack with shifts and
 // masks, convert, apply the group scale and offset; here the scale and offset are applied after the
 // products of each group).
 //
-// Nibble order. A code word holds in-features 8c .. 8c+7 in nibbles 0..7. One OR-and-mask per register
-// turns the word shifted right by 4j into the bf16 pair (128 + q_j, 128 + q_{j+4}), so the operand row
-// holds each word's in-features in the order 0 4 1 5 2 6 3 7. X' is permuted the same way inside every
-// 16-byte chunk (8 in-features) after it lands, which leaves the products and their sum unchanged.
-//
-// CTA (b, c) covers weight rows [128 b, 128 b + 128) and groups [c * gp, (c + 1) * gp) (gp even). Warps:
-//   0      loads: one TMA box of code words per two groups [128 rows x 32 words] (128-byte swizzle),
-//          X' per group as two [nt x 64] boxes (128-byte swizzle), and the groups' steps and zero
-//          points of the 128 rows (cp.async) into a ring of their own
-//   1      tensor memory; per group the whole warp permutes X' in place and sums Sx_g, then one thread
-//          issues the 8 MMAs (M = 128, N = nt, K = 16) into the group's accumulator
-//   2-9    unpack: warps 2-5 take the first 64 in-features of every group, warps 6-9 the second; lane l
-//          of warp 2 + q + 4h unpacks row 32 q + l into an operand tile (K-major, 128-byte swizzle)
-//   10-13  per group: the accumulator rows of their lane quarter, times step and minus the zero-point
-//          term, added to per-row registers; at the end Y (or this slice's partial sums)
+// CTA (b, c) covers weight rows [128 b, 128 b + 128) and groups [c * gp, (c + 1) * gp) (gp even). The
+// unpacked operand of a group (128 rows x 128 in-features) lives in tensor memory (tcgen05.mma reads A
+// from there), two groups at a time, next to the accumulators. Warps:
+//   0      loads: one TMA box of code words per two groups [128 rows x 32 words] (128-byte swizzle)
+//          and X' per group as two [nt x 64] boxes (128-byte swizzle), each into a ring of its own
+//   1      tensor memory; one thread issues the 8 MMAs of a group (M = 128, N = nt, K = 16)
+//   2-9    unpack: warps 2-5 take the even groups, warps 6-9 the odd ones; lane l of warp w unpacks row
+//          32 (w % 4) + l (the tensor-memory lanes warp w may write) with two 32-column stores; the four
+//          warps of the set also sum Sx_g from the group's X' tile
+//   10-13  per group: S_g of their lane quarter, minus the zero-point term, times step, added to per-row
+//          registers (steps and zero points read from global memory two groups ahead); at the end Y, or
+//          this slice's partial sums
 // With several slices the last CTA of a row block to finish (a per-block counter it resets to zero)
 // adds the slices' partial sums in slice order (deterministic). All waits are bounded; a timeout is
 // recorded in the caller's status word.
@@ -49,35 +46,32 @@ constexpr int GK = 128;                       // in-features per group
 constexpr int UK = 16;                        // K of one MMA
 constexpr int MAX_NT = 64;                    // tokens per launch (the MMA's N, a multiple of 16)
 constexpr int GROUPS_PER_BOX = 2;             // code box: 32 words = 128 bytes per row = 2 groups
-constexpr int C_STAGES = 2;                   // code boxes in flight
 constexpr int C_BYTES = ROWS * 128;           // 16 KB
-constexpr int A_STAGES = 3;                   // unpacked operand tiles (one k-block each)
-constexpr int A_BYTES = ROWS * BK * 2;        // 16 KB
-constexpr int SZ_STAGES = 4;                  // steps and zero points, one group each
-constexpr int SZ_BYTES = 2 * ROWS * 4;        // 1 KB
-constexpr int ACC_STAGES = 4;                 // group accumulators in tensor memory
+constexpr int A_COLS = GK / 2;                // tensor-memory columns of one group's operand (64)
 constexpr int UNPACK_WARPS = 8;
 constexpr int EPI_WARP0 = 2 + UNPACK_WARPS;   // warps 10-13
 constexpr int THREADS = 32 * (EPI_WARP0 + 4);  // 448
 constexpr int MAX_SLICES = 16;
+constexpr int SX_STAGES = 4;                  // Sx_g of the groups in flight between unpack and epilogue
 
 template <int NT>
 struct Shape {
-  static constexpr int X_STAGES = NT == 32 ? 2 : 4;               // X' groups in flight
-  static constexpr int X_BYTES = 2 * NT * 128;                     // one group: two [NT x 64] tiles
-  static constexpr int SX_STAGES = X_STAGES + ACC_STAGES;          // Sx_g ring (see the MMA warp)
-  static constexpr int SMEM = C_STAGES * C_BYTES + A_STAGES * A_BYTES + X_STAGES * X_BYTES +
-                              SZ_STAGES * SZ_BYTES + SX_STAGES * NT * 4 + 2 * NT * 4 + 1024;
-  static constexpr int CTAS_PER_SM = NT <= 32 ? 2 : 1;
-  static constexpr uint32_t TMEM_COLS = ACC_STAGES * NT <= 64 ? 64 : (ACC_STAGES * NT <= 128 ? 128 : 256);
+  static constexpr int CTAS_PER_SM = NT <= 16 ? 2 : 1;
+  static constexpr int C_STAGES = 3;                                    // code boxes in flight
+  static constexpr int X_BYTES = 2 * NT * 128;                          // one group: two [NT x 64] tiles
+  static constexpr int X_STAGES = NT <= 16 ? 8 : (96 * 1024) / X_BYTES; // X' groups in flight
+  static constexpr int ACC_STAGES = 4;                                  // group accumulators S_g
+  static constexpr int A_COL0 = ACC_STAGES * NT;                        // two groups' operands
+  static constexpr int USED_COLS = A_COL0 + 2 * A_COLS;
+  static constexpr uint32_t TMEM_COLS = USED_COLS <= 128 ? 128 : (USED_COLS <= 256 ? 256 : 512);
+  static constexpr int TPT = NT == 16 ? 8 : (NT == 32 ? 4 : 2);         // Sx threads per token
+  static constexpr int SMEM = C_STAGES * C_BYTES + X_STAGES * X_BYTES + SX_STAGES * NT * 4 + 1024;
 };
-static_assert(Shape<16>::SMEM <= 113 * 1024 && Shape<32>::SMEM <= 113 * 1024, "two CTAs per SM");
-static_assert(Shape<64>::SMEM <= 227 * 1024, "one CTA per SM");
+static_assert(Shape<16>::USED_COLS <= 256 && Shape<16>::SMEM <= 113 * 1024, "two CTAs per SM");
+static_assert(Shape<64>::USED_COLS <= 512, "tensor memory");
+static_assert(Shape<64>::SMEM <= 227 * 1024 && Shape<48>::SMEM <= 227 * 1024, "one CTA per SM");
 
-__host__ inline int smem_bytes(int nt) {
-  return nt <= 16 ? Shape<16>::SMEM : nt <= 32 ? Shape<32>::SMEM : nt <= 48 ? Shape<48>::SMEM : Shape<64>::SMEM;
-}
-__host__ inline int ctas_per_sm(int nt) { return nt <= 32 ? 2 : 1; }
+__host__ inline int ctas_per_sm(int nt) { return nt <= 16 ? 2 : 1; }
 
 // Slices of the groups per row block the workspace is sized for: enough for 512 CTAs, at most
 // MAX_SLICES. The workspace holds partial[n_rb][slices][MAX_NT][ROWS] fp32 and one counter per row block.
@@ -146,19 +140,6 @@ __device__ __forceinline__ void epilogue_sync() {  // warps 10-13 only
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
-__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-  return v;
-}
-__device__ __forceinline__ float ld_shared_f32(uint32_t a) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_shared_f32(uint32_t a, float v) {
-  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
-}
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
@@ -168,21 +149,28 @@ __device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
-// (128 + q) as bf16 for the nibbles j and j + 4 of a code word shifted right by 4 j: 0x4300 | q.
-__device__ __forceinline__ uint32_t nibble_pair_bf16(uint32_t w_shifted) {
-  uint32_t r;
-  asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(w_shifted));  // (a & b) | c
-  return r;
+// (128 + q) as bf16 pairs for the in-features 2j and 2j + 1 of a code word (nibbles 2j, 2j + 1 = byte j):
+// a byte permute puts byte j of the word in the low half and byte j of the word shifted right by 4 in the
+// high half, then an AND-OR keeps one nibble per half under the bf16 pattern of 128 (0x4300 | q).
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&v)[4]) {
+  const uint32_t w4 = w >> 4;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t t, r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(w), "r"(w4), "r"(static_cast<uint32_t>(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12))));
+    asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(t));  // (a & b) | c
+    v[j] = r;
+  }
 }
 
 template <int NT>
 __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     w4a16_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC, Params p) {
   using S = Shape<NT>;
+  constexpr int CS = S::C_STAGES, XS = S::X_STAGES, AS = S::ACC_STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[2 * C_STAGES + 2 * A_STAGES + 3 * S::X_STAGES + 2 * SZ_STAGES +
-                                        2 * ACC_STAGES];
+  __shared__ __align__(8) uint64_t bars[2 * CS + 2 * XS + 2 * 2 + 2 * AS + 2 * SX_STAGES];
   __shared__ uint32_t tmem_slot;
   __shared__ int failed;
   __shared__ unsigned int ticket;
@@ -193,58 +181,48 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
   const int slice = static_cast<int>(blockIdx.x) - rb * p.slices;
   const int64_t row0 = static_cast<int64_t>(rb) * ROWS;
   const int g0 = slice * p.g_per;
-  const int ng = max(0, min(p.g_per, p.num_groups - g0));  // even: num_groups and g_per are even
+  const int ng = max(0, min(p.g_per, p.num_groups - g0));
 
   const uint32_t bar0 = smem_u32(&bars[0]);
-  auto cfull_bar = [&](int c) { return bar0 + 8u * c; };
-  auto cempty_bar = [&](int c) { return bar0 + 8u * (C_STAGES + c); };
-  auto dq_bar = [&](int a) { return bar0 + 8u * (2 * C_STAGES + a); };
-  auto afree_bar = [&](int a) { return bar0 + 8u * (2 * C_STAGES + A_STAGES + a); };
-  auto xfull_bar = [&](int x) { return bar0 + 8u * (2 * C_STAGES + 2 * A_STAGES + x); };
-  auto xempty_bar = [&](int x) { return bar0 + 8u * (2 * C_STAGES + 2 * A_STAGES + S::X_STAGES + x); };
-  auto szfull_bar = [&](int z) { return bar0 + 8u * (2 * C_STAGES + 2 * A_STAGES + 2 * S::X_STAGES + z); };
-  auto szempty_bar = [&](int z) {
-    return bar0 + 8u * (2 * C_STAGES + 2 * A_STAGES + 2 * S::X_STAGES + SZ_STAGES + z);
-  };
-  auto accfull_bar = [&](int s) {
-    return bar0 + 8u * (2 * C_STAGES + 2 * A_STAGES + 2 * S::X_STAGES + 2 * SZ_STAGES + s);
-  };
-  auto accempty_bar = [&](int s) {
-    return bar0 + 8u * (2 * C_STAGES + 2 * A_STAGES + 2 * S::X_STAGES + 2 * SZ_STAGES + ACC_STAGES + s);
-  };
+  auto cfull_bar = [&](int c) { return bar0 + 8u * c; };                          // codes landed
+  auto cempty_bar = [&](int c) { return bar0 + 8u * (CS + c); };                  // codes read
+  auto xfull_bar = [&](int x) { return bar0 + 8u * (2 * CS + x); };               // X' landed
+  auto xempty_bar = [&](int x) { return bar0 + 8u * (2 * CS + XS + x); };         // MMAs done with X'
+  auto dq_bar = [&](int a) { return bar0 + 8u * (2 * CS + 2 * XS + a); };         // operand a written
+  auto afree_bar = [&](int a) { return bar0 + 8u * (2 * CS + 2 * XS + 2 + a); };  // MMAs done with it
+  auto accfull_bar = [&](int s) { return bar0 + 8u * (2 * CS + 2 * XS + 4 + s); };
+  auto accempty_bar = [&](int s) { return bar0 + 8u * (2 * CS + 2 * XS + 4 + AS + s); };
+  auto sxfull_bar = [&](int t) { return bar0 + 8u * (2 * CS + 2 * XS + 4 + 2 * AS + t); };
+  auto sxempty_bar = [&](int t) { return bar0 + 8u * (2 * CS + 2 * XS + 4 + 2 * AS + SX_STAGES + t); };
   const uint32_t base = smem_u32(smem);
   auto c_tile = [&](int c) { return base + static_cast<uint32_t>(c) * C_BYTES; };
-  auto a_tile = [&](int a) { return base + C_STAGES * C_BYTES + static_cast<uint32_t>(a) * A_BYTES; };
   auto x_tile = [&](int x, int h) {  // half h (in-features 64 h .. 64 h + 63 of the group)
-    return base + C_STAGES * C_BYTES + A_STAGES * A_BYTES + static_cast<uint32_t>(x) * S::X_BYTES +
-           static_cast<uint32_t>(h * NT * 128);
+    return base + CS * C_BYTES + static_cast<uint32_t>(x) * S::X_BYTES + static_cast<uint32_t>(h * NT * 128);
   };
-  const uint32_t sz_base = base + C_STAGES * C_BYTES + A_STAGES * A_BYTES + S::X_STAGES * S::X_BYTES;
-  auto sz_tile = [&](int z) { return sz_base + static_cast<uint32_t>(z) * SZ_BYTES; };  // [step, zero][row]
-  const uint32_t sx_base = sz_base + SZ_STAGES * SZ_BYTES;
-  auto sx_row = [&](int s) { return sx_base + static_cast<uint32_t>(s * NT * 4); };    // [NT] fp32
-  const uint32_t px_base = sx_base + S::SX_STAGES * NT * 4;                            // [2][NT] fp32
+  auto sx_slot = [&](int t) {  // Sx_g[NT] fp32
+    return base + CS * C_BYTES + XS * S::X_BYTES + static_cast<uint32_t>(t * NT * 4);
+  };
 
   if (threadIdx.x == 0) {
-    for (int c = 0; c < C_STAGES; ++c) {
+    for (int c = 0; c < CS; ++c) {
       mbar_init(cfull_bar(c), 1);
-      mbar_init(cempty_bar(c), UNPACK_WARPS);
+      mbar_init(cempty_bar(c), UNPACK_WARPS);  // each warp reads one of the box's two groups
     }
-    for (int a = 0; a < A_STAGES; ++a) {
-      mbar_init(dq_bar(a), UNPACK_WARPS / 2);  // the four warps of the half that writes the tile
-      mbar_init(afree_bar(a), 1);
-    }
-    for (int x = 0; x < S::X_STAGES; ++x) {
+    for (int x = 0; x < XS; ++x) {
       mbar_init(xfull_bar(x), 1);
       mbar_init(xempty_bar(x), 1);
     }
-    for (int z = 0; z < SZ_STAGES; ++z) {
-      mbar_init(szfull_bar(z), 32);  // the loader lanes' cp.async arrivals
-      mbar_init(szempty_bar(z), 4);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(dq_bar(a), UNPACK_WARPS / 2);  // the four warps of the set that writes operand a
+      mbar_init(afree_bar(a), 1);
     }
-    for (int s = 0; s < ACC_STAGES; ++s) {
-      mbar_init(accfull_bar(s), 2);  // the MMAs' commit and the MMA thread (Sx_g written)
+    for (int s = 0; s < AS; ++s) {
+      mbar_init(accfull_bar(s), 1);
       mbar_init(accempty_bar(s), 4);
+    }
+    for (int t = 0; t < SX_STAGES; ++t) {
+      mbar_init(sxfull_bar(t), UNPACK_WARPS / 2);
+      mbar_init(sxempty_bar(t), 4);
     }
     failed = 0;
     ticket = 0u;
@@ -252,22 +230,23 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmC);
   }
-  // Loads of local group i: its code box when i is even (the box holds groups i and i + 1), X', and
-  // the steps and zero points. Warp 0 only, all lanes; false when a wait gave up.
+  // Loads of local group i: its code box when i is even (the box holds groups i and i + 1) and X'.
+  // Warp 0 only, all lanes; false when a wait gave up.
   auto load_codes = [&](int i) -> bool {
     const int j = i / GROUPS_PER_BOX;
-    const int c = j % C_STAGES;
-    const uint32_t use = static_cast<uint32_t>(j / C_STAGES);
+    const int c = j % CS;
+    const uint32_t use = static_cast<uint32_t>(j / CS);
     if (use > 0 && !wait_warp(cempty_bar(c), (use - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
     if (lane == 0) {
       mbar_arrive_expect_tx(cfull_bar(c), C_BYTES);
       tma_load_2d(c_tile(c), &tmC, (g0 + i) * (GK / 8), static_cast<int32_t>(row0), cfull_bar(c));
     }
+    __syncwarp();
     return true;
   };
   auto load_x = [&](int i) -> bool {
-    const int x = i % S::X_STAGES;
-    const uint32_t use = static_cast<uint32_t>(i / S::X_STAGES);
+    const int x = i % XS;
+    const uint32_t use = static_cast<uint32_t>(i / XS);
     if (use > 0 && !wait_warp(xempty_bar(x), (use - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
     if (lane == 0) {
       mbar_arrive_expect_tx(xfull_bar(x), S::X_BYTES);
@@ -277,31 +256,14 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     __syncwarp();
     return true;
   };
-  auto load_sz = [&](int i) -> bool {
-    const int z = i % SZ_STAGES;
-    const uint32_t use = static_cast<uint32_t>(i / SZ_STAGES);
-    if (use > 0 && !wait_warp(szempty_bar(z), (use - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
-    const int64_t g = g0 + i;
-#pragma unroll
-    for (int jr = 0; jr < ROWS / 32; ++jr) {
-      const int r = lane + 32 * jr;
-      const int64_t o = min(row0 + r, p.O - 1);  // rows past O: any valid address (their codes are 0)
-      cp_async_4(sz_tile(z) + 4u * r, p.steps + o * p.G + g);
-      cp_async_4(sz_tile(z) + 4u * (ROWS + r), p.zeros + o * p.G + g);
-    }
-    cp_async_mbar_arrive(szfull_bar(z));
-    return true;
-  };
   // The first groups need no free slots: warp 0 requests them right after initialising the barriers, so
   // the first memory round trip overlaps the tensor-memory allocation and the CTA barrier.
-  const int pre_c = min(ng, C_STAGES * GROUPS_PER_BOX);
-  const int pre_x = min(ng, S::X_STAGES);
-  const int pre_z = min(ng, SZ_STAGES);
+  const int pre_c = min(ng, CS * GROUPS_PER_BOX);
+  const int pre_x = min(ng, XS);
   if (warp == 0) {
     __syncwarp();  // the barriers thread 0 initialised are visible to the whole warp
     for (int i = 0; i < pre_c; i += GROUPS_PER_BOX) load_codes(i);
     for (int i = 0; i < pre_x; ++i) load_x(i);
-    for (int i = 0; i < pre_z; ++i) load_sz(i);
   }
   if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), S::TMEM_COLS);
   tc_fence_before();
@@ -311,169 +273,183 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
 
   if (warp == 0) {
     // ------------------------------------------------------------------------------ loads
+    // Both rings are refilled in group order: a code box once its slot is free (the box CS boxes
+    // earlier unpacked), X' once its slot is (the MMAs XS groups earlier done).
     for (int i = 0; i < ng; ++i) {
       bool ok = true;
       if (i >= pre_c && i % GROUPS_PER_BOX == 0) ok = load_codes(i);
       if (ok && i >= pre_x) ok = load_x(i);
-      if (ok && i >= pre_z) ok = load_sz(i);
       if (!ok) {
         failed = 1;
         break;
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------------------ X' and MMA
-    // Per group: permute X' inside each 16-byte chunk to the unpacked operand's order 0 4 1 5 2 6 3 7
-    // and sum Sx_g[m] (fp32, in a fixed order: each of the two halves in chunk and then element order,
-    // then first half plus second half); then one thread issues the MMAs.
-    bool ok = true;
-    for (int i = 0; i < ng && ok; ++i) {
-      const int x = i % S::X_STAGES;
-      const int s = i % ACC_STAGES;
-      if (!wait_warp(xfull_bar(x), static_cast<uint32_t>(i / S::X_STAGES) & 1u, p, kSiteDecodeFull)) {
-        ok = false;
-        break;
-      }
-#pragma unroll 1
-      for (int item = lane; item < 2 * NT; item += 32) {  // (half h, token m)
-        const int h = item / NT, m = item - h * NT;
-        const uint32_t row = x_tile(x, h) + static_cast<uint32_t>(m) * 128u;
-        float sum = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t a = row + ((static_cast<uint32_t>(c) ^ static_cast<uint32_t>(m & 7)) << 4);
-          const uint4 v = ld_shared_v4(a);  // (k0 k1) (k2 k3) (k4 k5) (k6 k7)
-          const uint32_t e[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            sum = __fadd_rn(sum, __uint_as_float(e[t] << 16));
-            sum = __fadd_rn(sum, __uint_as_float(e[t] & 0xFFFF0000u));
-          }
-          st_shared_v4(a, make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
-                                     __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632)));
-        }
-        st_shared_f32(px_base + 4u * static_cast<uint32_t>(item), sum);
-      }
-      fence_proxy_async_smem();  // the MMAs read the permuted X' through the async proxy
-      __syncwarp();
-      for (int m = lane; m < NT; m += 32)
-        st_shared_f32(sx_row(i % S::SX_STAGES) + 4u * m,
-                      __fadd_rn(ld_shared_f32(px_base + 4u * m), ld_shared_f32(px_base + 4u * (NT + m))));
-      __syncwarp();
-      if (lane == 0) {
-        const int a0 = (2 * i) % A_STAGES, a1 = (2 * i + 1) % A_STAGES;
-        const uint32_t acc_use = static_cast<uint32_t>(i / ACC_STAGES);
-        if (!wait_thread(dq_bar(a0), static_cast<uint32_t>((2 * i) / A_STAGES) & 1u, p, kSiteDecodeDequant) ||
-            !wait_thread(dq_bar(a1), static_cast<uint32_t>((2 * i + 1) / A_STAGES) & 1u, p, kSiteDecodeDequant) ||
+    // ------------------------------------------------------------------------------ MMA
+    if (elect_one()) {
+      bool ok = true;
+      for (int i = 0; i < ng && ok; ++i) {
+        const int x = i % XS, s = i % AS, a = i % 2;
+        const uint32_t acc_use = static_cast<uint32_t>(i / AS);
+        if (!wait_thread(xfull_bar(x), static_cast<uint32_t>(i / XS) & 1u, p, kSiteDecodeFull) ||
+            !wait_thread(dq_bar(a), static_cast<uint32_t>(i / 2) & 1u, p, kSiteDecodeDequant) ||
             (acc_use > 0 && !wait_thread(accempty_bar(s), (acc_use - 1u) & 1u, p, kSiteDecodeAcc))) {
           ok = false;
-        } else {
-          tc_fence_after();
-          const uint32_t d = tmem_base + static_cast<uint32_t>(s * NT);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t at = a_tile(h == 0 ? a0 : a1), xt = x_tile(x, h);
-#pragma unroll
-            for (int kk = 0; kk < BK / UK; ++kk)
-              umma_bf16(d, smem_desc_sw128(at + kk * UK * 2), smem_desc_sw128(xt + kk * UK * 2), p.idesc,
-                        (h | kk) != 0 ? 1u : 0u);
-          }
-          umma_commit(afree_bar(a0));
-          umma_commit(afree_bar(a1));
-          umma_commit(xempty_bar(x));
-          umma_commit(accfull_bar(s));
-          mbar_arrive(accfull_bar(s));  // after the warp's Sx_g stores (ordered by the __syncwarp above)
+          break;
         }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(s * NT);
+        const uint32_t at = tmem_base + static_cast<uint32_t>(S::A_COL0 + a * A_COLS);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk)
+            umma_bf16_ts(d, at + static_cast<uint32_t>((h * (BK / UK) + kk) * (UK / 2)),
+                         smem_desc_sw128(x_tile(x, h) + kk * UK * 2), p.idesc, (h | kk) != 0 ? 1u : 0u);
+        umma_commit(afree_bar(a));
+        umma_commit(xempty_bar(x));
+        umma_commit(accfull_bar(s));
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) failed = 1;
     }
-    if (!ok) failed = 1;
     __syncwarp();
   } else if (warp < EPI_WARP0) {
-    // ------------------------------------------------------------------------------ unpack
-    const int q = (warp - 2) & 3, h = (warp - 2) >> 2;
+    // ------------------------------------------------------------------------------ unpack and Sx_g
+    // Warps 2-5 take the even groups into operand 0, 6-9 the odd ones into operand 1.
+    const int q = warp & 3, set = (warp - 2) >> 2;
     const int r = 32 * q + lane;
     const uint32_t sw = static_cast<uint32_t>(r & 7);
-    for (int i = 0; i < ng; ++i) {
-      const int j = i / GROUPS_PER_BOX, c = j % C_STAGES;
-      const int kb = 2 * i + h, a = kb % A_STAGES;
-      if (!wait_warp(cfull_bar(c), static_cast<uint32_t>(j / C_STAGES) & 1u, p, kSiteDecodeFull)) {
+    const uint32_t tl = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    // Sx_g: thread tt of the set's 128 sums 16 / TPT chunks (8 in-features each) of token tt / TPT, in
+    // chunk and element order; the TPT threads of a token (adjacent lanes) then add by a fixed tree.
+    constexpr int TPT = S::TPT, CPT = 16 / TPT;
+    const int tt = 32 * q + lane, m_sx = tt / TPT, part = tt % TPT;
+    for (int i = set; i < ng; i += 2) {
+      const int j = i / GROUPS_PER_BOX, c = j % CS;
+      const int x = i % XS, t = i % SX_STAGES;
+      if (!wait_warp(cfull_bar(c), static_cast<uint32_t>(j / CS) & 1u, p, kSiteDecodeFull)) {
         failed = 1;
         break;
       }
-      // words 16 (i % 2) + 8 h .. + 7 of row r: 16-byte chunks 4 (i % 2) + 2 h and + 1 of its swizzled line
-      const uint32_t chunk = static_cast<uint32_t>(4 * (i % GROUPS_PER_BOX) + 2 * h);
-      const uint4 w0 = ld_shared_v4(c_tile(c) + static_cast<uint32_t>(r) * 128u + ((chunk ^ sw) << 4));
-      const uint4 w1 = ld_shared_v4(c_tile(c) + static_cast<uint32_t>(r) * 128u + (((chunk + 1u) ^ sw) << 4));
-      const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      __syncwarp();
-      // the warp's last group of the box hands it back (the words are in registers)
-      if (lane == 0 && (i % GROUPS_PER_BOX == GROUPS_PER_BOX - 1 || i + 1 >= ng)) mbar_arrive(cempty_bar(c));
-      const uint32_t ause = static_cast<uint32_t>(kb / A_STAGES);
-      if (ause > 0 && !wait_warp(afree_bar(a), (ause - 1u) & 1u, p, kSiteDecodeEmpty)) {
-        failed = 1;
-        break;
-      }
-      const uint32_t line = a_tile(a) + static_cast<uint32_t>(r) * 128u;
+      // words 16 (i % 2) .. + 15 of row r: 16-byte chunks 4 (i % 2) .. + 3 of its swizzled line
+      const uint32_t line_c = c_tile(c) + static_cast<uint32_t>(r) * 128u;
+      uint4 wv[4];
 #pragma unroll
-      for (int t = 0; t < 8; ++t)
-        st_shared_v4(line + ((static_cast<uint32_t>(t) ^ sw) << 4),
-                     make_uint4(nibble_pair_bf16(w[t]), nibble_pair_bf16(w[t] >> 4), nibble_pair_bf16(w[t] >> 8),
-                                nibble_pair_bf16(w[t] >> 12)));
-      fence_proxy_async_smem();  // the tensor cores read the tile through the async proxy
+      for (int u = 0; u < 4; ++u)
+        wv[u] = ld_shared_v4(line_c + (((static_cast<uint32_t>(4 * (i % GROUPS_PER_BOX) + u)) ^ sw) << 4));
       __syncwarp();
-      if (lane == 0) mbar_arrive(dq_bar(a));
+      if (lane == 0) mbar_arrive(cempty_bar(c));  // the words are in registers
+      // Sx_g from the group's X' tile
+      const uint32_t sx_use = static_cast<uint32_t>(i / SX_STAGES);
+      if (!wait_warp(xfull_bar(x), static_cast<uint32_t>(i / XS) & 1u, p, kSiteDecodeFull) ||
+          (sx_use > 0 && !wait_warp(sxempty_bar(t), (sx_use - 1u) & 1u, p, kSiteDecodeEmpty))) {
+        failed = 1;
+        break;
+      }
+      float sum = 0.0f;
+      if (m_sx < NT) {
+#pragma unroll
+        for (int u = 0; u < CPT; ++u) {
+          const int ch = part * CPT + u, h = ch >> 3, cc = ch & 7;
+          const uint4 v = ld_shared_v4(x_tile(x, h) + static_cast<uint32_t>(m_sx) * 128u +
+                                       ((static_cast<uint32_t>(cc) ^ static_cast<uint32_t>(m_sx & 7)) << 4));
+          const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            sum = __fadd_rn(__fadd_rn(sum, __uint_as_float(e[k] << 16)), __uint_as_float(e[k] & 0xFFFF0000u));
+        }
+      }
+#pragma unroll
+      for (int off = 1; off < TPT; off <<= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, off));
+      if (part == 0 && m_sx < NT)
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_slot(t) + 4u * static_cast<uint32_t>(m_sx)), "f"(sum) : "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sxfull_bar(t));
+      // the operand
+      const uint32_t ause = static_cast<uint32_t>(i / 2);
+      if (ause > 0 && !wait_warp(afree_bar(set), (ause - 1u) & 1u, p, kSiteDecodeEmpty)) {
+        failed = 1;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t w[8] = {wv[2 * h].x, wv[2 * h].y, wv[2 * h].z, wv[2 * h].w,
+                               wv[2 * h + 1].x, wv[2 * h + 1].y, wv[2 * h + 1].z, wv[2 * h + 1].w};
+        uint32_t v[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          uint32_t v4[4];
+          unpack_word(w[u], v4);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) v[4 * u + k] = v4[k];
+        }
+        tmem_st32(tl + static_cast<uint32_t>(S::A_COL0 + set * A_COLS + h * (A_COLS / 2)), v);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_bar(set));
     }
   } else {
     // ------------------------------------------------------------------------------ group epilogue
     const int q = warp & 3;  // tensor-memory lane quarter this warp may read
     const int r = 32 * q + lane;
     const uint32_t tlane = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    const int64_t o_ld = min(row0 + r, p.O - 1);  // rows past O: any valid address (results dropped)
+    const float* st_row = p.steps + o_ld * p.G + g0;
+    const float* z_row = p.zeros + o_ld * p.G + g0;
     float y[NT];
 #pragma unroll
     for (int m = 0; m < NT; ++m) y[m] = 0.0f;
+    // steps and zero points two groups ahead
+    float st_n[2], z_n[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      st_n[u] = u < ng ? __ldg(st_row + u) : 0.0f;
+      z_n[u] = u < ng ? __ldg(z_row + u) : 0.0f;
+    }
     bool have = true;
     for (int i = 0; i < ng; ++i) {
-      const int z = i % SZ_STAGES, s = i % ACC_STAGES;
-      if (!wait_warp(szfull_bar(z), static_cast<uint32_t>(i / SZ_STAGES) & 1u, p, kSiteDecodeFull)) {
-        have = false;
-        break;
-      }
-      const float step = ld_shared_f32(sz_tile(z) + 4u * r);
-      const float c = __fadd_rn(128.0f, ld_shared_f32(sz_tile(z) + 4u * (ROWS + r)));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(szempty_bar(z));
-      if (!wait_warp(accfull_bar(s), static_cast<uint32_t>(i / ACC_STAGES) & 1u, p, kSiteDecodeAcc)) {
+      const int s = i % AS, t = i % SX_STAGES;
+      const float step = st_n[0];
+      const float c = __fadd_rn(128.0f, z_n[0]);
+      st_n[0] = st_n[1];
+      z_n[0] = z_n[1];
+      st_n[1] = i + 2 < ng ? __ldg(st_row + i + 2) : 0.0f;
+      z_n[1] = i + 2 < ng ? __ldg(z_row + i + 2) : 0.0f;
+      if (!wait_warp(accfull_bar(s), static_cast<uint32_t>(i / AS) & 1u, p, kSiteDecodeAcc) ||
+          !wait_warp(sxfull_bar(t), static_cast<uint32_t>(i / SX_STAGES) & 1u, p, kSiteDecodeAcc)) {
         have = false;
         break;
       }
       tc_fence_after();
-      // 16 accumulator columns at a time: y[m] += step * (S_g[r, m] - (128 + z) * Sx_g[m])
-      const uint32_t sx = sx_row(i % S::SX_STAGES);
+      // 16 columns at a time: y[m] += step * (S_g[r, m] - (128 + z) * Sx_g[m])
 #pragma unroll
       for (int cc = 0; cc < NT / 16; ++cc) {
-        float t16[16];
-        tmem_ld16(tlane + static_cast<uint32_t>(s * NT + 16 * cc), t16);
+        float sg[16];
+        tmem_ld16(tlane + static_cast<uint32_t>(s * NT + 16 * cc), sg);
 #pragma unroll
-        for (int m4 = 0; m4 < 16; m4 += 4) {
+        for (int k4 = 0; k4 < 16; k4 += 4) {
           float4 xs;
           asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                        : "=f"(xs.x), "=f"(xs.y), "=f"(xs.z), "=f"(xs.w)
-                       : "r"(sx + 4u * static_cast<uint32_t>(16 * cc + m4))
+                       : "r"(sx_slot(t) + 4u * static_cast<uint32_t>(16 * cc + k4))
                        : "memory");
           const float xv[4] = {xs.x, xs.y, xs.z, xs.w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int m = 16 * cc + m4 + k;
-            y[m] = __fmaf_rn(step, __fmaf_rn(-c, xv[k], t16[m4 + k]), y[m]);
+            const int m = 16 * cc + k4 + k;
+            y[m] = __fmaf_rn(step, __fmaf_rn(-c, xv[k], sg[k4 + k]), y[m]);
           }
         }
       }
-      // The accumulator and this group's Sx_g are read: hand both back (the Sx ring is sized so that
-      // its slot is rewritten only after this arrival).
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(accempty_bar(s));
+      if (lane == 0) {
+        mbar_arrive(accempty_bar(s));
+        mbar_arrive(sxempty_bar(t));
+      }
     }
     if (!have) failed = 1;
     if (p.slices == 1) {
