@@ -258,9 +258,13 @@ AWQ_API awq_status awq_scale_rows(const void *A, int64_t R, int64_t C, int64_t l
 /* ---------------------------------------------------------------------------------------------------
  * Deployment GEMM of a quantized linear (W4A16): Y = X' deq(W)^T, the weights read as the packed codes,
  * steps and zeros of awq_quantize_pack and dequantized on the fly ("GPU 硬件级反量化算子内联融合" on the
- * bjdmk.com.cn AWQ article): deq(W)[o, k] = bf16(RN32(RN32(q[o,k] - z[o,g]) * step[o,g])), g = k / 128.
+ * bjdmk.com.cn AWQ article), deq(W)[o, k] = (q[o,k] - z[o,g]) * step[o,g], g = k / 128.
  * X' is the layer input with the AWQ scales already folded out (X diag(s)^-1, e.g. by awq_scale_columns
- * on the previous norm weight). bf16 x bf16 products, fp32 accumulation on the tensor cores, bf16 output.
+ * on the previous norm weight). fp32 accumulation on the tensor cores, bf16 output. The weight enters as:
+ *   M > 64 tokens:  bf16(RN32(RN32(q - z) * step)), dequantized into the tensor-core operand tiles;
+ *   M <= 64 tokens: its exact value: the tensor cores sum (128 + q) * x' per group of 128 in-features
+ *                   (exact bf16 operands) and the step and zero point are applied per group and output,
+ *                   Y = sum_g step_g * (S_g - (128 + z_g) * sum_{k in g} x'_k), in fp32.
  *   X       device bf16 [M, K], row stride ldx (multiple of 8)
  *   codes   device uint32 [O, K/8], steps / zeros device float [O, K/128] (contiguous, as packed)
  *   Y       device bf16 [M, O], row stride ldy (multiple of 8)
@@ -271,8 +275,8 @@ AWQ_API awq_status awq_scale_rows(const void *A, int64_t R, int64_t C, int64_t l
  *              whatever their shapes), a group-major copy of steps and zeros (many tokens) and split-K
  *              partial sums (few tokens).
  * Requires K % 128 == 0, O % 8 == 0, M >= 1. M <= 64 runs a few-token kernel (weight rows on the MMA's M
- * side, K split across CTAs, partial sums added in a fixed order). A device timeout is reported by
- * awq_search_status() on the same workspace.
+ * side, groups split across CTAs, partial sums added in a fixed order). Both are deterministic. A device
+ * timeout is reported by awq_search_status() on the same workspace.
  * ------------------------------------------------------------------------------------------------- */
 AWQ_API size_t awq_w4a16_workspace_size(int64_t K, int64_t O);
 AWQ_API awq_status awq_w4a16_gemm(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *codes,

@@ -15,6 +15,11 @@
 // masks, convert, apply the group scale and offset; here the scale and offset are applied after the
 // products of each group).
 //
+// Nibble order. A code word holds in-features 8c .. 8c+7 in nibbles 0..7. One AND-OR per register turns
+// the word shifted right by 4j into the bf16 pair (128 + q_j, 128 + q_{j+4}), so the operand row holds
+// each word's in-features in the order 0 4 1 5 2 6 3 7. X' is permuted the same way inside every 16-byte
+// chunk (8 in-features) by the warps that sum Sx_g from it, which leaves the products and sums unchanged.
+//
 // CTA (b, c) covers weight rows [128 b, 128 b + 128) and groups [c * gp, (c + 1) * gp) (gp even). The
 // unpacked operand of a group (128 rows x 128 in-features) lives in tensor memory (tcgen05.mma reads A
 // from there), two groups at a time, next to the accumulators. Warps:
@@ -23,7 +28,7 @@
 //   1      tensor memory; one thread issues the 8 MMAs of a group (M = 128, N = nt, K = 16)
 //   2-9    unpack: warps 2-5 take the even groups, warps 6-9 the odd ones; lane l of warp w unpacks row
 //          32 (w % 4) + l (the tensor-memory lanes warp w may write) with two 32-column stores; the four
-//          warps of the set also sum Sx_g from the group's X' tile
+//          warps of the set also sum Sx_g from the group's X' tile and permute it in place
 //   10-13  per group: S_g of their lane quarter, minus the zero-point term, times step, added to per-row
 //          registers (steps and zero points read from global memory two groups ahead); at the end Y, or
 //          this slice's partial sums
@@ -103,13 +108,15 @@ struct Params {
 
 // Bounded wait by one thread; records a timeout (never reads the status, so a stale word from an earlier
 // call cannot cut this one short).
+// The waits let the hardware suspend the waiting threads (up to 20 us per try) instead of spinning, so
+// waiting warps take few issue slots from the unpack warps.
+constexpr uint32_t kSleepNs = 20000;
+
 __device__ __forceinline__ bool wait_thread(uint32_t bar, uint32_t parity, const Params& p, unsigned int where) {
-#pragma unroll 1
-  for (int i = 0; i < 256; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
   const uint64_t t0 = global_timer_ns();
 #pragma unroll 1
-  while (!mbar_try_wait(bar, parity))
+  while (!mbar_try_wait_sleep(bar, parity, kSleepNs))
     if (global_timer_ns() - t0 > p.limit_ns) {
       raise_timeout(p.status, where);
       return false;
@@ -120,15 +127,15 @@ __device__ __forceinline__ bool wait_thread(uint32_t bar, uint32_t parity, const
 // Warp-uniform bounded wait: every lane polls, the warp leaves together.
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const Params& p, unsigned int where) {
   // the phase has usually completed already: one poll before the timer is read
-  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  if (__all_sync(0xffffffffu, mbar_try_wait_sleep(bar, parity, kSleepNs))) return true;
   const int lane = threadIdx.x & 31;
   uint64_t t0 = 0;
   if (lane == 0) t0 = global_timer_ns();
 #pragma unroll 1
   for (uint32_t it = 0;; ++it) {
-    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    if (__all_sync(0xffffffffu, mbar_try_wait_sleep(bar, parity, kSleepNs))) return true;
     int give_up = 0;
-    if (lane == 0 && (it & 63u) == 63u && global_timer_ns() - t0 > p.limit_ns) {
+    if (lane == 0 && global_timer_ns() - t0 > p.limit_ns) {
       raise_timeout(p.status, where);
       give_up = 1;
     }
@@ -149,18 +156,25 @@ __device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
-// (128 + q) as bf16 pairs for the in-features 2j and 2j + 1 of a code word (nibbles 2j, 2j + 1 = byte j):
-// a byte permute puts byte j of the word in the low half and byte j of the word shifted right by 4 in the
-// high half, then an AND-OR keeps one nibble per half under the bf16 pattern of 128 (0x4300 | q).
+// (128 + q) as bf16 pairs from a code word: register j holds the nibbles j and j + 4 (in-features 8c + j and
+// 8c + j + 4 of word c) in its low and high half, 0x4300 | q each. The word shifted right by 4 j (a
+// multiply-high by 2^(32 - 4 j), which runs on the FMA pipe and leaves the ALU pipe to the AND-ORs)
+// brings both nibbles to bits 0-3 and 16-19.
+__device__ __forceinline__ uint32_t nibble_pair_bf16(uint32_t w_shifted) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(w_shifted));  // (a & b) | c
+  return r;
+}
+__device__ __forceinline__ uint32_t shr_fma(uint32_t w, uint32_t pow2) {
+  uint32_t r;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(pow2));
+  return r;
+}
 __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&v)[4]) {
-  const uint32_t w4 = w >> 4;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    uint32_t t, r;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(w), "r"(w4), "r"(static_cast<uint32_t>(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12))));
-    asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(t));  // (a & b) | c
-    v[j] = r;
-  }
+  v[0] = nibble_pair_bf16(w);
+  v[1] = nibble_pair_bf16(shr_fma(w, 1u << 28));
+  v[2] = nibble_pair_bf16(shr_fma(w, 1u << 24));
+  v[3] = nibble_pair_bf16(shr_fma(w, 1u << 20));
 }
 
 template <int NT>
@@ -351,14 +365,19 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
 #pragma unroll
         for (int u = 0; u < CPT; ++u) {
           const int ch = part * CPT + u, h = ch >> 3, cc = ch & 7;
-          const uint4 v = ld_shared_v4(x_tile(x, h) + static_cast<uint32_t>(m_sx) * 128u +
-                                       ((static_cast<uint32_t>(cc) ^ static_cast<uint32_t>(m_sx & 7)) << 4));
+          const uint32_t a = x_tile(x, h) + static_cast<uint32_t>(m_sx) * 128u +
+                             ((static_cast<uint32_t>(cc) ^ static_cast<uint32_t>(m_sx & 7)) << 4);
+          const uint4 v = ld_shared_v4(a);  // (k0 k1) (k2 k3) (k4 k5) (k6 k7)
           const uint32_t e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             sum = __fadd_rn(__fadd_rn(sum, __uint_as_float(e[k] << 16)), __uint_as_float(e[k] & 0xFFFF0000u));
+          // the operand's order 0 4 1 5 2 6 3 7
+          st_shared_v4(a, make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
+                                     __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632)));
         }
       }
+      fence_proxy_async_smem();  // the MMAs read the permuted X' through the async proxy
 #pragma unroll
       for (int off = 1; off < TPT; off <<= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, off));
       if (part == 0 && m_sx < NT)
