@@ -776,7 +776,6 @@ namespace {
 struct W4Layout {
   int64_t O_pad, G, n_rb;
   size_t steps_off, zeros_off, counter_off, partial_off, bytes;
-  int64_t units_per_rb, segs;  // few tokens: units (pairs of groups) per row block, partial slots per block
 };
 constexpr int64_t kW4MaxRowBlocks = 65536;  // few-token counters reserved for O up to 8M rows
 // [0, 512) status word and tile counter (cleared by each many-token call); [512, 512 + 256 KB) the
@@ -793,16 +792,15 @@ W4Layout w4_layout(int64_t K, int64_t O) {
   l.zeros_off = align_up(l.steps_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
   l.partial_off = align_up(l.zeros_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
   const int64_t rb = std::min(l.n_rb, kW4MaxRowBlocks);
-  l.units_per_rb = (l.G + 1) / 2;
-  l.segs = awq::dec::max_segs(rb, l.units_per_rb);
-  l.bytes = align_up(l.partial_off + static_cast<size_t>(rb) * l.segs * awq::dec::MAX_NT * awq::dec::ROWS * 4, 256);
+  l.bytes = align_up(l.partial_off + static_cast<size_t>(rb) * awq::dec::max_slices(rb) * awq::dec::MAX_NT *
+                                         awq::dec::ROWS * 4,
+                     256);
   return l;
 }
 
-// Few tokens: weight rows on the MMA's M side; the units (pairs of groups of a row block) are split evenly
-// over one wave of CTAs, and a row block shared by several CTAs is finished by the last of them. One
-// launch; the per-block counters are zero from the caller's initial zero fill and every call leaves them
-// zero.
+// Few tokens: weight rows on the MMA's M side, groups split into slices until every SM has a share,
+// slices added by the last CTA of each row block. One launch; the per-block counters are zero from the
+// caller's initial zero fill and every call leaves them zero.
 awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const uint32_t* codes, const float* steps,
                         const float* zeros, int64_t O, void* Y, int64_t ldy, void* workspace, const W4Layout& l,
                         awq_stream_t stream) {
@@ -810,9 +808,12 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   AWQ_TRY(device_info(&d));
   const int nt = static_cast<int>((M + 15) / 16 * 16);
   const int num_groups = static_cast<int>(K / 128);
-  const int64_t units = l.n_rb * l.units_per_rb;
-  const int64_t n_ctas = std::min<int64_t>({static_cast<int64_t>(awq::dec::ctas_per_sm(nt)) * d->sms, units,
-                                            awq::dec::MAX_CTAS});
+  // one wave of CTAs; a slice holds an even number of groups (one code box covers two)
+  int64_t slices = awq::dec::ctas_per_sm(nt) * static_cast<int64_t>(d->sms) / l.n_rb;
+  slices = std::max<int64_t>(1, std::min<int64_t>({slices, awq::dec::max_slices(l.n_rb), (num_groups + 1) / 2}));
+  const int g_per = static_cast<int>(((num_groups + slices - 1) / slices + 1) / 2 * 2);
+  slices = (num_groups + g_per - 1) / g_per;
+  if (l.n_rb * slices >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "O is too large");
   CUtensorMap tmX, tmC;
   AWQ_TRY(make_tmap(&tmX, X, M, K, ldx, nt));
   AWQ_TRY(make_tmap_codes_sw128(&tmC, codes, O, K / 8, awq::dec::ROWS));
@@ -829,14 +830,12 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   p.G = l.G;
   p.ldy = ldy;
   p.num_groups = num_groups;
-  p.units = units;
-  p.units_per_rb = static_cast<int>(l.units_per_rb);
-  p.n_ctas = static_cast<int>(n_ctas);
-  p.segs = static_cast<int>(l.segs);
+  p.g_per = g_per;
+  p.slices = static_cast<int>(slices);
   p.idesc = awq::idesc_bf16_f32(awq::dec::ROWS, static_cast<uint32_t>(nt));
   p.status = reinterpret_cast<awq::DeviceStatus*>(ws);
   p.limit_ns = g_wait_limit_ns.load();
-  const dim3 grid(static_cast<unsigned>(n_ctas));
+  const dim3 grid(static_cast<unsigned>(l.n_rb * slices));
   if (nt == 16)
     awq::dec::w4a16_decode_kernel<16><<<grid, awq::dec::THREADS, awq::dec::Shape<16>::SMEM, st>>>(tmX, tmC, p);
   else if (nt == 32)

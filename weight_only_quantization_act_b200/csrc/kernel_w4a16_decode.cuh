@@ -20,9 +20,7 @@
 // each word's in-features in the order 0 4 1 5 2 6 3 7. X' is permuted the same way inside every 16-byte
 // chunk (8 in-features) by the warps that sum Sx_g from it, which leaves the products and sums unchanged.
 //
-// Work units are pairs of groups (one code box) of one row block of 128 weight rows, numbered row block
-// by row block; CTA c of C takes the contiguous units [c U / C, (c + 1) U / C), so every CTA has the same
-// work to within one unit, and a CTA's run may end in one row block and go on in the next (stream-K). The
+// CTA (b, c) covers weight rows [128 b, 128 b + 128) and groups [c * gp, (c + 1) * gp) (gp even). The
 // unpacked operand of a group (128 rows x 128 in-features) lives in tensor memory (tcgen05.mma reads A
 // from there), two groups at a time, next to the accumulators. Warps:
 //   0      loads: one TMA box of code words per two groups [128 rows x 32 words] (128-byte swizzle)
@@ -32,12 +30,11 @@
 //          32 (w % 4) + l (the tensor-memory lanes warp w may write) with two 32-column stores; the four
 //          warps of the set also sum Sx_g from the group's X' tile and permute it in place
 //   10-13  per group: S_g of their lane quarter, minus the zero-point term, times step, added to per-row
-//          registers (steps and zero points read from global memory two groups ahead); at the end of a
-//          row block's run, Y (a row block in one CTA) or that CTA's partial sums
-// A row block shared by several CTAs is finished by the last of them (a per-block counter it resets to
-// zero), which adds the partial sums in CTA order (deterministic). With an odd number of groups the last
-// unit of each row block has a second, empty group (zero codes, zero X', zero step). All waits are
-// bounded; a timeout is recorded in the caller's status word.
+//          registers (steps and zero points read from global memory two groups ahead); at the end Y, or
+//          this slice's partial sums
+// With several slices the last CTA of a row block to finish (a per-block counter it resets to zero)
+// adds the slices' partial sums in slice order (deterministic). All waits are bounded; a timeout is
+// recorded in the caller's status word.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -59,6 +56,7 @@ constexpr int A_COLS = GK / 2;                // tensor-memory columns of one gr
 constexpr int UNPACK_WARPS = 8;
 constexpr int EPI_WARP0 = 2 + UNPACK_WARPS;   // warps 10-13
 constexpr int THREADS = 32 * (EPI_WARP0 + 4);  // 448
+constexpr int MAX_SLICES = 16;
 constexpr int SX_STAGES = 4;                  // Sx_g of the groups in flight between unpack and epilogue
 
 template <int NT>
@@ -80,12 +78,10 @@ static_assert(Shape<64>::SMEM <= 227 * 1024 && Shape<48>::SMEM <= 227 * 1024, "o
 
 __host__ inline int ctas_per_sm(int nt) { return nt <= 16 ? 2 : 1; }
 
-constexpr int64_t MAX_CTAS = 512;
-
-// Partial-sum slots per row block the workspace holds (partial[n_rb][segs][MAX_NT][ROWS] fp32): a row
-// block of `units` units is shared by at most min(units, C / n_rb + 2) of C <= MAX_CTAS CTAs.
-__host__ __device__ constexpr int64_t max_segs(int64_t n_rb, int64_t units) {
-  return units < MAX_CTAS / n_rb + 2 ? units : MAX_CTAS / n_rb + 2;
+// Slices of the groups per row block the workspace is sized for: enough for 512 CTAs, at most
+// MAX_SLICES. The workspace holds partial[n_rb][slices][MAX_NT][ROWS] fp32 and one counter per row block.
+__host__ __device__ constexpr int64_t max_slices(int64_t n_rb) {
+  return n_rb >= 512 ? 1 : ((512 + n_rb - 1) / n_rb < MAX_SLICES ? (512 + n_rb - 1) / n_rb : MAX_SLICES);
 }
 
 enum : unsigned int {
@@ -99,14 +95,12 @@ struct Params {
   const float* steps;     // [O][G]
   const float* zeros;     // [O][G]
   __nv_bfloat16* Y;       // [M][ldy]
-  float* partial;         // [n_rb][segs][NT][ROWS]
+  float* partial;         // [n_rb][slices][nt][ROWS]
   unsigned int* counter;  // [n_rb], zero at launch and left zero
   int64_t M, O, G, ldy;
   int num_groups;         // K / 128
-  int64_t units;          // n_rb * units_per_rb
-  int units_per_rb;       // ceil(num_groups / 2)
-  int n_ctas;
-  int segs;               // partial-sum slots per row block
+  int g_per;              // groups per slice, even
+  int slices;
   uint32_t idesc;
   DeviceStatus* status;
   uint64_t limit_ns;
@@ -193,17 +187,15 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
   __shared__ __align__(8) uint64_t bars[2 * CS + 2 * XS + 2 * 2 + 2 * AS + 2 * SX_STAGES];
   __shared__ uint32_t tmem_slot;
   __shared__ int failed;
-  __shared__ int last_of_block;
+  __shared__ unsigned int ticket;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // this CTA's units and groups: local group i is group g_of(i) of row block rb_of(i)
-  const int64_t cta = blockIdx.x;
-  const int64_t u0 = cta * p.units / p.n_ctas, u1 = (cta + 1) * p.units / p.n_ctas;
-  const int ng = static_cast<int>(2 * (u1 - u0));
-  auto rb_of = [&](int i) { return static_cast<int>((u0 + i / 2) / p.units_per_rb); };
-  auto g_of = [&](int i) { return static_cast<int>(2 * ((u0 + i / 2) % p.units_per_rb) + (i & 1)); };
-  auto cta_of_unit = [&](int64_t u) { return ((u + 1) * p.n_ctas - 1) / p.units; };
+  const int rb = static_cast<int>(blockIdx.x) / p.slices;
+  const int slice = static_cast<int>(blockIdx.x) - rb * p.slices;
+  const int64_t row0 = static_cast<int64_t>(rb) * ROWS;
+  const int g0 = slice * p.g_per;
+  const int ng = max(0, min(p.g_per, p.num_groups - g0));
 
   const uint32_t bar0 = smem_u32(&bars[0]);
   auto cfull_bar = [&](int c) { return bar0 + 8u * c; };                          // codes landed
@@ -247,7 +239,7 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
       mbar_init(sxempty_bar(t), 4);
     }
     failed = 0;
-    last_of_block = 0;
+    ticket = 0u;
     fence_barrier_init();
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmC);
@@ -261,7 +253,7 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     if (use > 0 && !wait_warp(cempty_bar(c), (use - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
     if (lane == 0) {
       mbar_arrive_expect_tx(cfull_bar(c), C_BYTES);
-      tma_load_2d(c_tile(c), &tmC, g_of(i) * (GK / 8), rb_of(i) * ROWS, cfull_bar(c));
+      tma_load_2d(c_tile(c), &tmC, (g0 + i) * (GK / 8), static_cast<int32_t>(row0), cfull_bar(c));
     }
     __syncwarp();
     return true;
@@ -272,8 +264,8 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     if (use > 0 && !wait_warp(xempty_bar(x), (use - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
     if (lane == 0) {
       mbar_arrive_expect_tx(xfull_bar(x), S::X_BYTES);
-      tma_load_2d(x_tile(x, 0), &tmX, g_of(i) * GK, 0, xfull_bar(x));
-      tma_load_2d(x_tile(x, 1), &tmX, g_of(i) * GK + BK, 0, xfull_bar(x));
+      tma_load_2d(x_tile(x, 0), &tmX, (g0 + i) * GK, 0, xfull_bar(x));
+      tma_load_2d(x_tile(x, 1), &tmX, (g0 + i) * GK + BK, 0, xfull_bar(x));
     }
     __syncwarp();
     return true;
@@ -284,11 +276,8 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
   const int pre_x = min(ng, XS);
   if (warp == 0) {
     __syncwarp();  // the barriers thread 0 initialised are visible to the whole warp
-    // in the order the groups need them: a box, then X' of its two groups
-    for (int i = 0; i < max(pre_c, pre_x); ++i) {
-      if (i < pre_c && i % GROUPS_PER_BOX == 0) load_codes(i);
-      if (i < pre_x) load_x(i);
-    }
+    for (int i = 0; i < pre_c; i += GROUPS_PER_BOX) load_codes(i);
+    for (int i = 0; i < pre_x; ++i) load_x(i);
   }
   if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), S::TMEM_COLS);
   tc_fence_before();
@@ -426,21 +415,19 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     const int q = warp & 3;  // tensor-memory lane quarter this warp may read
     const int r = 32 * q + lane;
     const uint32_t tlane = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-    // step and zero point of local group i for row r (0 for the empty group past an odd group count and
-    // for rows past O, whose results are dropped)
-    auto load_sz = [&](int i, float& st, float& z) {
-      const int64_t o = static_cast<int64_t>(rb_of(i)) * ROWS + r;
-      const int g = g_of(i);
-      const bool real = i < ng && o < p.O && g < p.num_groups;
-      st = real ? __ldg(p.steps + o * p.G + g) : 0.0f;
-      z = real ? __ldg(p.zeros + o * p.G + g) : 0.0f;
-    };
+    const int64_t o_ld = min(row0 + r, p.O - 1);  // rows past O: any valid address (results dropped)
+    const float* st_row = p.steps + o_ld * p.G + g0;
+    const float* z_row = p.zeros + o_ld * p.G + g0;
     float y[NT];
 #pragma unroll
     for (int m = 0; m < NT; ++m) y[m] = 0.0f;
-    float st_n[2], z_n[2];  // two groups ahead
-    load_sz(0, st_n[0], z_n[0]);
-    load_sz(1, st_n[1], z_n[1]);
+    // steps and zero points two groups ahead
+    float st_n[2], z_n[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      st_n[u] = u < ng ? __ldg(st_row + u) : 0.0f;
+      z_n[u] = u < ng ? __ldg(z_row + u) : 0.0f;
+    }
     bool have = true;
     for (int i = 0; i < ng; ++i) {
       const int s = i % AS, t = i % SX_STAGES;
@@ -448,114 +435,105 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
       const float c = __fadd_rn(128.0f, z_n[0]);
       st_n[0] = st_n[1];
       z_n[0] = z_n[1];
-      load_sz(i + 2, st_n[1], z_n[1]);
-      if (have && (!wait_warp(accfull_bar(s), static_cast<uint32_t>(i / AS) & 1u, p, kSiteDecodeAcc) ||
-                   !wait_warp(sxfull_bar(t), static_cast<uint32_t>(i / SX_STAGES) & 1u, p, kSiteDecodeAcc))) {
+      st_n[1] = i + 2 < ng ? __ldg(st_row + i + 2) : 0.0f;
+      z_n[1] = i + 2 < ng ? __ldg(z_row + i + 2) : 0.0f;
+      if (!wait_warp(accfull_bar(s), static_cast<uint32_t>(i / AS) & 1u, p, kSiteDecodeAcc) ||
+          !wait_warp(sxfull_bar(t), static_cast<uint32_t>(i / SX_STAGES) & 1u, p, kSiteDecodeAcc)) {
         have = false;
-        failed = 1;
+        break;
       }
-      if (have) {
-        tc_fence_after();
-        // 16 columns at a time: y[m] += step * (S_g[r, m] - (128 + z) * Sx_g[m])
+      tc_fence_after();
+      // 16 columns at a time: y[m] += step * (S_g[r, m] - (128 + z) * Sx_g[m])
 #pragma unroll
-        for (int cc = 0; cc < NT / 16; ++cc) {
-          float sg[16];
-          tmem_ld16(tlane + static_cast<uint32_t>(s * NT + 16 * cc), sg);
+      for (int cc = 0; cc < NT / 16; ++cc) {
+        float sg[16];
+        tmem_ld16(tlane + static_cast<uint32_t>(s * NT + 16 * cc), sg);
 #pragma unroll
-          for (int k4 = 0; k4 < 16; k4 += 4) {
-            float4 xs;
-            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                         : "=f"(xs.x), "=f"(xs.y), "=f"(xs.z), "=f"(xs.w)
-                         : "r"(sx_slot(t) + 4u * static_cast<uint32_t>(16 * cc + k4))
-                         : "memory");
-            const float xv[4] = {xs.x, xs.y, xs.z, xs.w};
+        for (int k4 = 0; k4 < 16; k4 += 4) {
+          float4 xs;
+          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(xs.x), "=f"(xs.y), "=f"(xs.z), "=f"(xs.w)
+                       : "r"(sx_slot(t) + 4u * static_cast<uint32_t>(16 * cc + k4))
+                       : "memory");
+          const float xv[4] = {xs.x, xs.y, xs.z, xs.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int m = 16 * cc + k4 + k;
-              y[m] = __fmaf_rn(step, __fmaf_rn(-c, xv[k], sg[k4 + k]), y[m]);
-            }
+          for (int k = 0; k < 4; ++k) {
+            const int m = 16 * cc + k4 + k;
+            y[m] = __fmaf_rn(step, __fmaf_rn(-c, xv[k], sg[k4 + k]), y[m]);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(accempty_bar(s));
-          mbar_arrive(sxempty_bar(t));
-        }
       }
-      // End of this CTA's run in row block rb: write Y, or this CTA's partial sums and a ticket; the
-      // last CTA of the block adds the partials in CTA order. Every CTA takes its ticket, even after a
-      // timeout, so the counters go back to zero.
-      const int rb = rb_of(i);
-      if (i + 1 < ng && rb_of(i + 1) == rb) continue;
-      const int64_t ub = static_cast<int64_t>(rb) * p.units_per_rb;
-      const int64_t c_first = cta_of_unit(ub);
-      const int nseg = static_cast<int>(cta_of_unit(ub + p.units_per_rb - 1) - c_first + 1);
-      const int64_t row0 = static_cast<int64_t>(rb) * ROWS;
-      if (nseg == 1) {
-        const int64_t o = row0 + r;
-#pragma unroll
-        for (int m = 0; m < NT; ++m)
-          if (m < p.M && o < p.O) p.Y[m * p.ldy + o] = __float2bfloat16_rn(have ? y[m] : 0.0f);
-      } else {
-        float* blk = p.partial + static_cast<int64_t>(rb) * p.segs * NT * ROWS;
-        float* mine = blk + static_cast<int64_t>(cta - c_first) * NT * ROWS + r;
-#pragma unroll
-        for (int m = 0; m < NT; ++m) __stcg(mine + m * ROWS, have ? y[m] : 0.0f);
-        __threadfence();
-        epilogue_sync();
-        if (warp == EPI_WARP0 && lane == 0) {
-          const unsigned int ticket = atomicAdd(p.counter + rb, 1u);
-          const int last = ticket == static_cast<unsigned int>(nseg - 1);
-          if (last) p.counter[rb] = 0u;
-          last_of_block = last;
-        }
-        epilogue_sync();
-        if (last_of_block) {
-          __threadfence();
-          // the four epilogue warps: four rows per item, eight partials in flight per thread
-          const int items = static_cast<int>(p.M) * (ROWS / 4);
-          for (int it = r; it < items; it += 128) {
-            const int tk = it / (ROWS / 4);
-            const int r4 = (it - tk * (ROWS / 4)) * 4;
-            if (row0 + r4 >= p.O) continue;  // O % 8 == 0: four rows are all in or all out
-            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 1
-            for (int c0 = 0; c0 < nseg; c0 += 8) {
-              float4 v[8];
-#pragma unroll
-              for (int k = 0; k < 8; ++k)
-                v[k] = c0 + k < nseg
-                           ? __ldcg(reinterpret_cast<const float4*>(blk + (static_cast<int64_t>(c0 + k) * NT + tk) * ROWS + r4))
-                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                if (c0 + k >= nseg) continue;
-                if (c0 + k == 0) {
-                  acc = v[0];  // CTA order: ((p0 + p1) + p2) + ...
-                } else {
-                  acc.x = __fadd_rn(acc.x, v[k].x);
-                  acc.y = __fadd_rn(acc.y, v[k].y);
-                  acc.z = __fadd_rn(acc.z, v[k].z);
-                  acc.w = __fadd_rn(acc.w, v[k].w);
-                }
-              }
-            }
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-            *reinterpret_cast<uint2*>(p.Y + tk * p.ldy + row0 + r4) =
-                make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
-          }
-        }
-        epilogue_sync();  // last_of_block is rewritten for the next row block
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(accempty_bar(s));
+        mbar_arrive(sxempty_bar(t));
       }
+    }
+    if (!have) failed = 1;
+    if (p.slices == 1) {
+      // One slice: the sums are the result; lane r writes row r of every token (coalesced per token).
+      const int64_t o = row0 + r;
 #pragma unroll
-      for (int m = 0; m < NT; ++m) y[m] = 0.0f;
+      for (int m = 0; m < NT; ++m)
+        if (m < p.M && o < p.O) p.Y[m * p.ldy + o] = __float2bfloat16_rn(have ? y[m] : 0.0f);
+    } else {
+      // Slice `slice` of the row block's partial sums, then a ticket.
+      float* mine = p.partial + (static_cast<int64_t>(rb) * p.slices + slice) * NT * ROWS + r;
+#pragma unroll
+      for (int m = 0; m < NT; ++m) __stcg(mine + m * ROWS, have ? y[m] : 0.0f);
+      __threadfence();
+      epilogue_sync();
+      if (warp == EPI_WARP0 && lane == 0) {
+        // Every CTA takes a ticket, even after a timeout, and the last one hands the counter back at
+        // zero, so the next call needs no clearing.
+        ticket = atomicAdd(p.counter + rb, 1u);
+        if (ticket == static_cast<unsigned int>(p.slices - 1)) p.counter[rb] = 0u;
+      }
     }
   }
 
   __syncwarp();
   __syncthreads();
+  if (p.slices > 1 && ticket == static_cast<unsigned int>(p.slices - 1)) {
+    // Last slice of this row block: every other slice's sums are visible (each CTA fenced before taking
+    // its ticket). The whole CTA adds them in slice order, four rows per item.
+    __threadfence();
+    const float* blk = p.partial + static_cast<int64_t>(rb) * p.slices * NT * ROWS;
+    const int items = static_cast<int>(p.M) * (ROWS / 4);
+    // One item per thread per pass and eight slices per round, so eight loads are in flight at once.
+    for (int it = static_cast<int>(threadIdx.x); it < items; it += THREADS) {
+      const int t = it / (ROWS / 4);
+      const int r4 = (it - t * (ROWS / 4)) * 4;
+      if (row0 + r4 >= p.O) continue;  // O % 8 == 0: four rows are all in or all out
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 1
+      for (int c0 = 0; c0 < p.slices; c0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          v[c] = c0 + c < p.slices
+                     ? __ldcg(reinterpret_cast<const float4*>(blk + (static_cast<int64_t>(c0 + c) * NT + t) * ROWS + r4))
+                     : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (c0 + c >= p.slices) continue;
+          if (c0 + c == 0) {
+            acc = v[0];  // slice order: ((s0 + s1) + s2) + ...
+          } else {
+            acc.x = __fadd_rn(acc.x, v[c].x);
+            acc.y = __fadd_rn(acc.y, v[c].y);
+            acc.z = __fadd_rn(acc.z, v[c].z);
+            acc.w = __fadd_rn(acc.w, v[c].w);
+          }
+        }
+      }
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+      *reinterpret_cast<uint2*>(p.Y + t * p.ldy + row0 + r4) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+    }
+  }
   if (failed) {  // let copies still in flight land before the shared memory is given up
     const uint64_t t0 = global_timer_ns();
     while (global_timer_ns() - t0 < 50000ull) __nanosleep(1000);
