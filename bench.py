@@ -478,8 +478,9 @@ def measure_int8_pack(Wd, scales):
 
 def measure_w4a16(Xd, Wd, scales):
     """The deployment GEMM on the quantized layer, and a dense bf16 GEMM (torch.matmul) of the same shapes
-    on the same harness as a comparator (measurement only): a prefill of all N calibration tokens, a
-    16-token decode on the whole layer, and a 16-token decode on its first 4096 rows and in-features.
+    on the same harness as a comparator (measurement only): a prefill of all N calibration tokens and a
+    16-token decode on the whole layer, and a 4096-token prefill and a 16-token decode on its first 4096
+    rows and in-features.
     Each is timed cold: a batch of launches, each after a 512 MiB L2 flush, between two events, minus a
     batch of flushes alone timed just before (single launches of a few microseconds would be read off an
     event clock that ticks in ~2 us steps); the median over seven such pairs. Batches hold 40 launches,
@@ -524,7 +525,8 @@ def measure_w4a16(Xd, Wd, scales):
         Xs = awq.scale_columns(X, s, divide=True)
         ws = torch.zeros(lib.awq_w4a16_workspace_size(X.shape[1], codes.shape[0]), dtype=torch.uint8,
                          device=X.device)
-        cases = (("decode", Xs[:16].contiguous()),) if prefix else (("prefill", Xs), ("decode", Xs[:16].contiguous()))
+        cases = (("prefill", Xs[:4096].contiguous()), ("decode", Xs[:16].contiguous())) if prefix else \
+            (("prefill", Xs), ("decode", Xs[:16].contiguous()))
         for name, A in cases:
             Y = torch.empty((A.shape[0], codes.shape[0]), dtype=torch.bfloat16, device=X.device)
             fn = lambda A=A, Y=Y: awq.w4a16_gemm(A, codes, steps, zeros, out=Y, workspace=ws)
@@ -539,10 +541,15 @@ def w4a16_summary(w4, peaks):
     """Rates of the W4A16 launches: prefill in TFLOP/s, decodes in HBM GB/s of their algorithmic bytes
     (codes O*K/2, steps and zeros 8*O*K/128, X' 2*M*K, Y 2*M*O), each beside the bf16 comparator."""
     out = {"comparator": "torch.matmul bf16 on the same shapes and harness (measurement only)"}
-    M, K, O = w4["prefill_shape"]
-    out.update({"prefill_shape_MKO": [M, K, O], "prefill_ms": w4["prefill_ms"], "prefill_bf16_ms": w4["prefill_bf16_ms"],
-                "prefill_tflops": 2.0 * M * O * K / (w4["prefill_ms"] / 1e3) / 1e12})
-    out["prefill_frac_of_peak"] = out["prefill_tflops"] / peaks["bf16_tflops"]
+    for prefix in ("", "small_"):
+        if f"{prefix}prefill_ms" not in w4:
+            continue
+        M, K, O = w4[f"{prefix}prefill_shape"]
+        ms = w4[f"{prefix}prefill_ms"]
+        tf = 2.0 * M * O * K / (ms / 1e3) / 1e12
+        out.update({f"{prefix}prefill_shape_MKO": [M, K, O], f"{prefix}prefill_ms": ms,
+                    f"{prefix}prefill_bf16_ms": w4[f"{prefix}prefill_bf16_ms"], f"{prefix}prefill_tflops": tf,
+                    f"{prefix}prefill_frac_of_peak": tf / peaks["bf16_tflops"]})
     for prefix in ("", "small_"):
         if f"{prefix}decode_ms" not in w4:
             continue

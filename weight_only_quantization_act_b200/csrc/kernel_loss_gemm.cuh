@@ -189,8 +189,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       int ready = -1;  // candidates <= ready are known to be fully produced
-      const uint64_t pol_x = p.keep_x ? policy_evict_last() : policy_evict_normal();
-      const uint64_t pol_d = policy_evict_normal();
+      // X fits L2: keep it (every band group re-reads it). Else the band group's dW rows are what the
+      // tiles in flight re-read, and an X tile is used by the group's few bands right away: keep the dW,
+      // let X go first.
+      const uint64_t pol_x = p.keep_x ? policy_evict_last() : policy_evict_first();
+      const uint64_t pol_d = p.keep_x ? policy_evict_normal() : policy_evict_last();
       for (int i = 0; ok; ++i) {
         int t;
         if (rank == 0) {

@@ -40,6 +40,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "numerics.cuh"
 #include "ptx.cuh"
 
 namespace awq {
@@ -276,8 +277,11 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
   const int pre_x = min(ng, XS);
   if (warp == 0) {
     __syncwarp();  // the barriers thread 0 initialised are visible to the whole warp
-    for (int i = 0; i < pre_c; i += GROUPS_PER_BOX) load_codes(i);
-    for (int i = 0; i < pre_x; ++i) load_x(i);
+    // in the order the groups need them: a box, then X' of its two groups
+    for (int i = 0; i < max(pre_c, pre_x); ++i) {
+      if (i < pre_c && i % GROUPS_PER_BOX == 0) load_codes(i);
+      if (i < pre_x) load_x(i);
+    }
   }
   if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), S::TMEM_COLS);
   tc_fence_before();
@@ -455,11 +459,13 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
                        : "=f"(xs.x), "=f"(xs.y), "=f"(xs.z), "=f"(xs.w)
                        : "r"(sx_slot(t) + 4u * static_cast<uint32_t>(16 * cc + k4))
                        : "memory");
-          const float xv[4] = {xs.x, xs.y, xs.z, xs.w};
+          // paired fp32: t = S - c * Sx, y = y + step * t, two tokens per instruction
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < 4; k += 2) {
             const int m = 16 * cc + k4 + k;
-            y[m] = __fmaf_rn(step, __fmaf_rn(-c, xv[k], sg[k4 + k]), y[m]);
+            const uint64_t t = fx2_fma(fx2(-c, -c), fx2(k == 0 ? xs.x : xs.z, k == 0 ? xs.y : xs.w),
+                                       fx2(sg[k4 + k], sg[k4 + k + 1]));
+            fx2_split(fx2_fma(fx2(step, step), t, fx2(y[m], y[m + 1])), y[m], y[m + 1]);
           }
         }
       }
