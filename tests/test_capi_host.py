@@ -172,7 +172,7 @@ def test_next_row_entry_points_reject_bad_arguments(lib):
 
 def test_w4a16_workspace_covers_its_regions(lib):
     # header (512 B) + the fixed few-token counter region (65536 x 4 B) + group-major steps and zeros
-    # (K/128 x O rounded up to 256, fp32, each) + split-K partial sums
+    # (K/128 x O rounded up to 256, fp32, each) + the few-token X' copy and group sums + split-K partials
     fixed = 512 + 65536 * 4
     for K, O in [(128, 8), (256, 256), (4096, 4096), (14336, 4096), (28672, 8192), (4096, 28672)]:
         ws = lib.awq_w4a16_workspace_size(K, O)

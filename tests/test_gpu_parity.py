@@ -38,6 +38,22 @@ def test_act_stats_strided_input():
     assert_bits_equal(awq.act_stats(Xd), orc.act_mean(wide[:, 128:384]), "strided")
 
 
+@pytest.mark.parametrize("shape", [(600, 1030), (37, 2), (513, 2056), (256, 1024)])
+def test_act_stats_special_magnitudes(shape):
+    """Zeros, subnormals and magnitudes across the whole finite bf16 exponent range, both signs, with a
+    ragged last column block (K % 8 != 0) and row counts off the 8-row load blocks."""
+    rng = np.random.default_rng(shape[0] + 31 * shape[1])
+    e = np.where(rng.random(shape) < 0.5, rng.integers(0, 255, shape), rng.integers(0, 4, shape))
+    bits = (rng.integers(0, 2, shape) << 15) | (e << 7) | rng.integers(0, 128, shape)
+    bits[rng.random(shape) < 0.1] = 0
+    X = bits.astype(np.uint16)
+    ld = -(-shape[1] // 8) * 8                     # row stride: the next multiple of 8
+    wide = np.zeros((shape[0], ld), np.uint16)
+    wide[:, :shape[1]] = X
+    Xd = bf16_to_device(wide)[:, :shape[1]]
+    assert_bits_equal(awq.act_stats(Xd), orc.act_mean(X), f"special magnitudes {shape}")
+
+
 def test_act_stats_tiny_workload():
     X, _, _ = inputs.make_inputs(inputs.workload(1))
     assert_bits_equal(awq.act_stats(bf16_to_device(X)), orc.act_mean(X), "workload 1")

@@ -187,9 +187,11 @@ def test_w4a16_repeated_runs_are_bit_identical(M, K, O):
 
 def test_w4a16_shared_workspace_across_calls_and_shapes():
     """One workspace, zero-filled once, serves every later call: the few-token kernel's per-block
-    counters are handed back at zero by each call, whatever the shape (different slice counts)."""
+    counters are handed back at zero by each call, whatever the shape (different slice counts), and
+    many-token calls with more tiles than CTA pairs (2048 x 5120 outputs: 80 tiles) share it."""
     lib = awq.load_library()
-    shapes = [(16, 4096, 1024), (5, 384, 600), (64, 2048, 1024), (16, 4096, 1024), (300, 512, 256), (1, 256, 136)]
+    shapes = [(16, 4096, 1024), (5, 384, 600), (2048, 512, 5120), (64, 2048, 1024), (16, 4096, 1024),
+              (2048, 512, 5120), (300, 512, 256), (1, 256, 136)]
     ws = torch.zeros(max(lib.awq_w4a16_workspace_size(K, O) for _, K, O in shapes), dtype=torch.uint8,
                      device="cuda")
     for n, (M, K, O) in enumerate(shapes):

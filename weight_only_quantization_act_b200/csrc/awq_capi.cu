@@ -114,8 +114,6 @@ awq_status device_info(DeviceInfo** out) {
   if (!d.gemm_attr_set) {
     AWQ_CUDA(cudaFuncSetAttribute(awq::lg::loss_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   awq::lg::SMEM_BYTES));
-    AWQ_CUDA(cudaFuncSetAttribute(awq::act_chunk_sums_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  awq::kActSmemBytes));
     AWQ_CUDA(cudaFuncSetAttribute(awq::quantize_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   awq::kPackSmemBytes));
     cudaLaunchConfig_t cfg = {};
@@ -298,7 +296,7 @@ awq_status check_matrix(const char* name, const void* p, int64_t rows, int64_t K
   return AWQ_OK;
 }
 
-// The chunk-sum kernel runs one grid row per 256-row chunk; a grid's y extent is at most 65535.
+// The interface bounds the statistic's rows by 65535 chunks of 256 (N <= 16,776,960).
 awq_status check_act_chunks(const char* name, int64_t rows) {
   const int64_t n_chunks = (rows + awq::kActChunk - 1) / awq::kActChunk;
   if (n_chunks > 65535)
@@ -311,6 +309,27 @@ awq_status check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(AWQ_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
   return AWQ_OK;
+}
+
+// Column sums of |A| (rows x K, stride ld) in the statistic's fixed order, then their means: the chunk-sum
+// kernel over (chunk, 512-column block) work items, as many CTAs as make every CTA take the same number of
+// items within kActCtasPerSm resident CTAs per SM, then the finaliser over the fp64 partial array part.
+awq_status launch_act_stats(const void* A, int64_t rows, int64_t K, int64_t ld, double* part, float* mean, int sms,
+                            cudaStream_t st) {
+  const int64_t n_chunks = (rows + awq::kActChunk - 1) / awq::kActChunk;
+  const int64_t items = n_chunks * ((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock);
+  const int64_t resident = static_cast<int64_t>(sms) * awq::kActCtasPerSm;
+  const int64_t per_cta = (items + resident - 1) / resident;
+  const int64_t ctas = (items + per_cta - 1) / per_cta;
+  awq::act_chunk_sums_kernel<<<static_cast<unsigned>(ctas), awq::kActThreads, 0, st>>>(
+      static_cast<const uint16_t*>(A), rows, K, ld, part);
+  {
+    awq_status s = check_launch("act_chunk_sums_kernel");
+    if (s != AWQ_OK) return s;
+  }
+  awq::act_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(part, rows, K,
+                                                                                   static_cast<int>(n_chunks), mean);
+  return check_launch("act_finalize_kernel");
 }
 
 #define AWQ_TRY(x)                      \
@@ -381,12 +400,7 @@ awq_status awq_act_stats(const void* X, int64_t N, int64_t K, int64_t ldx, void*
   AWQ_TRY(device_info(&d));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   double* part = static_cast<double*>(workspace);
-  dim3 grid(static_cast<unsigned>((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock), l.n_chunks);
-  awq::act_chunk_sums_kernel<<<grid, awq::kActThreads, awq::kActSmemBytes, st>>>(static_cast<const uint16_t*>(X), N, K,
-                                                                                 ldx, part);
-  AWQ_TRY(check_launch("act_chunk_sums_kernel"));
-  awq::act_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(part, N, K, l.n_chunks, act_mean);
-  AWQ_TRY(check_launch("act_finalize_kernel"));
+  AWQ_TRY(launch_act_stats(X, N, K, ldx, part, act_mean, d->sms, st));
   return ok();
 }
 
@@ -494,14 +508,8 @@ awq_status awq_search_ex(const void* X, int64_t N, int64_t K, int64_t ldx, const
   float* wmean = reinterpret_cast<float*>(ws + l.wmean_off);
   if (mode == awq::kScalesWeightAware) {
     // mean |W| per column: the activation statistic's fixed-order kernels run on W
-    const ActLayout wl = act_layout(O, K);
     double* wpart = reinterpret_cast<double*>(ws + l.wpart_off);
-    dim3 wgrid(static_cast<unsigned>((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock), wl.n_chunks);
-    awq::act_chunk_sums_kernel<<<wgrid, awq::kActThreads, awq::kActSmemBytes, st>>>(static_cast<const uint16_t*>(W), O,
-                                                                                     K, ldw, wpart);
-    AWQ_TRY(check_launch("act_chunk_sums_kernel"));
-    awq::act_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(wpart, O, K, wl.n_chunks, wmean);
-    AWQ_TRY(check_launch("act_finalize_kernel"));
+    AWQ_TRY(launch_act_stats(W, O, K, ldw, wpart, wmean, d->sms, st));
   }
   AWQ_TRY(launch_scale_table(act_mean, wmean, K, n_grid, mode, (flags & AWQ_FLAG_EXACT_POW) != 0, table, rtable, spart,
                              st));
@@ -605,11 +613,14 @@ awq_status awq_quantize_pack_ex(const void* W, int64_t O, int64_t K, int64_t ldw
   if (flags & ~AWQ_FLAG_EXACT_DIVISION) return fail(AWQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   DeviceInfo* d = nullptr;
   AWQ_TRY(device_info(&d));
-  // one resident wave of warps; each warp then walks rows of its segment
+  // One resident wave of CTAs, each on one segment (1024 in-features) and 8 rows at a time: as many CTAs
+  // per segment as fit, with every segment given the same number (fewer CTAs than segments: each CTA
+  // walks several segments).
   const int64_t segs = (K + awq::kPackWarpCols - 1) / awq::kPackWarpCols;
-  const int64_t items = O * segs;
-  const int64_t max_blocks = static_cast<int64_t>(d->sms) * 2;  // 2 blocks of 256 threads fit per SM
-  const int64_t blocks = std::min<int64_t>(max_blocks, (items * 32 + awq::kPackThreads - 1) / awq::kPackThreads);
+  const int64_t row_octets = (O + awq::kPackThreads / 32 - 1) / (awq::kPackThreads / 32);
+  const int64_t max_blocks = static_cast<int64_t>(d->sms) * awq::kPackCtasPerSm;
+  int64_t blocks = std::min<int64_t>(max_blocks, row_octets * segs);
+  if (blocks > segs) blocks = blocks / segs * segs;
   awq::quantize_pack_kernel<<<static_cast<unsigned>(blocks), awq::kPackThreads, awq::kPackSmemBytes,
                               reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint16_t*>(W), O, K, ldw, scales, (flags & AWQ_FLAG_EXACT_DIVISION) ? 1 : 0, codes, steps,
@@ -728,12 +739,7 @@ extern "C" awq_status awq_act_stats_noalloc(const void* X, int64_t N, int64_t K,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // Each (chunk, column) entry the finaliser reads is written first by this call, so the scratch needs
   // no clearing; what the previous call left there is simply overwritten.
-  dim3 grid(static_cast<unsigned>((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock), l.n_chunks);
-  awq::act_chunk_sums_kernel<<<grid, awq::kActThreads, awq::kActSmemBytes, st>>>(static_cast<const uint16_t*>(X), N, K,
-                                                                                 ldx, part);
-  AWQ_TRY(check_launch("act_chunk_sums_kernel"));
-  awq::act_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(part, N, K, l.n_chunks, act_mean);
-  AWQ_TRY(check_launch("act_finalize_kernel"));
+  AWQ_TRY(launch_act_stats(X, N, K, ldx, part, act_mean, d->sms, st));
   return ok();
 }
 
@@ -775,13 +781,14 @@ extern "C" awq_status awq_scale_rows(const void* A, int64_t R, int64_t C, int64_
 namespace {
 struct W4Layout {
   int64_t O_pad, G, n_rb;
-  size_t steps_off, zeros_off, counter_off, partial_off, bytes;
+  size_t steps_off, zeros_off, counter_off, xp_off, sx_off, partial_off, bytes;
 };
 constexpr int64_t kW4MaxRowBlocks = 65536;  // few-token counters reserved for O up to 8M rows
 // [0, 512) status word and tile counter (cleared by each many-token call); [512, 512 + 256 KB) the
 // few-token kernel's per-row-block counters, at the same place for every shape and written by nothing
 // else, so they stay zero from one call to the next whatever the shapes; then the group-major steps and
-// zeros (many tokens) and the split-K partial sums (few tokens).
+// zeros (many tokens), and the few-token kernel's permuted copy of X' (64 rows), group sums and split-K
+// partial sums.
 W4Layout w4_layout(int64_t K, int64_t O) {
   W4Layout l;
   l.O_pad = (O + awq::lg::BN - 1) / awq::lg::BN * awq::lg::BN;
@@ -790,7 +797,9 @@ W4Layout w4_layout(int64_t K, int64_t O) {
   l.counter_off = 512;
   l.steps_off = l.counter_off + static_cast<size_t>(kW4MaxRowBlocks) * 4;
   l.zeros_off = align_up(l.steps_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
-  l.partial_off = align_up(l.zeros_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
+  l.xp_off = align_up(l.zeros_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
+  l.sx_off = align_up(l.xp_off + static_cast<size_t>(awq::dec::MAX_NT) * K * 2, 256);
+  l.partial_off = align_up(l.sx_off + static_cast<size_t>(l.G) * awq::dec::MAX_NT * 4, 256);
   const int64_t rb = std::min(l.n_rb, kW4MaxRowBlocks);
   l.bytes = align_up(l.partial_off + static_cast<size_t>(rb) * awq::dec::max_slices(rb) * awq::dec::MAX_NT *
                                          awq::dec::ROWS * 4,
@@ -814,17 +823,23 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   const int g_per = static_cast<int>(((num_groups + slices - 1) / slices + 1) / 2 * 2);
   slices = (num_groups + g_per - 1) / g_per;
   if (l.n_rb * slices >= (1ll << 31)) return fail(AWQ_ERR_INVALID_ARG, "O is too large");
-  CUtensorMap tmX, tmC;
-  AWQ_TRY(make_tmap(&tmX, X, M, K, ldx, nt));
-  AWQ_TRY(make_tmap_codes_sw128(&tmC, codes, O, K / 8, awq::dec::ROWS));
   char* ws = static_cast<char*>(workspace);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint16_t* xp = reinterpret_cast<uint16_t*>(ws + l.xp_off);
+  float* sx = reinterpret_cast<float*>(ws + l.sx_off);
+  CUtensorMap tmX, tmC;
+  AWQ_TRY(make_tmap(&tmX, xp, nt, K, K, nt));
+  AWQ_TRY(make_tmap_codes_sw128(&tmC, codes, O, K / 8, awq::dec::ROWS));
+  awq::dec::decode_prep_kernel<<<static_cast<unsigned>(num_groups), awq::dec::PREP_THREADS, 0, st>>>(
+      static_cast<const uint16_t*>(X), M, K, ldx, nt, xp, sx);
+  AWQ_TRY(check_launch("decode_prep_kernel"));
   awq::dec::Params p;
   p.steps = steps;
   p.zeros = zeros;
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.partial = reinterpret_cast<float*>(ws + l.partial_off);
   p.counter = reinterpret_cast<unsigned int*>(ws + l.counter_off);
+  p.sx = sx;
   p.M = M;
   p.O = O;
   p.G = l.G;
@@ -835,15 +850,29 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   p.idesc = awq::idesc_bf16_f32(awq::dec::ROWS, static_cast<uint32_t>(nt));
   p.status = reinterpret_cast<awq::DeviceStatus*>(ws);
   p.limit_ns = g_wait_limit_ns.load();
-  const dim3 grid(static_cast<unsigned>(l.n_rb * slices));
-  if (nt == 16)
-    awq::dec::w4a16_decode_kernel<16><<<grid, awq::dec::THREADS, awq::dec::Shape<16>::SMEM, st>>>(tmX, tmC, p);
-  else if (nt == 32)
-    awq::dec::w4a16_decode_kernel<32><<<grid, awq::dec::THREADS, awq::dec::Shape<32>::SMEM, st>>>(tmX, tmC, p);
-  else if (nt == 48)
-    awq::dec::w4a16_decode_kernel<48><<<grid, awq::dec::THREADS, awq::dec::Shape<48>::SMEM, st>>>(tmX, tmC, p);
-  else
-    awq::dec::w4a16_decode_kernel<64><<<grid, awq::dec::THREADS, awq::dec::Shape<64>::SMEM, st>>>(tmX, tmC, p);
+  // launched as a programmatic dependent of the prep kernel: its prologue and first code loads overlap it
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(l.n_rb * slices));
+  cfg.blockDim = dim3(awq::dec::THREADS);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (nt == 16) {
+    cfg.dynamicSmemBytes = awq::dec::Shape<16>::SMEM;
+    AWQ_CUDA(cudaLaunchKernelEx(&cfg, awq::dec::w4a16_decode_kernel<16>, tmX, tmC, p));
+  } else if (nt == 32) {
+    cfg.dynamicSmemBytes = awq::dec::Shape<32>::SMEM;
+    AWQ_CUDA(cudaLaunchKernelEx(&cfg, awq::dec::w4a16_decode_kernel<32>, tmX, tmC, p));
+  } else if (nt == 48) {
+    cfg.dynamicSmemBytes = awq::dec::Shape<48>::SMEM;
+    AWQ_CUDA(cudaLaunchKernelEx(&cfg, awq::dec::w4a16_decode_kernel<48>, tmX, tmC, p));
+  } else {
+    cfg.dynamicSmemBytes = awq::dec::Shape<64>::SMEM;
+    AWQ_CUDA(cudaLaunchKernelEx(&cfg, awq::dec::w4a16_decode_kernel<64>, tmX, tmC, p));
+  }
   AWQ_TRY(check_launch("w4a16_decode_kernel"));
   return ok();
 }

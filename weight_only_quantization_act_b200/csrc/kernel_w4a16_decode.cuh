@@ -18,17 +18,20 @@
 // Nibble order. A code word holds in-features 8c .. 8c+7 in nibbles 0..7. One AND-OR per register turns
 // the word shifted right by 4j into the bf16 pair (128 + q_j, 128 + q_{j+4}), so the operand row holds
 // each word's in-features in the order 0 4 1 5 2 6 3 7. X' is permuted the same way inside every 16-byte
-// chunk (8 in-features) by the warps that sum Sx_g from it, which leaves the products and sums unchanged.
+// chunk (8 in-features), which leaves the products and sums unchanged. A small kernel before this one
+// writes that permuted copy of X' (nt rows, zero past M) and every Sx_g once, instead of every CTA
+// redoing them; it lets this kernel start early (programmatic dependent launch), and only the loader
+// waits for it, after requesting its first code boxes.
 //
 // CTA (b, c) covers weight rows [128 b, 128 b + 128) and groups [c * gp, (c + 1) * gp) (gp even). The
 // unpacked operand of a group (128 rows x 128 in-features) lives in tensor memory (tcgen05.mma reads A
-// from there), two groups at a time, next to the accumulators. Warps:
-//   0      loads: one TMA box of code words per two groups [128 rows x 32 words] (128-byte swizzle)
-//          and X' per group as two [nt x 64] boxes (128-byte swizzle), each into a ring of its own
+// from there), three groups at a time, next to the accumulators. Warps:
+//   0      loads: one TMA box of code words per two groups [128 rows x 32 words] (128-byte swizzle),
+//          X' per group as two [nt x 64] boxes (128-byte swizzle) and Sx_g (one bulk copy), each into a
+//          ring of its own
 //   1      tensor memory; one thread issues the 8 MMAs of a group (M = 128, N = nt, K = 16)
 //   2-9    unpack: warps 2-5 take the even groups, warps 6-9 the odd ones; lane l of warp w unpacks row
-//          32 (w % 4) + l (the tensor-memory lanes warp w may write) with two 32-column stores; the four
-//          warps of the set also sum Sx_g from the group's X' tile and permute it in place
+//          32 (w % 4) + l (the tensor-memory lanes warp w may write) with two 32-column stores
 //   10-13  per group: S_g of their lane quarter, minus the zero-point term, times step, added to per-row
 //          registers (steps and zero points read from global memory two groups ahead); at the end Y, or
 //          this slice's partial sums
@@ -58,7 +61,8 @@ constexpr int UNPACK_WARPS = 8;
 constexpr int EPI_WARP0 = 2 + UNPACK_WARPS;   // warps 10-13
 constexpr int THREADS = 32 * (EPI_WARP0 + 4);  // 448
 constexpr int MAX_SLICES = 16;
-constexpr int SX_STAGES = 4;                  // Sx_g of the groups in flight between unpack and epilogue
+constexpr int SX_STAGES = 8;                  // Sx_g of the groups in flight between loader and epilogue
+constexpr int SZ_AHEAD = 4;                   // groups of steps and zero points an epilogue thread has in flight
 
 template <int NT>
 struct Shape {
@@ -67,8 +71,9 @@ struct Shape {
   static constexpr int X_BYTES = 2 * NT * 128;                          // one group: two [NT x 64] tiles
   static constexpr int X_STAGES = NT <= 16 ? 8 : (96 * 1024) / X_BYTES; // X' groups in flight
   static constexpr int ACC_STAGES = 4;                                  // group accumulators S_g
-  static constexpr int A_COL0 = ACC_STAGES * NT;                        // two groups' operands
-  static constexpr int USED_COLS = A_COL0 + 2 * A_COLS;
+  static constexpr int A_BUFS = 3;                                      // group operands in flight
+  static constexpr int A_COL0 = ACC_STAGES * NT;
+  static constexpr int USED_COLS = A_COL0 + A_BUFS * A_COLS;
   static constexpr uint32_t TMEM_COLS = USED_COLS <= 128 ? 128 : (USED_COLS <= 256 ? 256 : 512);
   static constexpr int TPT = NT == 16 ? 8 : (NT == 32 ? 4 : 2);         // Sx threads per token
   static constexpr int SMEM = C_STAGES * C_BYTES + X_STAGES * X_BYTES + SX_STAGES * NT * 4 + 1024;
@@ -98,6 +103,7 @@ struct Params {
   __nv_bfloat16* Y;       // [M][ldy]
   float* partial;         // [n_rb][slices][nt][ROWS]
   unsigned int* counter;  // [n_rb], zero at launch and left zero
+  const float* sx;        // [G][nt] group sums of X' (decode_prep_kernel)
   int64_t M, O, G, ldy;
   int num_groups;         // K / 128
   int g_per;              // groups per slice, even
@@ -178,14 +184,50 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&v)[4]) {
   v[3] = nibble_pair_bf16(shr_fma(w, 1u << 20));
 }
 
+// X' for the few-token kernel: Xp[m][k] = X[m][k] for m < M, zero for M <= m < nt, with each 16-byte chunk
+// of 8 in-features in the operand order 0 4 1 5 2 6 3 7; Sx[g][m] = sum of X[m][k] over the group's 128
+// in-features in increasing k (fp32, zero past M). One CTA per group.
+constexpr int PREP_THREADS = 128;
+__global__ void __launch_bounds__(PREP_THREADS) decode_prep_kernel(const uint16_t* __restrict__ X, int64_t M,
+                                                                   int64_t K, int64_t ldx, int nt,
+                                                                   uint16_t* __restrict__ Xp, float* __restrict__ Sx) {
+  pdl_launch_dependents();
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * GK;
+  for (int task = threadIdx.x; task < nt * (GK / 8); task += PREP_THREADS) {
+    const int m = task / (GK / 8), ch = task % (GK / 8);
+    const uint4 v = m < M ? *reinterpret_cast<const uint4*>(X + m * ldx + k0 + 8 * ch) : make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(Xp + static_cast<int64_t>(m) * K + k0 + 8 * ch) =
+        make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632), __byte_perm(v.y, v.w, 0x5410),
+                   __byte_perm(v.y, v.w, 0x7632));
+  }
+  if (threadIdx.x < nt) {
+    const int m = threadIdx.x;
+    float sum = 0.0f;
+    if (m < M) {
+      const uint4* row = reinterpret_cast<const uint4*>(X + m * ldx + k0);
+#pragma unroll 4
+      for (int ch = 0; ch < GK / 8; ++ch) {
+        const uint4 v = row[ch];
+        const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          sum = __fadd_rn(__fadd_rn(sum, __uint_as_float(e[k] << 16)), __uint_as_float(e[k] & 0xFFFF0000u));
+      }
+    }
+    Sx[static_cast<int64_t>(blockIdx.x) * nt + m] = sum;
+  }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     w4a16_decode_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC, Params p) {
+  // tmX covers the permuted copy Xp [nt][K]; p.sx holds Sx [G][nt] (both from decode_prep_kernel)
   using S = Shape<NT>;
   constexpr int CS = S::C_STAGES, XS = S::X_STAGES, AS = S::ACC_STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[2 * CS + 2 * XS + 2 * 2 + 2 * AS + 2 * SX_STAGES];
+  constexpr int AB = S::A_BUFS;
+  __shared__ __align__(8) uint64_t bars[2 * CS + 2 * XS + 2 * AB + 2 * AS + 2 * SX_STAGES];
   __shared__ uint32_t tmem_slot;
   __shared__ int failed;
   __shared__ unsigned int ticket;
@@ -204,11 +246,11 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
   auto xfull_bar = [&](int x) { return bar0 + 8u * (2 * CS + x); };               // X' landed
   auto xempty_bar = [&](int x) { return bar0 + 8u * (2 * CS + XS + x); };         // MMAs done with X'
   auto dq_bar = [&](int a) { return bar0 + 8u * (2 * CS + 2 * XS + a); };         // operand a written
-  auto afree_bar = [&](int a) { return bar0 + 8u * (2 * CS + 2 * XS + 2 + a); };  // MMAs done with it
-  auto accfull_bar = [&](int s) { return bar0 + 8u * (2 * CS + 2 * XS + 4 + s); };
-  auto accempty_bar = [&](int s) { return bar0 + 8u * (2 * CS + 2 * XS + 4 + AS + s); };
-  auto sxfull_bar = [&](int t) { return bar0 + 8u * (2 * CS + 2 * XS + 4 + 2 * AS + t); };
-  auto sxempty_bar = [&](int t) { return bar0 + 8u * (2 * CS + 2 * XS + 4 + 2 * AS + SX_STAGES + t); };
+  auto afree_bar = [&](int a) { return bar0 + 8u * (2 * CS + 2 * XS + AB + a); };  // MMAs done with it
+  auto accfull_bar = [&](int s) { return bar0 + 8u * (2 * CS + 2 * XS + 2 * AB + s); };
+  auto accempty_bar = [&](int s) { return bar0 + 8u * (2 * CS + 2 * XS + 2 * AB + AS + s); };
+  auto sxfull_bar = [&](int t) { return bar0 + 8u * (2 * CS + 2 * XS + 2 * AB + 2 * AS + t); };
+  auto sxempty_bar = [&](int t) { return bar0 + 8u * (2 * CS + 2 * XS + 2 * AB + 2 * AS + SX_STAGES + t); };
   const uint32_t base = smem_u32(smem);
   auto c_tile = [&](int c) { return base + static_cast<uint32_t>(c) * C_BYTES; };
   auto x_tile = [&](int x, int h) {  // half h (in-features 64 h .. 64 h + 63 of the group)
@@ -227,8 +269,8 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
       mbar_init(xfull_bar(x), 1);
       mbar_init(xempty_bar(x), 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(dq_bar(a), UNPACK_WARPS / 2);  // the four warps of the set that writes operand a
+    for (int a = 0; a < AB; ++a) {
+      mbar_init(dq_bar(a), UNPACK_WARPS / 2);  // the four warps of the set that writes the group
       mbar_init(afree_bar(a), 1);
     }
     for (int s = 0; s < AS; ++s) {
@@ -236,7 +278,7 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
       mbar_init(accempty_bar(s), 4);
     }
     for (int t = 0; t < SX_STAGES; ++t) {
-      mbar_init(sxfull_bar(t), UNPACK_WARPS / 2);
+      mbar_init(sxfull_bar(t), 1);  // the loader's arrive with the bulk copy's bytes
       mbar_init(sxempty_bar(t), 4);
     }
     failed = 0;
@@ -259,14 +301,18 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     __syncwarp();
     return true;
   };
+  // X' of local group i, and its Sx_g into the Sx ring (freed by the epilogue).
   auto load_x = [&](int i) -> bool {
-    const int x = i % XS;
-    const uint32_t use = static_cast<uint32_t>(i / XS);
+    const int x = i % XS, t = i % SX_STAGES;
+    const uint32_t use = static_cast<uint32_t>(i / XS), sx_use = static_cast<uint32_t>(i / SX_STAGES);
     if (use > 0 && !wait_warp(xempty_bar(x), (use - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
+    if (sx_use > 0 && !wait_warp(sxempty_bar(t), (sx_use - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
     if (lane == 0) {
       mbar_arrive_expect_tx(xfull_bar(x), S::X_BYTES);
       tma_load_2d(x_tile(x, 0), &tmX, (g0 + i) * GK, 0, xfull_bar(x));
       tma_load_2d(x_tile(x, 1), &tmX, (g0 + i) * GK + BK, 0, xfull_bar(x));
+      mbar_arrive_expect_tx(sxfull_bar(t), NT * 4);
+      bulk_load(sx_slot(t), p.sx + static_cast<int64_t>(g0 + i) * NT, NT * 4, sxfull_bar(t));
     }
     __syncwarp();
     return true;
@@ -274,14 +320,14 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
   // The first groups need no free slots: warp 0 requests them right after initialising the barriers, so
   // the first memory round trip overlaps the tensor-memory allocation and the CTA barrier.
   const int pre_c = min(ng, CS * GROUPS_PER_BOX);
-  const int pre_x = min(ng, XS);
+  const int pre_x = min(ng, min(XS, SX_STAGES));
   if (warp == 0) {
     __syncwarp();  // the barriers thread 0 initialised are visible to the whole warp
-    // in the order the groups need them: a box, then X' of its two groups
-    for (int i = 0; i < max(pre_c, pre_x); ++i) {
-      if (i < pre_c && i % GROUPS_PER_BOX == 0) load_codes(i);
-      if (i < pre_x) load_x(i);
-    }
+    // the code boxes first (they do not depend on the kernel before this one), then, once its X' copy
+    // and group sums are complete, X' and Sx of the first groups
+    for (int i = 0; i < pre_c; i += GROUPS_PER_BOX) load_codes(i);
+    pdl_wait();
+    for (int i = 0; i < pre_x; ++i) load_x(i);
   }
   if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), S::TMEM_COLS);
   tc_fence_before();
@@ -307,10 +353,10 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     if (elect_one()) {
       bool ok = true;
       for (int i = 0; i < ng && ok; ++i) {
-        const int x = i % XS, s = i % AS, a = i % 2;
+        const int x = i % XS, s = i % AS, a = i % AB;
         const uint32_t acc_use = static_cast<uint32_t>(i / AS);
         if (!wait_thread(xfull_bar(x), static_cast<uint32_t>(i / XS) & 1u, p, kSiteDecodeFull) ||
-            !wait_thread(dq_bar(a), static_cast<uint32_t>(i / 2) & 1u, p, kSiteDecodeDequant) ||
+            !wait_thread(dq_bar(a), static_cast<uint32_t>(i / AB) & 1u, p, kSiteDecodeDequant) ||
             (acc_use > 0 && !wait_thread(accempty_bar(s), (acc_use - 1u) & 1u, p, kSiteDecodeAcc))) {
           ok = false;
           break;
@@ -332,19 +378,14 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     }
     __syncwarp();
   } else if (warp < EPI_WARP0) {
-    // ------------------------------------------------------------------------------ unpack and Sx_g
-    // Warps 2-5 take the even groups into operand 0, 6-9 the odd ones into operand 1.
+    // ------------------------------------------------------------------------------ unpack
+    // Warps 2-5 take the even groups, 6-9 the odd ones; group i goes to operand buffer i % 3.
     const int q = warp & 3, set = (warp - 2) >> 2;
     const int r = 32 * q + lane;
     const uint32_t sw = static_cast<uint32_t>(r & 7);
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-    // Sx_g: thread tt of the set's 128 sums 16 / TPT chunks (8 in-features each) of token tt / TPT, in
-    // chunk and element order; the TPT threads of a token (adjacent lanes) then add by a fixed tree.
-    constexpr int TPT = S::TPT, CPT = 16 / TPT;
-    const int tt = 32 * q + lane, m_sx = tt / TPT, part = tt % TPT;
     for (int i = set; i < ng; i += 2) {
       const int j = i / GROUPS_PER_BOX, c = j % CS;
-      const int x = i % XS, t = i % SX_STAGES;
       if (!wait_warp(cfull_bar(c), static_cast<uint32_t>(j / CS) & 1u, p, kSiteDecodeFull)) {
         failed = 1;
         break;
@@ -357,40 +398,10 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
         wv[u] = ld_shared_v4(line_c + (((static_cast<uint32_t>(4 * (i % GROUPS_PER_BOX) + u)) ^ sw) << 4));
       __syncwarp();
       if (lane == 0) mbar_arrive(cempty_bar(c));  // the words are in registers
-      // Sx_g from the group's X' tile
-      const uint32_t sx_use = static_cast<uint32_t>(i / SX_STAGES);
-      if (!wait_warp(xfull_bar(x), static_cast<uint32_t>(i / XS) & 1u, p, kSiteDecodeFull) ||
-          (sx_use > 0 && !wait_warp(sxempty_bar(t), (sx_use - 1u) & 1u, p, kSiteDecodeEmpty))) {
-        failed = 1;
-        break;
-      }
-      float sum = 0.0f;
-      if (m_sx < NT) {
-#pragma unroll
-        for (int u = 0; u < CPT; ++u) {
-          const int ch = part * CPT + u, h = ch >> 3, cc = ch & 7;
-          const uint32_t a = x_tile(x, h) + static_cast<uint32_t>(m_sx) * 128u +
-                             ((static_cast<uint32_t>(cc) ^ static_cast<uint32_t>(m_sx & 7)) << 4);
-          const uint4 v = ld_shared_v4(a);  // (k0 k1) (k2 k3) (k4 k5) (k6 k7)
-          const uint32_t e[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            sum = __fadd_rn(__fadd_rn(sum, __uint_as_float(e[k] << 16)), __uint_as_float(e[k] & 0xFFFF0000u));
-          // the operand's order 0 4 1 5 2 6 3 7
-          st_shared_v4(a, make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
-                                     __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632)));
-        }
-      }
-      fence_proxy_async_smem();  // the MMAs read the permuted X' through the async proxy
-#pragma unroll
-      for (int off = 1; off < TPT; off <<= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, off));
-      if (part == 0 && m_sx < NT)
-        asm volatile("st.shared.f32 [%0], %1;" ::"r"(sx_slot(t) + 4u * static_cast<uint32_t>(m_sx)), "f"(sum) : "memory");
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sxfull_bar(t));
       // the operand
-      const uint32_t ause = static_cast<uint32_t>(i / 2);
-      if (ause > 0 && !wait_warp(afree_bar(set), (ause - 1u) & 1u, p, kSiteDecodeEmpty)) {
+      const int a = i % AB;
+      const uint32_t ause = static_cast<uint32_t>(i / AB);
+      if (ause > 0 && !wait_warp(afree_bar(a), (ause - 1u) & 1u, p, kSiteDecodeEmpty)) {
         failed = 1;
         break;
       }
@@ -407,12 +418,12 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
 #pragma unroll
           for (int k = 0; k < 4; ++k) v[4 * u + k] = v4[k];
         }
-        tmem_st32(tl + static_cast<uint32_t>(S::A_COL0 + set * A_COLS + h * (A_COLS / 2)), v);
+        tmem_st32(tl + static_cast<uint32_t>(S::A_COL0 + a * A_COLS + h * (A_COLS / 2)), v);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(dq_bar(set));
+      if (lane == 0) mbar_arrive(dq_bar(a));
     }
   } else {
     // ------------------------------------------------------------------------------ group epilogue
@@ -425,10 +436,10 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     float y[NT];
 #pragma unroll
     for (int m = 0; m < NT; ++m) y[m] = 0.0f;
-    // steps and zero points two groups ahead
-    float st_n[2], z_n[2];
+    // steps and zero points SZ_AHEAD groups ahead, in registers
+    float st_n[SZ_AHEAD], z_n[SZ_AHEAD];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < SZ_AHEAD; ++u) {
       st_n[u] = u < ng ? __ldg(st_row + u) : 0.0f;
       z_n[u] = u < ng ? __ldg(z_row + u) : 0.0f;
     }
@@ -437,10 +448,13 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
       const int s = i % AS, t = i % SX_STAGES;
       const float step = st_n[0];
       const float c = __fadd_rn(128.0f, z_n[0]);
-      st_n[0] = st_n[1];
-      z_n[0] = z_n[1];
-      st_n[1] = i + 2 < ng ? __ldg(st_row + i + 2) : 0.0f;
-      z_n[1] = i + 2 < ng ? __ldg(z_row + i + 2) : 0.0f;
+#pragma unroll
+      for (int u = 0; u + 1 < SZ_AHEAD; ++u) {
+        st_n[u] = st_n[u + 1];
+        z_n[u] = z_n[u + 1];
+      }
+      st_n[SZ_AHEAD - 1] = i + SZ_AHEAD < ng ? __ldg(st_row + i + SZ_AHEAD) : 0.0f;
+      z_n[SZ_AHEAD - 1] = i + SZ_AHEAD < ng ? __ldg(z_row + i + SZ_AHEAD) : 0.0f;
       if (!wait_warp(accfull_bar(s), static_cast<uint32_t>(i / AS) & 1u, p, kSiteDecodeAcc) ||
           !wait_warp(sxfull_bar(t), static_cast<uint32_t>(i / SX_STAGES) & 1u, p, kSiteDecodeAcc)) {
         have = false;

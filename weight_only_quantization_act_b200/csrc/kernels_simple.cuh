@@ -14,12 +14,12 @@ namespace awq {
 // order (256-row chunks; rows in increasing order inside a chunk; chunk totals in chunk order).
 // ===================================================================================================
 constexpr int kMaxGrid = 64;  // largest n_grid (AWQ_MAX_N_GRID)
-constexpr int kActChunk = 256;          // rows per chunk of the fixed-order sum
-constexpr int kActThreads = 256;        // one column per thread
-constexpr int kActColsPerBlock = kActThreads;
-constexpr int kActStageRows = 16;       // rows per cp.async stage (16 x 512 B = 8 KB)
-constexpr int kActStages = 8;           // stages in flight per CTA (64 KB)
-constexpr int kActSmemBytes = kActStages * kActStageRows * kActColsPerBlock * 2;
+constexpr int kActChunk = 256;       // rows per chunk of the fixed-order sum
+constexpr int kActCols = 8;          // adjacent columns per thread: one 16-byte load per row
+constexpr int kActThreads = 64;
+constexpr int kActColsPerBlock = kActThreads * kActCols;  // 512 columns per work item
+constexpr int kActRowsAhead = 4;     // rows per block of loads (two blocks in flight per thread)
+constexpr int kActCtasPerSm = 16;    // resident CTAs per SM the host sizes the grid for
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -30,72 +30,133 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(Pending) : "memory");
 }
 
-// grid (ceil(K / 256), n_chunks). The CTA streams its chunk's 256-column slab through shared memory
-// with cp.async (8 stages of 16 rows in flight); thread t then adds column t's values in row order.
+// 16 bytes that are read once: not kept in L1.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+// The magnitude of a bf16 as a double scaled by 2^-896: the bf16's 15 magnitude bits moved to the top of
+// the double (its 8-bit exponent field becomes the low bits of the double's 11-bit one, its 7 mantissa
+// bits the leading mantissa bits), i.e. |x| * 2^(127 - 1023) exactly, zero and subnormal bf16 values
+// included (they become zero and subnormal doubles). This replaces a conversion instruction per element
+// by an AND and a multiply on the integer and FMA pipes. Finite inputs only (the interface's contract).
+//
+// Sums of these are exactly 2^-896 times the fp64 sums of the unscaled values in the same order: the
+// addends are non-negative, so a running sum only grows; while it is below 2^-1022 (scaled) every sum of
+// bf16 magnitudes is exact in both scalings (multiples of 2^-133 with few significant bits), and from
+// there on every result is a normal double in both, where rounding commutes with the power-of-two scale.
+__device__ __forceinline__ double scaled_abs_lo(uint32_t w) { return __hiloint2double((w & 0x7FFFu) * 8192u, 0); }
+__device__ __forceinline__ double scaled_abs_hi(uint32_t w) {
+  return __hiloint2double(__umulhi(w & 0x7FFF0000u, 1u << 29), 0);
+}
+constexpr double kActUnscale = 0x1p896;
+
+__device__ __forceinline__ void add_row8(double (&acc)[kActCols], const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] = __dadd_rn(acc[2 * i], scaled_abs_lo(w[i]));
+    acc[2 * i + 1] = __dadd_rn(acc[2 * i + 1], scaled_abs_hi(w[i]));
+  }
+}
+
+// Work item (chunk ch, column block cb) = rows [256 ch, 256 ch + 256) x columns [512 cb, 512 cb + 512);
+// items are numbered chunk-major and CTA b takes items b, b + gridDim.x, ... Thread t sums its 8 adjacent
+// columns down the chunk, one row at a time in increasing order (fp64, scaled by 2^-896), from 16-byte
+// loads in blocks of 4 rows, the next block's loads issued before the current block's additions, and
+// writes the 8 scaled chunk sums to part[ch][k]. K is even, so a ragged last column block ends on a whole
+// pair; its thread reads pairs with 4-byte loads.
 __global__ void __launch_bounds__(kActThreads) act_chunk_sums_kernel(const uint16_t* __restrict__ X,
                                                                      int64_t N, int64_t K, int64_t ldx,
                                                                      double* __restrict__ part) {
-  extern __shared__ __align__(16) uint16_t act_stage[];  // [kActStages][kActStageRows][256]
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kActColsPerBlock;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kActChunk;
-  const int rows = static_cast<int>(min(static_cast<int64_t>(kActChunk), N - r0));
-  const int n_stages = (rows + kActStageRows - 1) / kActStageRows;
-  // copy assignment: each thread moves 2 x 16 B of a stage (rows tid/32 and tid/32 + 8, piece tid%32)
-  const int piece = threadIdx.x & 31;
-  const int64_t pcol = c0 + piece * 8;
-  const uint32_t pbytes = pcol >= K ? 0u : static_cast<uint32_t>(min(static_cast<int64_t>(8), K - pcol) * 2);
-  const uint32_t smem0 = static_cast<uint32_t>(__cvta_generic_to_shared(act_stage));
-  auto issue = [&](int stg) {
-    if (stg < n_stages) {
-      const int slot = stg % kActStages;
+  constexpr int B = kActRowsAhead;
+  const int64_t nx = (K + kActColsPerBlock - 1) / kActColsPerBlock;
+  const int64_t items = nx * ((N + kActChunk - 1) / kActChunk);
+#pragma unroll 1
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int64_t ch = it / nx;
+    const int64_t c = (it - ch * nx) * kActColsPerBlock + static_cast<int64_t>(threadIdx.x) * kActCols;
+    if (c >= K) continue;
+    const int64_t r0 = ch * kActChunk;
+    const int nr = static_cast<int>(min(static_cast<int64_t>(kActChunk), N - r0));
+    const uint16_t* p = X + r0 * ldx + c;
+    double acc[kActCols];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int rr = (threadIdx.x >> 5) + 8 * h;
-        const int row = stg * kActStageRows + rr;
-        const uint32_t dst = smem0 + static_cast<uint32_t>(((slot * kActStageRows + rr) * kActColsPerBlock +
-                                                            piece * 8) * 2);
-        const bool ok = row < rows && pbytes != 0u;
-        const uint16_t* src = ok ? X + (r0 + row) * ldx + pcol : X;
-        cp_async_16(dst, src, ok ? pbytes : 0u);
+    for (int j = 0; j < kActCols; ++j) acc[j] = 0.0;
+    if (c + kActCols <= K) {
+      const int nb = nr / B;  // whole blocks; the last nr % B rows follow one at a time
+      uint4 va[B], vb[B];
+      if (nb > 0) {
+#pragma unroll
+        for (int u = 0; u < B; ++u) va[u] = ld_stream16(p + u * ldx);
       }
-    }
-    cp_async_commit();  // an empty group keeps the wait arithmetic uniform
-  };
 #pragma unroll 1
-  for (int stg = 0; stg < kActStages - 1; ++stg) issue(stg);
-  const int64_t col = c0 + threadIdx.x;
-  double sum = 0.0;
-#pragma unroll 1
-  for (int stg = 0; stg < n_stages; ++stg) {
-    issue(stg + kActStages - 1);
-    cp_async_wait<kActStages - 1>();
-    __syncthreads();
-    const int slot = stg % kActStages;
-    const int nr = min(kActStageRows, rows - stg * kActStageRows);
-    const uint16_t* sp = act_stage + (slot * kActStageRows) * kActColsPerBlock + threadIdx.x;
-    if (nr == kActStageRows) {
+      for (int b = 0; b < nb; b += 2) {
+        if (b + 1 < nb) {
 #pragma unroll
-      for (int r = 0; r < kActStageRows; ++r)
-        sum = __dadd_rn(sum, fabs(static_cast<double>(__uint_as_float(static_cast<uint32_t>(sp[r * kActColsPerBlock]) << 16))));
+          for (int u = 0; u < B; ++u) vb[u] = ld_stream16(p + ((b + 1) * B + u) * ldx);
+        }
+#pragma unroll
+        for (int u = 0; u < B; ++u) add_row8(acc, va[u]);
+        if (b + 2 < nb) {
+#pragma unroll
+          for (int u = 0; u < B; ++u) va[u] = ld_stream16(p + ((b + 2) * B + u) * ldx);
+        }
+        if (b + 1 < nb) {
+#pragma unroll
+          for (int u = 0; u < B; ++u) add_row8(acc, vb[u]);
+        }
+      }
+#pragma unroll 1
+      for (int r = nb * B; r < nr; ++r) add_row8(acc, ld_stream16(p + r * ldx));
+      double2* out = reinterpret_cast<double2*>(part + ch * K + c);  // K even, c % 8 == 0: 16-byte aligned
+#pragma unroll
+      for (int j = 0; j < kActCols / 2; ++j) out[j] = make_double2(acc[2 * j], acc[2 * j + 1]);
     } else {
-      for (int r = 0; r < nr; ++r)
-        sum = __dadd_rn(sum, fabs(static_cast<double>(__uint_as_float(static_cast<uint32_t>(sp[r * kActColsPerBlock]) << 16))));
+      const int pairs = static_cast<int>((K - c) / 2);  // 1 to 3
+#pragma unroll 1
+      for (int r = 0; r < nr; ++r) {
+        const uint32_t* q = reinterpret_cast<const uint32_t*>(p + r * ldx);
+#pragma unroll
+        for (int i = 0; i < kActCols / 2; ++i)
+          if (i < pairs) {
+            const uint32_t w = __ldg(q + i);
+            acc[2 * i] = __dadd_rn(acc[2 * i], scaled_abs_lo(w));
+            acc[2 * i + 1] = __dadd_rn(acc[2 * i + 1], scaled_abs_hi(w));
+          }
+      }
+#pragma unroll
+      for (int i = 0; i < kActCols / 2; ++i)
+        if (i < pairs) {
+          part[ch * K + c + 2 * i] = acc[2 * i];
+          part[ch * K + c + 2 * i + 1] = acc[2 * i + 1];
+        }
     }
-    __syncthreads();  // the slot is refilled by the next iteration's issue
   }
-  cp_async_wait<0>();
-  if (col < K) part[static_cast<int64_t>(blockIdx.y) * K + col] = sum;
 }
 
-// grid ceil(K / 256): chunk totals in chunk order, then the mean.
+// grid ceil(K / 256): the scaled chunk totals in chunk order (exactly 2^-896 times the unscaled fp64
+// sum, by the argument above), the exact power-of-two unscale, then the mean. Eight chunks' loads are in
+// flight per thread; the additions stay in chunk order.
 __global__ void __launch_bounds__(256) act_finalize_kernel(const double* __restrict__ part, int64_t N,
                                                            int64_t K, int n_chunks,
                                                            float* __restrict__ act_mean) {
   const int64_t k = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   if (k >= K) return;
   double S = 0.0;
-  for (int c = 0; c < n_chunks; ++c) S = __dadd_rn(S, part[static_cast<int64_t>(c) * K + k]);
-  act_mean[k] = __double2float_rn(__ddiv_rn(S, static_cast<double>(N)));
+  for (int c = 0; c < n_chunks; c += 8) {
+    double v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = c + u < n_chunks ? __ldcg(part + static_cast<int64_t>(c + u) * K + k) : 0.0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (c + u < n_chunks) S = __dadd_rn(S, v[u]);
+  }
+  act_mean[k] = __double2float_rn(__ddiv_rn(__dmul_rn(S, kActUnscale), static_cast<double>(N)));
 }
 
 // ===================================================================================================
@@ -440,55 +501,58 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(const double* __r
 constexpr int kPackThreads = 256;
 constexpr int kPackCols = 32;                    // in-features per lane (4 lanes per group of 128)
 constexpr int kPackWarpCols = 32 * kPackCols;    // 1024 in-features (one segment) per warp
-constexpr int kPackStages = 6;                   // rows in flight per warp (cp.async ring)
+constexpr int kPackStages = 4;                   // rows in flight per warp (cp.async ring)
 constexpr int kPackStageBytes = kPackWarpCols * 2;                                   // 2 KB
-constexpr int kPackSmemBytes = kPackStages * (kPackThreads / 32) * kPackStageBytes;  // 96 KB
+constexpr int kPackScaleBytes = kPackWarpCols * 4;                                   // 4 KB
+constexpr int kPackSmemBytes = kPackStages * (kPackThreads / 32) * kPackStageBytes + kPackScaleBytes;  // 68 KB
+constexpr int kPackCtasPerSm = 3;
 
-// Warp v owns segment v % segs and rows v / segs, v / segs + wps, ... (wps = warps per segment): the
-// segment's scales stay in registers. Each lane streams its own 64 bytes of the next rows through a
-// ring in shared memory with cp.async (up to kPackStages - 1 rows in flight per warp, no registers
-// held); a lane only reads back what it copied itself, so the ring is laid out for conflict-free
-// access (16-byte piece j of lane l at slot offset 16 (32 j + l)) and needs no warp synchronisation.
-// With fewer warps than segments a warp walks several whole segments.
-__global__ void __launch_bounds__(kPackThreads, 2) quantize_pack_kernel(
+// CTA b owns segment b % segs and, warp w, rows 8 (b / segs) + w, stepping by 8 x (CTAs per segment);
+// with fewer CTAs than segments a CTA walks several whole segments. The segment's scales sit once in
+// shared memory (16-byte piece j of lane l's 32 at offset 16 (32 j + l): conflict-free) and are read back
+// for every row, which keeps registers for three CTAs per SM. Each lane streams its own 64 bytes of the
+// next rows through a ring in shared memory with cp.async (up to kPackStages - 1 rows in flight per
+// warp, no registers held); a lane only reads back what it copied itself, laid out the same way, so the
+// ring needs no synchronisation.
+__global__ void __launch_bounds__(kPackThreads, kPackCtasPerSm) quantize_pack_kernel(
     const uint16_t* __restrict__ W, int64_t O, int64_t K, int64_t ldw, const float* __restrict__ scales,
     int exact, uint32_t* __restrict__ codes, float* __restrict__ steps, float* __restrict__ zeros) {
   extern __shared__ __align__(16) uint8_t pack_ring[];
   const int64_t segs = (K + kPackWarpCols - 1) / kPackWarpCols;
-  const int64_t v = (static_cast<int64_t>(blockIdx.x) * kPackThreads + threadIdx.x) >> 5;
-  const int64_t total = (static_cast<int64_t>(gridDim.x) * kPackThreads) >> 5;
+  const int64_t ctas = gridDim.x;
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(pack_ring)) +
-                        static_cast<uint32_t>((threadIdx.x >> 5) * kPackStages * kPackStageBytes) +
+  const uint32_t smem0 = static_cast<uint32_t>(__cvta_generic_to_shared(pack_ring));
+  const uint32_t scl = smem0 + static_cast<uint32_t>(kPackStages * (kPackThreads / 32) * kPackStageBytes) +
+                       static_cast<uint32_t>(lane) * 16u;
+  const uint32_t ring = smem0 + static_cast<uint32_t>(warp * kPackStages * kPackStageBytes) +
                         static_cast<uint32_t>(lane) * 16u;
   int64_t seg_first, seg_step, row_first, row_step;
-  if (total >= segs) {
-    const int64_t wps = total / segs;
-    if (v >= wps * segs) return;  // whole warps exit together
-    seg_first = v % segs;
+  if (ctas >= segs) {
+    const int64_t cps = ctas / segs;
+    if (static_cast<int64_t>(blockIdx.x) >= cps * segs) return;  // the whole CTA
+    seg_first = blockIdx.x % segs;
     seg_step = segs;  // one segment
-    row_first = v / segs;
-    row_step = wps;
+    row_first = (blockIdx.x / segs) * (kPackThreads / 32) + warp;
+    row_step = cps * (kPackThreads / 32);
   } else {
-    seg_first = v;
-    seg_step = total;
-    row_first = 0;
-    row_step = 1;
+    seg_first = blockIdx.x;
+    seg_step = ctas;
+    row_first = warp;
+    row_step = kPackThreads / 32;
   }
   for (int64_t seg = seg_first; seg < segs; seg += seg_step) {
     const int64_t k0 = seg * kPackWarpCols + static_cast<int64_t>(lane) * kPackCols;
     const bool active = k0 < K;  // K % 128 == 0: 4-lane groups are all active or all idle
-    float s[kPackCols];
-    if (active) {
-      const float4* ps = reinterpret_cast<const float4*>(scales + k0);
-#pragma unroll
-      for (int i = 0; i < kPackCols / 4; ++i) {
-        const float4 x = __ldg(ps + i);
-        s[4 * i] = x.x; s[4 * i + 1] = x.y; s[4 * i + 2] = x.z; s[4 * i + 3] = x.w;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < kPackCols; ++i) s[i] = 1.0f;
+    {
+      // thread (w, l) stages piece w of lane l's scales (1.0 past K)
+      const int64_t kk = seg * kPackWarpCols + static_cast<int64_t>(lane) * kPackCols + 4 * warp;
+      const float4 x = kk < K ? __ldg(reinterpret_cast<const float4*>(scales + kk)) : make_float4(1.f, 1.f, 1.f, 1.f);
+      __syncthreads();  // the previous segment's scales are no longer read
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(scl + static_cast<uint32_t>(warp * 512)),
+                   "f"(x.x), "f"(x.y), "f"(x.z), "f"(x.w)
+                   : "memory");
+      __syncthreads();
     }
     // row i of this warp is o = row_first + i * row_step, staged in slot i % kPackStages
     auto issue = [&](int64_t i) {
@@ -516,22 +580,35 @@ __global__ void __launch_bounds__(kPackThreads, 2) quantize_pack_kernel(
                      : "=r"(cur[j].x), "=r"(cur[j].y), "=r"(cur[j].z), "=r"(cur[j].w)
                      : "r"(src + static_cast<uint32_t>(j * 512))
                      : "memory");
-      // w' = RN(w * s) in pairs (elements 2i, 2i+1 of the lane's 32 in-features)
+      // w' = RN(w * s) in pairs (elements 2i, 2i+1 of the lane's 32 in-features); the lane's max and min
+      // by a tree of three-input min/max (8 partial results of 4 elements each, then 3, then 1)
       uint64_t wp2[kPackCols / 2];
-      float mx = -__int_as_float(0x7f800000), mn = __int_as_float(0x7f800000);
+      float px[8], pn[8];
 #pragma unroll
       for (int v4 = 0; v4 < 4; ++v4) {
         const uint32_t uu[4] = {cur[v4].x, cur[v4].y, cur[v4].z, cur[v4].w};
+        float4 sa, sb;  // scales of elements 8 v4 .. 8 v4 + 7
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(sa.x), "=f"(sa.y), "=f"(sa.z), "=f"(sa.w)
+                     : "r"(scl + static_cast<uint32_t>(2 * v4 * 512)));
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(sb.x), "=f"(sb.y), "=f"(sb.z), "=f"(sb.w)
+                     : "r"(scl + static_cast<uint32_t>((2 * v4 + 1) * 512)));
+        wp2[4 * v4 + 0] = fx2_mul(fx2(bf16_lo(uu[0]), bf16_hi(uu[0])), fx2(sa.x, sa.y));
+        wp2[4 * v4 + 1] = fx2_mul(fx2(bf16_lo(uu[1]), bf16_hi(uu[1])), fx2(sa.z, sa.w));
+        wp2[4 * v4 + 2] = fx2_mul(fx2(bf16_lo(uu[2]), bf16_hi(uu[2])), fx2(sb.x, sb.y));
+        wp2[4 * v4 + 3] = fx2_mul(fx2(bf16_lo(uu[3]), bf16_hi(uu[3])), fx2(sb.z, sb.w));
 #pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const int e = 8 * v4 + 2 * e2;
-          wp2[e / 2] = fx2_mul(fx2(bf16_lo(uu[e2]), bf16_hi(uu[e2])), fx2(s[e], s[e + 1]));
-          float a, b;
-          fx2_split(wp2[e / 2], a, b);
-          mx = max3f(mx, a, b);
-          mn = min3f(mn, a, b);
+        for (int h = 0; h < 2; ++h) {
+          float a0, b0, a1, b1;
+          fx2_split(wp2[4 * v4 + 2 * h], a0, b0);
+          fx2_split(wp2[4 * v4 + 2 * h + 1], a1, b1);
+          px[2 * v4 + h] = max3f(a0, b0, fmaxf(a1, b1));
+          pn[2 * v4 + h] = min3f(a0, b0, fminf(a1, b1));
         }
       }
+      float mx = max3f(max3f(px[0], px[1], px[2]), max3f(px[3], px[4], px[5]), fmaxf(px[6], px[7]));
+      float mn = min3f(min3f(pn[0], pn[1], pn[2]), min3f(pn[3], pn[4], pn[5]), fminf(pn[6], pn[7]));
 #pragma unroll
       for (int off = 1; off < 4; off <<= 1) {
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -546,25 +623,30 @@ __global__ void __launch_bounds__(kPackThreads, 2) quantize_pack_kernel(
         // t = RN(RN(w' * rstep) + C); its low byte is the code; pairs of codes are joined by one
         // integer multiply-add (t1 * 16 + t0: the low byte is c0 + 16 c1, no carry out of it), two
         // pairs by another (p23 * 256 + p01), and the two halves of a word by a byte permute.
+        // The tie test |d| < kTieMargin is taken on RN(d^2) < RN(kTieMargin^2), which implies it (RN is
+        // monotone), from a paired multiply and one three-input max per pair.
         const uint64_t rs2 = fx2(g.rstep, g.rstep), C2 = fx2(C, C);
-        float dmax = 0.0f;
+        float dq[4];
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
           uint32_t p[4];  // p[e2]: low byte = codes of elements 8w + 2e2 and 8w + 2e2 + 1
+          float q0 = 0.0f, q1 = 0.0f;
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
             const uint64_t qa = fx2_mul(wp2[4 * w + e2], rs2);
             const uint64_t t = fx2_add(qa, C2);
             const uint64_t d = fx2_sub(qa, fx2_sub(t, C2));
             float d0, d1, t0, t1;
-            fx2_split(d, d0, d1);
+            fx2_split(fx2_mul(d, d), d0, d1);
             fx2_split(t, t0, t1);
-            dmax = max3f(dmax, fabsf(d0), fabsf(d1));
+            if (e2 < 2) q0 = max3f(q0, d0, d1);
+            else q1 = max3f(q1, d0, d1);
             p[e2] = __float_as_uint(t1) * 16u + __float_as_uint(t0);
           }
+          dq[w] = fmaxf(q0, q1);
           word[w] = __byte_perm(p[1] * 256u + p[0], p[3] * 256u + p[2], 0x5410);
         }
-        fast = dmax < kTieMargin;
+        fast = fmaxf(fmaxf(dq[0], dq[1]), fmaxf(dq[2], dq[3])) < kTieMarginSq;
       }
       if (!fast) {
 #pragma unroll

@@ -294,6 +294,7 @@ __device__ __forceinline__ float min3f(float a, float b, float c) {
 // ===================================================================================================
 constexpr float kQuantMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr float kTieMargin = 0.5f - 0x1p-14f;
+constexpr float kTieMarginSq = 0.24993896484375f;  // RN32(kTieMargin^2) = RN32(0.25 - 2^-14 + 2^-28) = 0.25 - 2^-14
 
 __device__ __forceinline__ bool fast_group(const GroupParams& g, float mx, float mn, float& C) {
   if (!(fabsf(g.zero) < 2097152.0f)) return false;
