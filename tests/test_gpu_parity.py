@@ -38,15 +38,19 @@ def test_act_stats_strided_input():
     assert_bits_equal(awq.act_stats(Xd), orc.act_mean(wide[:, 128:384]), "strided")
 
 
-@pytest.mark.parametrize("shape", [(600, 1030), (37, 2), (513, 2056), (256, 1024)])
+@pytest.mark.parametrize("shape", [(600, 1030), (37, 2), (513, 2056), (256, 1024), (51277, 1030)])
 def test_act_stats_special_magnitudes(shape):
     """Zeros, subnormals and magnitudes across the whole finite bf16 exponent range, both signs, with a
-    ragged last column block (K % 8 != 0) and row counts off the 8-row load blocks."""
+    ragged last column block (K % 8 != 0) and row counts off the load blocks. The small shapes take the
+    narrow chunk-sum kernel; 51277 x 1030 (201 chunks, the last ragged, x 3 column blocks) takes the wide
+    one, whose last column block holds 6 columns."""
     rng = np.random.default_rng(shape[0] + 31 * shape[1])
-    e = np.where(rng.random(shape) < 0.5, rng.integers(0, 255, shape), rng.integers(0, 4, shape))
-    bits = (rng.integers(0, 2, shape) << 15) | (e << 7) | rng.integers(0, 128, shape)
-    bits[rng.random(shape) < 0.1] = 0
-    X = bits.astype(np.uint16)
+    u16 = np.uint16
+    e = rng.integers(0, 255, shape, dtype=u16)
+    small = rng.integers(0, 2, shape, dtype=np.uint8).astype(bool)
+    e[small] = e[small] & u16(3)                   # half the entries: exponent fields 0-3 (subnormal, tiny)
+    X = (rng.integers(0, 2, shape, dtype=u16) << u16(15)) | (e << u16(7)) | rng.integers(0, 128, shape, dtype=u16)
+    X[rng.integers(0, 10, shape, dtype=np.uint8) == 0] = 0
     ld = -(-shape[1] // 8) * 8                     # row stride: the next multiple of 8
     wide = np.zeros((shape[0], ld), np.uint16)
     wide[:, :shape[1]] = X

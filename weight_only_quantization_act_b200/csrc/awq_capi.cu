@@ -311,18 +311,27 @@ awq_status check_launch(const char* what) {
   return AWQ_OK;
 }
 
-// Column sums of |A| (rows x K, stride ld) in the statistic's fixed order, then their means: the chunk-sum
-// kernel over (chunk, 512-column block) work items, as many CTAs as make every CTA take the same number of
-// items within kActCtasPerSm resident CTAs per SM, then the finaliser over the fp64 partial array part.
+// Column sums of |A| (rows x K, stride ld) in the statistic's fixed order, then their means: a chunk-sum
+// kernel over (chunk, column block) work items, as many CTAs as make every CTA take the same number of
+// items within the resident CTAs of the device, then the finaliser over the fp64 partial array part. Layers
+// with fewer than four 512-column items per SM take the narrow kernel (256-column items, more rows in
+// flight per thread).
 awq_status launch_act_stats(const void* A, int64_t rows, int64_t K, int64_t ld, double* part, float* mean, int sms,
                             cudaStream_t st) {
   const int64_t n_chunks = (rows + awq::kActChunk - 1) / awq::kActChunk;
-  const int64_t items = n_chunks * ((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock);
-  const int64_t resident = static_cast<int64_t>(sms) * awq::kActCtasPerSm;
+  const int64_t wide_items = n_chunks * ((K + awq::kActColsPerBlock - 1) / awq::kActColsPerBlock);
+  const bool narrow = wide_items < 4ll * sms;
+  const int64_t items = narrow ? n_chunks * ((K + awq::kActNarrowColsPerBlock - 1) / awq::kActNarrowColsPerBlock)
+                               : wide_items;
+  const int64_t resident = static_cast<int64_t>(sms) * (narrow ? awq::kActNarrowCtasPerSm : awq::kActCtasPerSm);
   const int64_t per_cta = (items + resident - 1) / resident;
   const int64_t ctas = (items + per_cta - 1) / per_cta;
-  awq::act_chunk_sums_kernel<<<static_cast<unsigned>(ctas), awq::kActThreads, 0, st>>>(
-      static_cast<const uint16_t*>(A), rows, K, ld, part);
+  if (narrow)
+    awq::act_chunk_sums_narrow_kernel<<<static_cast<unsigned>(ctas), awq::kActNarrowThreads, 0, st>>>(
+        static_cast<const uint16_t*>(A), rows, K, ld, part);
+  else
+    awq::act_chunk_sums_kernel<<<static_cast<unsigned>(ctas), awq::kActThreads, 0, st>>>(
+        static_cast<const uint16_t*>(A), rows, K, ld, part);
   {
     awq_status s = check_launch("act_chunk_sums_kernel");
     if (s != AWQ_OK) return s;
