@@ -33,7 +33,7 @@
 //   2-9    unpack: warps 2-5 take the even groups, warps 6-9 the odd ones; lane l of warp w unpacks row
 //          32 (w % 4) + l (the tensor-memory lanes warp w may write) with two 32-column stores
 //   10-13  per group: S_g of their lane quarter, minus the zero-point term, times step, added to per-row
-//          registers (steps and zero points read from global memory two groups ahead); at the end Y, or
+//          registers (steps and zero points read from global memory four groups ahead); at the end Y, or
 //          this slice's partial sums
 // With several slices the last CTA of a row block to finish (a per-block counter it resets to zero)
 // adds the slices' partial sums in slice order (deterministic). All waits are bounded; a timeout is
@@ -185,13 +185,16 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&v)[4]) {
 }
 
 // X' for the few-token kernel: Xp[m][k] = X[m][k] for m < M, zero for M <= m < nt, with each 16-byte chunk
-// of 8 in-features in the operand order 0 4 1 5 2 6 3 7; Sx[g][m] = sum of X[m][k] over the group's 128
-// in-features in increasing k (fp32, zero past M). One CTA per group.
+// of 8 in-features in the operand order 0 4 1 5 2 6 3 7; Sx[g][m] = the sum of X[m][k] over the group's
+// 128 in-features (fp32: each chunk's 8 values in increasing k, then the 16 chunk sums in order; zero past
+// M). One CTA per group; every (token, chunk) pair is one 16-byte load, so the kernel is one memory round
+// trip long.
 constexpr int PREP_THREADS = 128;
 __global__ void __launch_bounds__(PREP_THREADS) decode_prep_kernel(const uint16_t* __restrict__ X, int64_t M,
                                                                    int64_t K, int64_t ldx, int nt,
                                                                    uint16_t* __restrict__ Xp, float* __restrict__ Sx) {
   pdl_launch_dependents();
+  __shared__ float chunk_sum[MAX_NT][GK / 8];
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * GK;
   for (int task = threadIdx.x; task < nt * (GK / 8); task += PREP_THREADS) {
     const int m = task / (GK / 8), ch = task % (GK / 8);
@@ -199,21 +202,19 @@ __global__ void __launch_bounds__(PREP_THREADS) decode_prep_kernel(const uint16_
     *reinterpret_cast<uint4*>(Xp + static_cast<int64_t>(m) * K + k0 + 8 * ch) =
         make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632), __byte_perm(v.y, v.w, 0x5410),
                    __byte_perm(v.y, v.w, 0x7632));
+    const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+    float sum = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      sum = __fadd_rn(__fadd_rn(sum, __uint_as_float(e[k] << 16)), __uint_as_float(e[k] & 0xFFFF0000u));
+    chunk_sum[m][ch] = sum;
   }
+  __syncthreads();
   if (threadIdx.x < nt) {
     const int m = threadIdx.x;
     float sum = 0.0f;
-    if (m < M) {
-      const uint4* row = reinterpret_cast<const uint4*>(X + m * ldx + k0);
-#pragma unroll 4
-      for (int ch = 0; ch < GK / 8; ++ch) {
-        const uint4 v = row[ch];
-        const uint32_t e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          sum = __fadd_rn(__fadd_rn(sum, __uint_as_float(e[k] << 16)), __uint_as_float(e[k] & 0xFFFF0000u));
-      }
-    }
+    for (int ch = 0; ch < GK / 8; ++ch) sum = __fadd_rn(sum, chunk_sum[m][ch]);
     Sx[static_cast<int64_t>(blockIdx.x) * nt + m] = sum;
   }
 }
