@@ -128,6 +128,20 @@ def test_quantize_pack_bit_exact(flags, scale_kind):
     assert_bits_equal(zeros, wzeros, "zeros")
 
 
+def test_quantize_pack_very_wide_rows():
+    """More 1024-in-feature segments than CTAs fit on the device (576 > 3 per SM x 148), so a CTA walks
+    several segments and restages the segment's scales between them: K = 589824 (576 whole segments) and
+    K = 589440 (the last segment 640 in-features, its upper lanes idle)."""
+    for K in (589824, 589824 - 384):
+        W = inputs.random_bf16((9, K), seed=21, scale=0.02)
+        s = (1.0 + np.random.default_rng(22).random(K)).astype(F32)
+        codes, steps, zeros = awq.quantize_pack(bf16_to_device(W), torch.from_numpy(s).cuda())
+        wc, ws, wz = orc.quantize_pack(W, s)
+        assert np.array_equal(codes.cpu().numpy().view(np.uint32), wc), K
+        assert_bits_equal(steps, ws, f"steps K={K}")
+        assert_bits_equal(zeros, wz, f"zeros K={K}")
+
+
 def test_quantize_pack_ragged_rows_and_stride():
     W = inputs.random_bf16((77, 640), seed=12, scale=0.02)
     s = orc.scale_table(orc.act_mean(inputs.random_bf16((64, 640), 13, outliers=3, factor=40)), 20)[17]

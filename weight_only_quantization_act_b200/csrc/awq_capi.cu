@@ -336,8 +336,8 @@ awq_status launch_act_stats(const void* A, int64_t rows, int64_t K, int64_t ld, 
     awq_status s = check_launch("act_chunk_sums_kernel");
     if (s != AWQ_OK) return s;
   }
-  awq::act_finalize_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, st>>>(part, rows, K,
-                                                                                   static_cast<int>(n_chunks), mean);
+  awq::act_finalize_kernel<<<static_cast<unsigned>((K + awq::kActFinalizeThreads - 1) / awq::kActFinalizeThreads),
+                             awq::kActFinalizeThreads, 0, st>>>(part, rows, K, static_cast<int>(n_chunks), mean);
   return check_launch("act_finalize_kernel");
 }
 
