@@ -67,6 +67,23 @@ def test_w4a16_matches_oracle(M, K, O):
     check_against_oracle(Xp, words, steps, zeros, Y)
 
 
+# Few tokens on layers with more 128-row blocks than CTAs fit on the device at once (B200: 296 at 16
+# tokens, 148 above): X' is then prepared by a kernel of its own that the GEMM follows as a programmatic
+# dependent, instead of inside the GEMM's cooperative launch; both paths, run back to back, share the
+# workspace's per-group flags.
+@pytest.mark.parametrize("M,K,O", [(16, 256, 38400), (40, 384, 19200), (16, 256, 512)])
+def test_w4a16_decode_both_preparation_paths(M, K, O):
+    _, _, (words, steps, zeros) = quantized(O, K, M + K + O + 5)
+    Xp = inputs.random_bf16((M, K), 3 * M + 2, scale=1.0)
+    lib = awq.load_library()
+    ws = torch.zeros(lib.awq_w4a16_workspace_size(K, O), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        Y = awq.w4a16_gemm(bf16_to_device(Xp), torch.from_numpy(words.view(np.int32)).cuda(),
+                           torch.from_numpy(steps).cuda(), torch.from_numpy(zeros).cuda(), workspace=ws)
+        torch.cuda.synchronize()
+        check_against_oracle(Xp, words, steps, zeros, Y)
+
+
 # Many tokens at the tile counts the prefill kernel really runs: tiles of 512 tokens x 256 weight rows
 # handed out dynamically over the device's CTA pairs (74 on B200), so most pairs run a second and a
 # third tile. This is where the one-tile-ahead index publishing, the code ring across tiles and the

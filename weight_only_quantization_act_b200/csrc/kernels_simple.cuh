@@ -209,22 +209,22 @@ __global__ void __launch_bounds__(kActNarrowThreads) act_chunk_sums_narrow_kerne
   }
 }
 
-// grid ceil(K / 128) of 128 threads: the scaled chunk totals in chunk order (exactly 2^-896 times the
-// unscaled fp64 sum, by the argument above), the exact power-of-two unscale, then the mean. Sixteen
+// grid ceil(K / 256) of 256 threads: the scaled chunk totals in chunk order (exactly 2^-896 times the
+// unscaled fp64 sum, by the argument above), the exact power-of-two unscale, then the mean. Eight
 // chunks' loads are in flight per thread; the additions stay in chunk order.
-constexpr int kActFinalizeThreads = 128;
+constexpr int kActFinalizeThreads = 256;
 __global__ void __launch_bounds__(kActFinalizeThreads) act_finalize_kernel(const double* __restrict__ part, int64_t N,
                                                                            int64_t K, int n_chunks,
                                                                            float* __restrict__ act_mean) {
   const int64_t k = static_cast<int64_t>(blockIdx.x) * kActFinalizeThreads + threadIdx.x;
   if (k >= K) return;
   double S = 0.0;
-  for (int c = 0; c < n_chunks; c += 16) {
-    double v[16];
+  for (int c = 0; c < n_chunks; c += 8) {
+    double v[8];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) v[u] = c + u < n_chunks ? __ldcg(part + static_cast<int64_t>(c + u) * K + k) : 0.0;
+    for (int u = 0; u < 8; ++u) v[u] = c + u < n_chunks ? __ldcg(part + static_cast<int64_t>(c + u) * K + k) : 0.0;
 #pragma unroll
-    for (int u = 0; u < 16; ++u)
+    for (int u = 0; u < 8; ++u)
       if (c + u < n_chunks) S = __dadd_rn(S, v[u]);
   }
   act_mean[k] = __double2float_rn(__ddiv_rn(__dmul_rn(S, kActUnscale), static_cast<double>(N)));
