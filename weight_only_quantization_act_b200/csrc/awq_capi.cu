@@ -50,6 +50,7 @@ struct DeviceInfo {
   bool gemm_attr_set = false;
   int gemm_clusters = 0;  // CTA pairs of the loss GEMM that fit on the device at once
   int w4_clusters = 0;    // CTA pairs of the W4A16 GEMM that fit on the device at once
+  int dec_occ[4] = {0, 0, 0, 0};  // few-token GEMM CTAs per SM for 16, 32, 48, 64 tokens
 };
 
 constexpr int kMaxDevices = 64;
@@ -135,14 +136,22 @@ awq_status device_info(DeviceInfo** out) {
     cfg.dynamicSmemBytes = awq::dq::SMEM_BYTES;
     AWQ_CUDA(cudaOccupancyMaxActiveClusters(&d.w4_clusters, awq::dq::w4a16_gemm_kernel, &cfg));
     if (d.w4_clusters < 1) return fail(AWQ_ERR_UNSUPPORTED, "the W4A16 GEMM does not fit on this device");
-    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  awq::dec::Shape<16>::SMEM));
-    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  awq::dec::Shape<32>::SMEM));
-    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<48>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  awq::dec::Shape<48>::SMEM));
-    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  awq::dec::Shape<64>::SMEM));
+    // the few-token kernel: shared memory first in the carveout, and the CTAs per SM that really fit
+    {
+      const void* fns[4] = {reinterpret_cast<const void*>(awq::dec::w4a16_decode_kernel<16>),
+                            reinterpret_cast<const void*>(awq::dec::w4a16_decode_kernel<32>),
+                            reinterpret_cast<const void*>(awq::dec::w4a16_decode_kernel<48>),
+                            reinterpret_cast<const void*>(awq::dec::w4a16_decode_kernel<64>)};
+      const int smem[4] = {awq::dec::Shape<16>::SMEM, awq::dec::Shape<32>::SMEM, awq::dec::Shape<48>::SMEM,
+                           awq::dec::Shape<64>::SMEM};
+      for (int i = 0; i < 4; ++i) {
+        AWQ_CUDA(cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, smem[i]));
+        AWQ_CUDA(cudaFuncSetAttribute(fns[i], cudaFuncAttributePreferredSharedMemoryCarveout,
+                                      cudaSharedmemCarveoutMaxShared));
+        AWQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.dec_occ[i], fns[i], awq::dec::THREADS, smem[i]));
+        if (d.dec_occ[i] < 1) return fail(AWQ_ERR_UNSUPPORTED, "the few-token W4A16 GEMM does not fit on this device");
+      }
+    }
     d.gemm_attr_set = true;
   }
   *out = &d;
@@ -829,7 +838,8 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   const int nt = static_cast<int>((M + 15) / 16 * 16);
   const int num_groups = static_cast<int>(K / 128);
   // one wave of CTAs; a slice holds an even number of groups (one code box covers two)
-  int64_t slices = awq::dec::ctas_per_sm(nt) * static_cast<int64_t>(d->sms) / l.n_rb;
+  const int occ = d->dec_occ[nt / 16 - 1];  // CTAs per SM that fit
+  int64_t slices = static_cast<int64_t>(occ) * d->sms / l.n_rb;
   slices = std::max<int64_t>(1, std::min<int64_t>({slices, awq::dec::max_slices(l.n_rb), (num_groups + 1) / 2}));
   const int g_per = static_cast<int>(((num_groups + slices - 1) / slices + 1) / 2 * 2);
   slices = (num_groups + g_per - 1) / g_per;
@@ -846,7 +856,7 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   // dependent.
   const int64_t ctas = l.n_rb * slices;
   const bool prep_in_kernel =
-      ctas <= static_cast<int64_t>(awq::dec::ctas_per_sm(nt)) * d->sms && num_groups <= kW4MaxPrepGroups;
+      ctas <= static_cast<int64_t>(occ) * d->sms && num_groups <= kW4MaxPrepGroups;
   if (!prep_in_kernel) {
     awq::dec::decode_prep_kernel<<<static_cast<unsigned>(num_groups), awq::dec::PREP_THREADS, 0, st>>>(
         static_cast<const uint16_t*>(X), M, K, ldx, nt, xp, sx);

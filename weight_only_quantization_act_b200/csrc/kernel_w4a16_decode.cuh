@@ -77,14 +77,11 @@ struct Shape {
   static constexpr int A_COL0 = ACC_STAGES * NT;
   static constexpr int USED_COLS = A_COL0 + A_BUFS * A_COLS;
   static constexpr uint32_t TMEM_COLS = USED_COLS <= 128 ? 128 : (USED_COLS <= 256 ? 256 : 512);
-  static constexpr int TPT = NT == 16 ? 8 : (NT == 32 ? 4 : 2);         // Sx threads per token
   static constexpr int SMEM = C_STAGES * C_BYTES + X_STAGES * X_BYTES + SX_STAGES * NT * 4 + 1024;
 };
 static_assert(Shape<16>::USED_COLS <= 256 && Shape<16>::SMEM <= 113 * 1024, "two CTAs per SM");
 static_assert(Shape<64>::USED_COLS <= 512, "tensor memory");
 static_assert(Shape<64>::SMEM <= 227 * 1024 && Shape<48>::SMEM <= 227 * 1024, "one CTA per SM");
-
-__host__ inline int ctas_per_sm(int nt) { return nt <= 16 ? 2 : 1; }
 
 // Slices of the groups per row block the workspace is sized for: enough for 512 CTAs, at most
 // MAX_SLICES. The workspace holds partial[n_rb][slices][MAX_NT][ROWS] fp32 and one counter per row block.
