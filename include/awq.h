@@ -272,14 +272,12 @@ AWQ_API awq_status awq_scale_rows(const void *A, int64_t R, int64_t C, int64_t l
  *              (e.g. cudaMemsetAsync once after allocating it). It holds the status word and a tile
  *              counter, a fixed 256 KB region of per-block counters (M <= 64 tokens; every call leaves
  *              them at zero, and nothing else writes there, so one zero fill serves all later calls
- *              whatever their shapes), 128 KB of per-group flags (M <= 64; likewise left at zero), a
- *              group-major copy of steps and zeros (many tokens), and for M <= 64 a permuted copy of X
- *              (64 rows), its per-group sums and split-K partial sums. After a device timeout the
- *              flags and counters may be left set: zero-fill the workspace again before reusing it.
- *              M <= 64 is one cooperative launch when its CTAs fit on the device at once (its CTAs
- *              prepare the X copy and group sums and publish them to each other), else two launches
- *              on `stream`: a small kernel that prepares them and the GEMM as its programmatic
- *              dependent. K <= 2,097,152 for the one-launch form.
+ *              whatever their shapes), a group-major copy of steps and zeros (many tokens), and for
+ *              M <= 64 a permuted copy of X (64 rows), its per-group sums and split-K partial sums.
+ *              After a device timeout the counters may be left set: zero-fill the workspace again
+ *              before reusing it. M <= 64 is two launches on `stream`: a small kernel that writes the
+ *              X copy and group sums, and the GEMM as its programmatic dependent (it starts early and
+ *              waits for them).
  * Requires K % 128 == 0, O % 8 == 0, M >= 1. M <= 64 runs a few-token kernel (weight rows on the MMA's M
  * side, groups split across CTAs, partial sums added in a fixed order). Both are deterministic. A device
  * timeout is reported by awq_search_status() on the same workspace.

@@ -68,11 +68,10 @@ def test_w4a16_matches_oracle(M, K, O):
 
 
 # Few tokens on layers with more 128-row blocks than CTAs fit on the device at once (B200: 296 at 16
-# tokens, 148 above): X' is then prepared by a kernel of its own that the GEMM follows as a programmatic
-# dependent, instead of inside the GEMM's cooperative launch; both paths, run back to back, share the
-# workspace's per-group flags.
+# tokens, 148 above), so the GEMM runs in several waves with one slice per block, next to a layer that
+# fits one wave; run twice on one workspace (the per-block counters are handed back at zero).
 @pytest.mark.parametrize("M,K,O", [(16, 256, 38400), (40, 384, 19200), (16, 256, 512)])
-def test_w4a16_decode_both_preparation_paths(M, K, O):
+def test_w4a16_decode_more_blocks_than_one_wave(M, K, O):
     _, _, (words, steps, zeros) = quantized(O, K, M + K + O + 5)
     Xp = inputs.random_bf16((M, K), 3 * M + 2, scale=1.0)
     lib = awq.load_library()

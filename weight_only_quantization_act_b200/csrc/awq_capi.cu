@@ -799,14 +799,12 @@ extern "C" awq_status awq_scale_rows(const void* A, int64_t R, int64_t C, int64_
 namespace {
 struct W4Layout {
   int64_t O_pad, G, n_rb;
-  size_t steps_off, zeros_off, counter_off, prep_flag_off, xp_off, sx_off, partial_off, bytes;
+  size_t steps_off, zeros_off, counter_off, xp_off, sx_off, partial_off, bytes;
 };
 constexpr int64_t kW4MaxRowBlocks = 65536;  // few-token counters reserved for O up to 8M rows
-constexpr int64_t kW4MaxPrepGroups = 16384;  // in-kernel X' preparation flags for K up to 2M
 // [0, 512) status word and tile counter (cleared by each many-token call); [512, 512 + 256 KB) the
-// few-token kernel's per-row-block counters and then 128 KB of its per-group preparation flags and
-// counts, at the same places for every shape and written by nothing else, so they stay zero from one call
-// to the next whatever the shapes; then the group-major steps and zeros (many tokens), and the few-token
+// few-token kernel's per-row-block counters, at the same place for every shape and written by nothing
+// else, so they stay zero from one call to the next whatever the shapes; then the group-major steps and zeros (many tokens), and the few-token
 // kernel's permuted copy of X' (64 rows), group sums and split-K partial sums.
 W4Layout w4_layout(int64_t K, int64_t O) {
   W4Layout l;
@@ -814,8 +812,7 @@ W4Layout w4_layout(int64_t K, int64_t O) {
   l.G = K / 128;
   l.n_rb = (O + awq::dec::ROWS - 1) / awq::dec::ROWS;
   l.counter_off = 512;
-  l.prep_flag_off = l.counter_off + static_cast<size_t>(kW4MaxRowBlocks) * 4;
-  l.steps_off = l.prep_flag_off + static_cast<size_t>(kW4MaxPrepGroups) * 2 * 4;
+  l.steps_off = l.counter_off + static_cast<size_t>(kW4MaxRowBlocks) * 4;
   l.zeros_off = align_up(l.steps_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
   l.xp_off = align_up(l.zeros_off + static_cast<size_t>(l.G) * l.O_pad * 4, 256);
   l.sx_off = align_up(l.xp_off + static_cast<size_t>(awq::dec::MAX_NT) * K * 2, 256);
@@ -851,17 +848,10 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   CUtensorMap tmX, tmC;
   AWQ_TRY(make_tmap(&tmX, xp, nt, K, K, nt));
   AWQ_TRY(make_tmap_codes_sw128(&tmC, codes, O, K / 8, awq::dec::ROWS));
-  // X' is prepared inside the GEMM (a cooperative launch: its CTAs publish groups to each other) when all
-  // CTAs fit on the device at once, else by a kernel of its own that the GEMM follows as a programmatic
-  // dependent.
   const int64_t ctas = l.n_rb * slices;
-  const bool prep_in_kernel =
-      ctas <= static_cast<int64_t>(occ) * d->sms && num_groups <= kW4MaxPrepGroups;
-  if (!prep_in_kernel) {
-    awq::dec::decode_prep_kernel<<<static_cast<unsigned>(num_groups), awq::dec::PREP_THREADS, 0, st>>>(
-        static_cast<const uint16_t*>(X), M, K, ldx, nt, xp, sx);
-    AWQ_TRY(check_launch("decode_prep_kernel"));
-  }
+  awq::dec::decode_prep_kernel<<<static_cast<unsigned>(num_groups), awq::dec::PREP_THREADS, 0, st>>>(
+      static_cast<const uint16_t*>(X), M, K, ldx, nt, xp, sx);
+  AWQ_TRY(check_launch("decode_prep_kernel"));
   awq::dec::Params p;
   p.steps = steps;
   p.zeros = zeros;
@@ -869,14 +859,6 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   p.partial = reinterpret_cast<float*>(ws + l.partial_off);
   p.counter = reinterpret_cast<unsigned int*>(ws + l.counter_off);
   p.sx = sx;
-  p.X = static_cast<const uint16_t*>(X);
-  p.xp = xp;
-  p.prep_flag = reinterpret_cast<unsigned int*>(ws + l.prep_flag_off);
-  p.prep_count = p.prep_flag + kW4MaxPrepGroups;
-  p.ldx = ldx;
-  p.K = K;
-  p.n_rb = static_cast<int>(l.n_rb);
-  p.prep_in_kernel = prep_in_kernel ? 1 : 0;
   p.M = M;
   p.O = O;
   p.G = l.G;
@@ -891,14 +873,9 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(awq::dec::THREADS);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  if (prep_in_kernel) {
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-  } else {  // its prologue and first code loads overlap the prep kernel
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-  }
+  cudaLaunchAttribute attr[1];  // a programmatic dependent of the prep kernel: its prologue and first code
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // loads overlap it
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (nt == 16) {

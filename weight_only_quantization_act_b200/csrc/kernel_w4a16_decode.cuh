@@ -18,12 +18,10 @@
 // Nibble order. A code word holds in-features 8c .. 8c+7 in nibbles 0..7. One AND-OR per register turns
 // the word shifted right by 4j into the bf16 pair (128 + q_j, 128 + q_{j+4}), so the operand row holds
 // each word's in-features in the order 0 4 1 5 2 6 3 7. X' is permuted the same way inside every 16-byte
-// chunk (8 in-features), which leaves the products and sums unchanged. That permuted copy of X' (nt rows,
-// zero past M) and every Sx_g are prepared once per call instead of by every CTA: when all CTAs fit on the
-// device at once (a cooperative launch), each CTA's epilogue warps prepare a share of its slice's groups
-// first and publish each through a per-group flag, and the loaders wait for a group's flag before loading
-// it; otherwise a small kernel before this one prepares them and this kernel follows it as a programmatic
-// dependent (only the loader waits for it, after requesting its first code boxes).
+// chunk (8 in-features), which leaves the products and sums unchanged. A small kernel before this one
+// writes that permuted copy of X' (nt rows, zero past M) and every Sx_g once, instead of every CTA
+// redoing them; it lets this kernel start early (programmatic dependent launch), and only the loader
+// waits for it, after requesting its first code boxes.
 //
 // CTA (b, c) covers weight rows [128 b, 128 b + 128) and groups [c * gp, (c + 1) * gp) (gp even). The
 // unpacked operand of a group (128 rows x 128 in-features) lives in tensor memory (tcgen05.mma reads A
@@ -94,7 +92,6 @@ enum : unsigned int {
   kSiteDecodeFull = 21,
   kSiteDecodeDequant = 22,
   kSiteDecodeAcc = 23,
-  kSiteDecodePrep = 24,
 };
 
 struct Params {
@@ -103,18 +100,7 @@ struct Params {
   __nv_bfloat16* Y;       // [M][ldy]
   float* partial;         // [n_rb][slices][nt][ROWS]
   unsigned int* counter;  // [n_rb], zero at launch and left zero
-  float* sx;              // [G][nt] group sums of X'
-  // X' preparation inside this kernel (prep_in_kernel = 1, a cooperative launch): CTA (b, c) prepares the
-  // groups g0 + j of its slice with j = b, b + n_rb, ... and publishes each through prep_flag[g]; every
-  // CTA of the slice waits for a group's flag before loading its X' and Sx_g, and the last of them resets
-  // the flag and prep_count[g] to zero. Otherwise decode_prep_kernel ran before this kernel.
-  const uint16_t* X;      // [M][ldx]
-  uint16_t* xp;           // [nt][K]
-  unsigned int* prep_flag;   // [G], zero at launch and left zero
-  unsigned int* prep_count;  // [G], zero at launch and left zero
-  int64_t ldx, K;
-  int n_rb;
-  int prep_in_kernel;
+  const float* sx;        // [G][nt] group sums of X' (decode_prep_kernel)
   int64_t M, O, G, ldy;
   int num_groups;         // K / 128
   int g_per;              // groups per slice, even
@@ -195,18 +181,19 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&v)[4]) {
   v[3] = nibble_pair_bf16(shr_fma(w, 1u << 20));
 }
 
-// X' for the few-token kernel, one group g: Xp[m][k] = X[m][k] for m < M, zero for M <= m < nt, with each
-// 16-byte chunk of 8 in-features in the operand order 0 4 1 5 2 6 3 7; Sx[g][m] = the sum of X[m][k] over
-// the group's 128 in-features (fp32: each chunk's 8 values in increasing k, then the 16 chunk sums in
-// order; zero past M). Done by 128 threads (t = 0..127) that share chunk_sum and the barrier `sync`; every
-// (token, chunk) pair is one 16-byte load, so a group is one memory round trip.
+// X' for the few-token kernel: Xp[m][k] = X[m][k] for m < M, zero for M <= m < nt, with each 16-byte chunk
+// of 8 in-features in the operand order 0 4 1 5 2 6 3 7; Sx[g][m] = the sum of X[m][k] over the group's
+// 128 in-features (fp32: each chunk's 8 values in increasing k, then the 16 chunk sums in order; zero past
+// M). One CTA per group; every (token, chunk) pair is one 16-byte load, so the kernel is one memory round
+// trip long.
 constexpr int PREP_THREADS = 128;
-template <typename Sync>
-__device__ __forceinline__ void prep_group(const uint16_t* __restrict__ X, int64_t M, int64_t K, int64_t ldx, int nt,
-                                           int64_t g, uint16_t* __restrict__ Xp, float* __restrict__ Sx,
-                                           float (*chunk_sum)[GK / 8], int t, Sync sync) {
-  const int64_t k0 = g * GK;
-  for (int task = t; task < nt * (GK / 8); task += PREP_THREADS) {
+__global__ void __launch_bounds__(PREP_THREADS) decode_prep_kernel(const uint16_t* __restrict__ X, int64_t M,
+                                                                   int64_t K, int64_t ldx, int nt,
+                                                                   uint16_t* __restrict__ Xp, float* __restrict__ Sx) {
+  pdl_launch_dependents();
+  __shared__ float chunk_sum[MAX_NT][GK / 8];
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * GK;
+  for (int task = threadIdx.x; task < nt * (GK / 8); task += PREP_THREADS) {
     const int m = task / (GK / 8), ch = task % (GK / 8);
     const uint4 v = m < M ? *reinterpret_cast<const uint4*>(X + m * ldx + k0 + 8 * ch) : make_uint4(0u, 0u, 0u, 0u);
     *reinterpret_cast<uint4*>(Xp + static_cast<int64_t>(m) * K + k0 + 8 * ch) =
@@ -219,24 +206,14 @@ __device__ __forceinline__ void prep_group(const uint16_t* __restrict__ X, int64
       sum = __fadd_rn(__fadd_rn(sum, __uint_as_float(e[k] << 16)), __uint_as_float(e[k] & 0xFFFF0000u));
     chunk_sum[m][ch] = sum;
   }
-  sync();
-  if (t < nt) {
+  __syncthreads();
+  if (threadIdx.x < nt) {
+    const int m = threadIdx.x;
     float sum = 0.0f;
 #pragma unroll
-    for (int ch = 0; ch < GK / 8; ++ch) sum = __fadd_rn(sum, chunk_sum[t][ch]);
-    Sx[g * nt + t] = sum;
+    for (int ch = 0; ch < GK / 8; ++ch) sum = __fadd_rn(sum, chunk_sum[m][ch]);
+    Sx[static_cast<int64_t>(blockIdx.x) * nt + m] = sum;
   }
-  sync();  // chunk_sum may be reused for the next group
-}
-
-// The same as a kernel of its own (one CTA per group), for launches whose CTAs do not all fit on the
-// device at once; the GEMM then follows as its programmatic dependent.
-__global__ void __launch_bounds__(PREP_THREADS) decode_prep_kernel(const uint16_t* __restrict__ X, int64_t M,
-                                                                   int64_t K, int64_t ldx, int nt,
-                                                                   uint16_t* __restrict__ Xp, float* __restrict__ Sx) {
-  pdl_launch_dependents();
-  __shared__ float chunk_sum[MAX_NT][GK / 8];
-  prep_group(X, M, K, ldx, nt, blockIdx.x, Xp, Sx, chunk_sum, static_cast<int>(threadIdx.x), [] { __syncthreads(); });
 }
 
 template <int NT>
@@ -252,7 +229,6 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
   __shared__ uint32_t tmem_slot;
   __shared__ int failed;
   __shared__ unsigned int ticket;
-  __shared__ float prep_sum[NT][GK / 8];  // in-kernel X' preparation (epilogue warps)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -329,29 +305,6 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     const uint32_t use = static_cast<uint32_t>(i / XS), sx_use = static_cast<uint32_t>(i / SX_STAGES);
     if (use > 0 && !wait_warp(xempty_bar(x), (use - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
     if (sx_use > 0 && !wait_warp(sxempty_bar(t), (sx_use - 1u) & 1u, p, kSiteDecodeEmpty)) return false;
-    if (p.prep_in_kernel) {
-      // the group's X' and Sx_g are published by the CTA that prepared them (bounded wait, acquire, then a
-      // proxy fence for the TMA reads); the last CTA of the slice to see the flag hands it back at zero
-      const int64_t g = g0 + i;
-      int have = 1;
-      if (lane == 0) {
-        const uint64_t t0 = global_timer_ns();
-        while (ld_acquire_u32(p.prep_flag + g) == 0u)
-          if (global_timer_ns() - t0 > p.limit_ns) {
-            raise_timeout(p.status, kSiteDecodePrep);
-            have = 0;
-            break;
-          }
-        if (have) {
-          fence_proxy_async_global();
-          if (atomicAdd(p.prep_count + g, 1u) == static_cast<unsigned int>(p.n_rb - 1)) {
-            p.prep_count[g] = 0u;
-            p.prep_flag[g] = 0u;
-          }
-        }
-      }
-      if (!__shfl_sync(0xffffffffu, have, 0)) return false;
-    }
     if (lane == 0) {
       mbar_arrive_expect_tx(xfull_bar(x), S::X_BYTES);
       tma_load_2d(x_tile(x, 0), &tmX, (g0 + i) * GK, 0, xfull_bar(x));
@@ -365,15 +318,13 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
   // The first groups need no free slots: warp 0 requests them right after initialising the barriers, so
   // the first memory round trip overlaps the tensor-memory allocation and the CTA barrier.
   const int pre_c = min(ng, CS * GROUPS_PER_BOX);
-  // (with the preparation in this kernel, X' is loaded only after the CTA barrier, in the main loop: its
-  // producers, the epilogue warps, start after that barrier)
-  const int pre_x = p.prep_in_kernel ? 0 : min(ng, min(XS, SX_STAGES));
+  const int pre_x = min(ng, min(XS, SX_STAGES));
   if (warp == 0) {
     __syncwarp();  // the barriers thread 0 initialised are visible to the whole warp
     // the code boxes first (they do not depend on the kernel before this one), then, once its X' copy
     // and group sums are complete, X' and Sx of the first groups
     for (int i = 0; i < pre_c; i += GROUPS_PER_BOX) load_codes(i);
-    if (!p.prep_in_kernel) pdl_wait();
+    pdl_wait();
     for (int i = 0; i < pre_x; ++i) load_x(i);
   }
   if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), S::TMEM_COLS);
@@ -474,18 +425,6 @@ __global__ void __launch_bounds__(THREADS, Shape<NT>::CTAS_PER_SM)
     }
   } else {
     // ------------------------------------------------------------------------------ group epilogue
-    if (p.prep_in_kernel) {
-      // first this CTA's share of the slice's X' preparation: groups g0 + j, j = rb, rb + n_rb, ...
-      const int et = static_cast<int>(threadIdx.x) - 32 * EPI_WARP0;
-      for (int j = rb; j < ng; j += p.n_rb) {
-        prep_group(p.X, p.M, p.K, p.ldx, NT, static_cast<int64_t>(g0 + j), p.xp, p.sx, prep_sum, et,
-                   [] { epilogue_sync(); });
-        fence_proxy_async_global();  // the generic-proxy writes, for the other CTAs' TMA reads
-        __threadfence();
-        epilogue_sync();
-        if (et == 0) atomicExch(p.prep_flag + g0 + j, 1u);
-      }
-    }
     const int q = warp & 3;  // tensor-memory lane quarter this warp may read
     const int r = 32 * q + lane;
     const uint32_t tlane = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
