@@ -50,7 +50,6 @@ struct DeviceInfo {
   bool gemm_attr_set = false;
   int gemm_clusters = 0;  // CTA pairs of the loss GEMM that fit on the device at once
   int w4_clusters = 0;    // CTA pairs of the W4A16 GEMM that fit on the device at once
-  int dec_occ[4] = {0, 0, 0, 0};  // few-token GEMM CTAs per SM for 16, 32, 48, 64 tokens
 };
 
 constexpr int kMaxDevices = 64;
@@ -136,22 +135,14 @@ awq_status device_info(DeviceInfo** out) {
     cfg.dynamicSmemBytes = awq::dq::SMEM_BYTES;
     AWQ_CUDA(cudaOccupancyMaxActiveClusters(&d.w4_clusters, awq::dq::w4a16_gemm_kernel, &cfg));
     if (d.w4_clusters < 1) return fail(AWQ_ERR_UNSUPPORTED, "the W4A16 GEMM does not fit on this device");
-    // the few-token kernel: shared memory first in the carveout, and the CTAs per SM that really fit
-    {
-      const void* fns[4] = {reinterpret_cast<const void*>(awq::dec::w4a16_decode_kernel<16>),
-                            reinterpret_cast<const void*>(awq::dec::w4a16_decode_kernel<32>),
-                            reinterpret_cast<const void*>(awq::dec::w4a16_decode_kernel<48>),
-                            reinterpret_cast<const void*>(awq::dec::w4a16_decode_kernel<64>)};
-      const int smem[4] = {awq::dec::Shape<16>::SMEM, awq::dec::Shape<32>::SMEM, awq::dec::Shape<48>::SMEM,
-                           awq::dec::Shape<64>::SMEM};
-      for (int i = 0; i < 4; ++i) {
-        AWQ_CUDA(cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, smem[i]));
-        AWQ_CUDA(cudaFuncSetAttribute(fns[i], cudaFuncAttributePreferredSharedMemoryCarveout,
-                                      cudaSharedmemCarveoutMaxShared));
-        AWQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.dec_occ[i], fns[i], awq::dec::THREADS, smem[i]));
-        if (d.dec_occ[i] < 1) return fail(AWQ_ERR_UNSUPPORTED, "the few-token W4A16 GEMM does not fit on this device");
-      }
-    }
+    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::dec::Shape<16>::SMEM));
+    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::dec::Shape<32>::SMEM));
+    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<48>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::dec::Shape<48>::SMEM));
+    AWQ_CUDA(cudaFuncSetAttribute(awq::dec::w4a16_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  awq::dec::Shape<64>::SMEM));
     d.gemm_attr_set = true;
   }
   *out = &d;
@@ -804,8 +795,9 @@ struct W4Layout {
 constexpr int64_t kW4MaxRowBlocks = 65536;  // few-token counters reserved for O up to 8M rows
 // [0, 512) status word and tile counter (cleared by each many-token call); [512, 512 + 256 KB) the
 // few-token kernel's per-row-block counters, at the same place for every shape and written by nothing
-// else, so they stay zero from one call to the next whatever the shapes; then the group-major steps and zeros (many tokens), and the few-token
-// kernel's permuted copy of X' (64 rows), group sums and split-K partial sums.
+// else, so they stay zero from one call to the next whatever the shapes; then the group-major steps and
+// zeros (many tokens), and the few-token kernel's permuted copy of X' (64 rows), group sums and split-K
+// partial sums.
 W4Layout w4_layout(int64_t K, int64_t O) {
   W4Layout l;
   l.O_pad = (O + awq::lg::BN - 1) / awq::lg::BN * awq::lg::BN;
@@ -835,8 +827,11 @@ awq_status w4a16_decode(const void* X, int64_t M, int64_t K, int64_t ldx, const 
   const int nt = static_cast<int>((M + 15) / 16 * 16);
   const int num_groups = static_cast<int>(K / 128);
   // one wave of CTAs; a slice holds an even number of groups (one code box covers two)
-  const int occ = d->dec_occ[nt / 16 - 1];  // CTAs per SM that fit
-  int64_t slices = static_cast<int64_t>(occ) * d->sms / l.n_rb;
+  // Slices sized for two CTAs per SM at 16 tokens and one above. (At the default shared-memory carveout a
+  // cooperative launch of that many 16-token CTAs was refused as too large for one wave; preferring shared
+  // memory in the carveout let them all fit, and the 16 x 28672 -> 8192 layer then ran slower, 74 against
+  // 56 us.)
+  int64_t slices = static_cast<int64_t>(nt <= 16 ? 2 : 1) * d->sms / l.n_rb;
   slices = std::max<int64_t>(1, std::min<int64_t>({slices, awq::dec::max_slices(l.n_rb), (num_groups + 1) / 2}));
   const int g_per = static_cast<int>(((num_groups + slices - 1) / slices + 1) / 2 * 2);
   slices = (num_groups + g_per - 1) / g_per;
