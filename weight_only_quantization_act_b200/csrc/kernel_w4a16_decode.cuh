@@ -156,9 +156,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
   return v;
 }
-__device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
 
 // (128 + q) as bf16 pairs from a code word: register j holds the nibbles j and j + 4 (in-features 8c + j and
 // 8c + j + 4 of word c) in its low and high half, 0x4300 | q each. The word shifted right by 4 j (a

@@ -1,8 +1,8 @@
 // ptx.cuh - thin inline-PTX wrappers for the sm_100a features the tensor-core kernels use: mbarriers
-// with bounded waits (local and cluster-scope), TMA tile loads (no multicast) and stores,
-// tensor-memory allocation for one CTA or a CTA pair, tcgen05.mma kind::f16 issued for one CTA
-// (cta_group::1) or a CTA pair (cta_group::2) with its commits, and tcgen05.ld of the fp32
-// accumulator.
+// with bounded waits (local and cluster-scope), TMA tile loads (no multicast), bulk copies and stores,
+// programmatic dependent launch, tensor-memory allocation for one CTA or a CTA pair, tcgen05.mma
+// kind::f16 issued for one CTA (A from tensor memory) or a CTA pair (cta_group::2) with its commits, and
+// tcgen05.ld / tcgen05.st of tensor memory.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -211,16 +211,8 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 }
 
 // Tile load of one CTA of a CTA pair whose MMA is issued by the pair's even CTA: the bytes land in this
-// CTA's shared memory and are counted on `bar`, which may be the even CTA's barrier. No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t c0, int32_t c1,
-                                                 uint32_t bar_cluster) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster)
-      : "memory");
-}
-
+// CTA's shared memory and are counted on `bar_cluster`, which may be the even CTA's barrier; L2 policy
+// from createpolicy. No multicast.
 __device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap* map, int32_t c0, int32_t c1,
                                                       uint32_t bar_cluster, uint64_t policy) {
   asm volatile(
@@ -307,16 +299,6 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t cta_mask
       : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32, shapes from the instruction descriptor.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // D[tmem] (+)= A[tmem] * B[smem]^T, bf16 x bf16 -> fp32: A read from tensor memory (row i of A in lane
 // i, two consecutive K elements per 32-bit column, so one K = 16 step spans 8 columns).
 __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
@@ -339,12 +321,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
       "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
-}
-// 8 consecutive 32-bit columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -402,27 +378,6 @@ __device__ __forceinline__ void bulk_wait_read() {
 }
 // Wait until every bulk group of this thread has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-// ------------------------------------------------------------------------------------ cp.async
-// 4-byte asynchronous copy global -> shared (this CTA).
-__device__ __forceinline__ void cp_async_4(uint32_t dst_smem, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst_smem), "l"(src) : "memory");
-}
-// 8-byte asynchronous copy global -> shared (both addresses 8-byte aligned).
-__device__ __forceinline__ void cp_async_8(uint32_t dst_smem, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst_smem), "l"(src) : "memory");
-}
-// One arrival on `bar` once every cp.async this thread issued so far has landed (the arrival is one of
-// the barrier's expected arrivals: .noinc).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
-  return v;
-}
 
 // Shared-memory matrix descriptor for a K-major bf16 tile written by TMA with 128-byte swizzle: rows
 // of 64 elements (128 B) stored back to back, 8-row swizzle atoms of 1024 B. Fields: start address
